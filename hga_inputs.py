@@ -1,0 +1,142 @@
+"""Seeded synthetic inputs for one routed-HGA attention layer.
+
+This module only draws random numbers and plants structure (per-chunk key
+offsets, needle groups).  It holds none of the method's arithmetic, so both the
+CUDA path and the CPU oracle can be fed from it without sharing code.
+
+Workloads (shapes of the Qwen3-8B attention layer: 32 query heads, 8 KV heads,
+head dim 128; chunk 64, group 8, query block 64 as in "Long-Context
+Fine-Tuning with Limited VRAM", pith.science free-parameter ledger and
+Figure 1 caption; segment 2048 tokens as the TBPTT segment length there):
+
+* ``tiny_f32``   1 x (4 q / 1 kv) heads, 1024 history + 256 segment tokens,
+                 top-4 chunks / top-8 groups, float32, chunk offsets of scale 1.
+* ``ctx4k``      4096 context = 2048 history + 2048 segment, top-16 / top-64, bf16.
+* ``ctx16k``     16384 context = 14336 history + 2048 segment, top-16 / top-64, bf16.
+* ``ctx131k``    131072 context = 129024 history + 2048 segment, top-32 / top-128,
+                 bf16, forward only, 64 planted needle groups.
+* ``ctx16k_b4``  the 16K layer at batch 4 (tiered-history workload shape).
+
+Value distributions: Q, V, dO ~ N(0, 1); K = N(0, 1) + s * o_c where o_c ~ N(0, I)
+is one offset per (batch, KV head, 64-token chunk) of the context (history
+and segment alike) and s is the workload's offset scale.  Tensors are drawn in
+float32 on the CPU from a ``torch.Generator`` seeded with ``seed`` and then
+rounded (round-to-nearest-even) to the workload dtype, so every consumer sees
+identical values.
+
+Needles: for each of ``needles`` distinct (KV head, query block) targets a
+random unit direction u is drawn; ``needle_q`` * u is added to every query of
+the target block in the KV head's query heads, and ``needle_k`` * u to the 8
+keys of one randomly chosen history group (distinct groups).
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    hist_len: int
+    seg_len: int
+    top_chunks: int
+    top_groups: int
+    dtype: str                 # "f32" | "bf16"
+    offset_scale: float
+    chunk: int = 64
+    group: int = 8
+    qblock: int = 64
+    backward: bool = True
+    needles: int = 0
+    needle_q: float = 1.0
+    needle_k: float = 32.0
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def nblk(self) -> int:
+        return self.seg_len // self.qblock
+
+    @property
+    def nch(self) -> int:
+        return self.hist_len // self.chunk
+
+    @property
+    def ngr(self) -> int:
+        return self.hist_len // self.group
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny_f32": Workload("tiny_f32", 1, 4, 1, 128, 1024, 256, 4, 8, "f32", 1.0),
+    "ctx4k": Workload("ctx4k", 1, 32, 8, 128, 2048, 2048, 16, 64, "bf16", 0.5),
+    "ctx16k": Workload("ctx16k", 1, 32, 8, 128, 14336, 2048, 16, 64, "bf16", 0.5),
+    "ctx131k": Workload("ctx131k", 1, 32, 8, 128, 129024, 2048, 32, 128, "bf16", 0.5,
+                        backward=False, needles=64),
+    "ctx16k_b4": Workload("ctx16k_b4", 4, 32, 8, 128, 14336, 2048, 16, 64, "bf16", 0.5),
+}
+
+
+def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu") -> dict:
+    """Draw q [B,Hq,S,D], k_hist/v_hist [B,Hkv,H,D], k_seg/v_seg [B,Hkv,S,D], d_o [B,Hq,S,D].
+
+    Returns a dict of tensors (dtype ``w.torch_dtype``) plus ``needles``: a long tensor
+    [n, 3] of (kv head, query block, history group) for planted needles (batch 0)."""
+    g = torch.Generator().manual_seed(int(seed))
+    B, Hq, Hkv, D, H, S = w.B, w.Hq, w.Hkv, w.D, w.hist_len, w.seg_len
+    C = w.chunk
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+    q = normal(B, Hq, S, D)
+    # one offset per (b, kv head, chunk) of the whole context [history | segment]
+    n_ctx_chunks = (H + S + C - 1) // C
+    offs = normal(B, Hkv, n_ctx_chunks, D) * w.offset_scale
+    per_tok = offs.repeat_interleave(C, dim=2)[:, :, : H + S]
+    k_hist = normal(B, Hkv, H, D) + per_tok[:, :, :H]
+    k_seg = normal(B, Hkv, S, D) + per_tok[:, :, H:]
+    v_hist = normal(B, Hkv, H, D)
+    v_seg = normal(B, Hkv, S, D)
+    d_o = normal(B, Hq, S, D)
+
+    needles = torch.zeros(0, 3, dtype=torch.long)
+    if w.needles:
+        G = Hq // Hkv
+        n = w.needles
+        targets = torch.randperm(Hkv * w.nblk, generator=g)[:n]
+        groups = torch.randperm(w.ngr, generator=g)[:n]
+        dirs = normal(n, D)
+        dirs = dirs / dirs.norm(dim=1, keepdim=True)
+        rows = []
+        for i in range(n):
+            kh, blk = int(targets[i]) // w.nblk, int(targets[i]) % w.nblk
+            j = int(groups[i])
+            q[0, kh * G:(kh + 1) * G, blk * w.qblock:(blk + 1) * w.qblock] += w.needle_q * dirs[i]
+            k_hist[0, kh, j * w.group:(j + 1) * w.group] += w.needle_k * dirs[i]
+            rows.append((kh, blk, j))
+        needles = torch.tensor(rows, dtype=torch.long)
+
+    dt = w.torch_dtype
+    out = dict(q=q, k_hist=k_hist, v_hist=v_hist, k_seg=k_seg, v_seg=v_seg, d_o=d_o)
+    out = {k: v.to(dt).contiguous().to(device) for k, v in out.items()}
+    out["needles"] = needles
+    return out
+
+
+def sample_ids(n_total: int, n: int, seed: int) -> torch.Tensor:
+    """``n`` distinct ids in [0, n_total), sorted, from a seeded generator (for sampled checks)."""
+    g = torch.Generator().manual_seed(int(seed) + 7919)
+    n = min(n, n_total)
+    return torch.randperm(n_total, generator=g)[:n].sort().values
