@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-HGA hot path: one Qwen3-8B-shaped attention layer at 16K context.
+
+Workload (default ``ctx16k``): batch 1, 32 query / 8 KV heads, head dim 128, bf16 with fp32
+accumulation; 14336 detached history tokens + 2048 active-segment tokens; chunk 64, group 8,
+query block 64; top-16 chunks then top-64 groups (512 routed tokens per block).  One step =
+the whole hot path on synthetic inputs already in HBM: key summaries, routing, forward,
+backward (6 kernel launches).  Metric: active-segment tokens per second, forward + backward.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own layer (different seed):
+the KV heads / batches of the method are independent, so there is no collective in the data
+path ("scaling": "weak"); the timed region is bracketed by barriers and the step time is
+the max over ranks.  ``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import hga_inputs as HI  # noqa: E402
+
+METRIC = "routed HGA attn tokens/sec fwd+bwd per layer at 16K ctx; % of HBM/tensor roofline"
+L2_FLUSH_BYTES = 512 << 20          # > 126 MB L2: written between timed steps
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def work_model(w) -> dict:
+    """Algorithmic work of each kernel of one step (bytes or flops per launch)."""
+    B, Hq, Hkv, D, H, S = w.B, w.Hq, w.Hkv, w.D, w.hist_len, w.seg_len
+    esz = 2 if w.dtype == "bf16" else 4
+    routed_pairs = B * Hq * S * 8 * w.top_groups            # (query, routed key) pairs
+    local_pairs = B * Hq * S * (S + 1) // 2                 # causal (query, segment key) pairs
+    nch, ngr, nblk = H // 64, H // 8, S // 64
+    return {
+        "summaries": ("hbm", B * Hkv * H * D * esz + B * Hkv * (ngr + nch) * D * 4),
+        "route": ("hbm", B * Hq * S * D * esz + B * Hkv * (nch + ngr) * D * 4
+                  + B * Hkv * nblk * (w.top_chunks + w.top_groups) * 4),
+        "attn_fwd": ("tensor", 4 * D * (routed_pairs + local_pairs)),
+        "bwd_preprocess": ("hbm", 2 * B * Hq * S * D * esz + B * Hq * S * 4),
+        "bwd_dkdv": ("tensor", 8 * D * local_pairs),
+        "bwd_dq": ("tensor", 6 * D * (routed_pairs + local_pairs)),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="hga_clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [c.strip() for c in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+            os.unlink(self.path)
+        except OSError:
+            return None
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def all_max(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_slice_pass(w, x) -> float:
+    """The CPU oracle over KV head 0 of batch 0 (its G query heads, every block): summaries,
+    routing, forward and backward.  Returns seconds."""
+    from oracle import oracle as O
+    G = w.Hq // w.Hkv
+    s = {k: (v[:1, :G] if k in ("q", "d_o") else v[:1, :1]) for k, v in x.items() if k != "needles"}
+    t0 = time.perf_counter()
+    r = O.route_from_inputs(s["q"], s["k_hist"], 1, w.top_chunks, w.top_groups, prec=32)
+    O.attn_fwd(s["q"], s["k_hist"], s["v_hist"], s["k_seg"], s["v_seg"], r["group_idx"])
+    O.attn_bwd(s["q"], s["k_hist"], s["v_hist"], s["k_seg"], s["v_seg"], r["group_idx"], s["d_o"])
+    return time.perf_counter() - t0
+
+
+ORACLE_SAMPLE = ("one (batch, KV head) slice of the layer -- its 4 query heads over all 32 query blocks: "
+                 "summaries, routing, forward and backward in the float64 C oracle on one host thread; "
+                 "the layer is B*Hkv such independent slices of equal work, so tokens/s = B*S / (B*Hkv * t_slice)")
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    x = HI.make_inputs(w, args.seed)
+    for _ in range(args.warmup):
+        oracle_slice_pass(w, x)
+    ts = [oracle_slice_pass(w, x) for _ in range(args.steps)]
+    t_step = statistics.mean(ts) * w.B * w.Hkv           # the whole layer
+    value = w.B * w.seg_len / t_step
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": _config(w, args), "gpu_launches": 0,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": ORACLE_SAMPLE},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, args):
+    return {"workload": f"{w.name}: routed HGA layer, B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, "
+                        f"history={w.hist_len}, segment={w.seg_len}, chunk=64, group=8, qblock=64, "
+                        f"top_chunks={w.top_chunks}, top_groups={w.top_groups}, {w.dtype}",
+            "global_batch": w.B * args.gpus, "seq_len": w.hist_len + w.seg_len, "active_segment": w.seg_len,
+            "parallelism": f"independent layer per GPU x{args.gpus}",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
+    ap.add_argument("--workload", default="ctx16k", choices=sorted(HI.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = HI.WORKLOADS[args.workload]
+    world, rank, local = dist_setup()
+    if args.gpus != world and world > 1:
+        args.gpus = world
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import hierarchical_kv_routing_tok_b200 as H
+    from hierarchical_kv_routing_tok_b200 import _capi as C
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x_cpu = HI.make_inputs(w, args.seed + rank)
+    x = {k: v.to(dev) for k, v in x_cpu.items() if k != "needles"}
+    cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    step = H.LayerStep(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+    calls = step.calls(x, stream.cuda_stream)
+    names = [n for n, _ in calls]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(max(args.warmup, 3)):
+        for _, c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    if H.read_status(step.ws) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            for j, (_, c) in enumerate(calls):
+                c()
+                ev[i][j + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(K)]
+    kern_ms = {n: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)] for j, n in enumerate(names)}
+    t_step = all_max(sum(step_ms) / K, world, dev) * 1e-3
+    tokens = w.B * w.seg_len * world
+    value = tokens / t_step
+    if H.read_status(step.ws) != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    # roofline of the dominant kernel
+    wm = work_model(w)
+    pk = _peaks()
+    dom = max(names, key=lambda n: sum(kern_ms[n]))
+    avg_s = sum(kern_ms[dom]) / K * 1e-3
+    bound, work = wm[dom]
+    if bound == "tensor":
+        achieved, peak, unit = work / avg_s / 1e12, pk["bf16"], "TFLOP/s"
+    else:
+        achieved, peak, unit = work / avg_s / 1e9, pk["hbm"], "GB/s"
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            tr = json.load(f).get(f"{w.name}:{dom}")
+        if tr and tr.get("kernel_source_sha") == _kernel_sha():
+            traffic = tr["dram_bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic, "kernel": dom, "peak_source": f"{pk['src']} (burst)",
+                "per_kernel_us": {n: 1e3 * sum(v) / K for n, v in kern_ms.items()},
+                "per_kernel_frac": {n: (wm[n][1] / (sum(kern_ms[n]) / K * 1e-3)
+                                        / ((pk["bf16"] * 1e12) if wm[n][0] == "tensor" else (pk["hbm"] * 1e9)))
+                                    for n in names}}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        in_names = ["q", "k_hist", "v_hist", "k_seg", "v_seg", "d_o"]
+        host_in = {k: x_cpu[k].pin_memory() for k in in_names}
+        outs = [step.o, step.dq, step.dk, step.dv]
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        K2 = max(3, min(K, 10))
+
+        def e2e_step():
+            for k in in_names:
+                x[k].copy_(host_in[k], non_blocking=True)
+            for _, c in calls:
+                c()
+            for d, h in zip(outs, host_out):
+                h.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K2):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        t_e2e = all_max(e0.elapsed_time(e1) / K2, world, dev) * 1e-3
+        e2e = {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": t_e2e * 1e3}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_slice = oracle_slice_pass(w, x_cpu)
+        cpu = {"value": w.B * w.seg_len / (t_slice * w.B * w.Hkv), "unit": "tokens/s", "cores": 1,
+               "kind": "oracle", "sample": ORACLE_SAMPLE, "slice_seconds": t_slice}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": _config(w, args), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": K * len(calls), "clocks": clk.summary(),
+                "kernels_per_step": names}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def _kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_kv_routing_tok_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

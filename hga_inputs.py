@@ -140,3 +140,23 @@ def sample_ids(n_total: int, n: int, seed: int) -> torch.Tensor:
     g = torch.Generator().manual_seed(int(seed) + 7919)
     n = min(n, n_total)
     return torch.randperm(n_total, generator=g)[:n].sort().values
+
+
+# Small and edge-case shapes used by the parity tests (all fit the oracle in seconds).
+WORKLOADS["small_bf16"] = Workload("small_bf16", 2, 8, 2, 128, 1024, 512, 4, 16, "bf16", 0.5)
+
+EDGE_WORKLOADS = {
+    # a single history chunk, a single query block, budget of one chunk / one group
+    "one_chunk_f32": WORKLOADS["tiny_f32"].with_(name="one_chunk_f32", hist_len=64, seg_len=64,
+                                                 top_chunks=1, top_groups=1),
+    # 5 groups = 40 routed keys: a ragged routed tile
+    "ragged_groups_f32": WORKLOADS["tiny_f32"].with_(name="ragged_groups_f32", top_groups=5),
+    # one query head per KV head, batch 2, 9 groups (72 routed keys), bf16
+    "gqa1_b2_bf16": Workload("gqa1_b2_bf16", 2, 2, 2, 128, 512, 128, 2, 9, "bf16", 1.0),
+    # eight query heads per KV head, budget covering the whole history (dense equivalence)
+    "gqa8_dense_f32": Workload("gqa8_dense_f32", 1, 8, 1, 128, 256, 192, 4, 32, "f32", 1.0),
+    # tiny layer with every chunk and group selected (dense equivalence)
+    "dense_tiny_f32": WORKLOADS["tiny_f32"].with_(name="dense_tiny_f32", top_chunks=16, top_groups=128),
+    # maximal group budget for the chosen chunks (k_g = 8 k_c), bf16
+    "max_groups_bf16": WORKLOADS["small_bf16"].with_(name="max_groups_bf16", B=1, top_groups=32),
+}

@@ -1,0 +1,228 @@
+"""PyTorch-facing wrapper of the routed-HGA C ABI.
+
+PyTorch provides device memory and the current CUDA stream; every computation
+runs in ``libhga.so``.  Tensors must be CUDA, contiguous, in the layouts of
+``include/hga.h``: q/o/d_o/dq ``[B, Hq, S, D]``, history K/V ``[B, Hkv, H, D]``,
+segment K/V and their gradients ``[B, Hkv, S, D]``.
+
+Method: "Long-Context Fine-Tuning with Limited VRAM" (gist.science Technical
+Summary 2.1-2.2; pith.science review Figures 1-2).  Routing runs without
+gradient; the history K/V are detached; only q and the active segment get
+gradients.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _capi as C
+
+_DT = {torch.float32: C.HGA_F32, torch.bfloat16: C.HGA_BF16}
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def make_config(q: torch.Tensor, k_hist: torch.Tensor, top_chunks: int, top_groups: int,
+                softmax_scale: float | None = None) -> C.HGAConfig:
+    """Configuration from q [B,Hq,S,D] and k_hist [B,Hkv,H,D]."""
+    if q.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    B, Hq, S, D = q.shape
+    Hkv, H = k_hist.shape[1], k_hist.shape[2]
+    return C.make_config(B, Hq, Hkv, H, S, top_chunks, top_groups, dtype=_DT[q.dtype], D=D,
+                         softmax_scale=float(softmax_scale or 0.0))
+
+
+def _tdtype(cfg) -> torch.dtype:
+    return torch.bfloat16 if cfg.dtype == C.HGA_BF16 else torch.float32
+
+
+def new_workspace(cfg, device) -> torch.Tensor:
+    """Zero-initialised workspace (the leading status word must start at 0)."""
+    return torch.zeros(C.workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def build_summaries(cfg, k_hist, group_sum=None, chunk_sum=None, workspace=None):
+    B, Hkv, H, D = cfg.B, cfg.Hkv, cfg.hist_len, cfg.D
+    _need(k_hist, "k_hist", (B, Hkv, H, D), _tdtype(cfg))
+    dev = k_hist.device
+    if group_sum is None:
+        group_sum = torch.empty(B, Hkv, H // cfg.group, D, dtype=torch.float32, device=dev)
+    if chunk_sum is None:
+        chunk_sum = torch.empty(B, Hkv, H // cfg.chunk, D, dtype=torch.float32, device=dev)
+    _need(group_sum, "group_sum", (B, Hkv, H // cfg.group, D), torch.float32)
+    _need(chunk_sum, "chunk_sum", (B, Hkv, H // cfg.chunk, D), torch.float32)
+    C.build_summaries(cfg, k_hist.data_ptr(), group_sum.data_ptr(), chunk_sum.data_ptr(),
+                      workspace.data_ptr() if workspace is not None else None, _stream(k_hist))
+    return group_sum, chunk_sum
+
+
+def route(cfg, q, group_sum, chunk_sum, chunk_idx=None, group_idx=None, workspace=None):
+    B, Hq, Hkv, S, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.D
+    nblk = S // cfg.qblock
+    _need(q, "q", (B, Hq, S, D), _tdtype(cfg))
+    dev = q.device
+    if chunk_idx is None:
+        chunk_idx = torch.empty(B, Hkv, nblk, cfg.top_chunks, dtype=torch.int32, device=dev)
+    if group_idx is None:
+        group_idx = torch.empty(B, Hkv, nblk, cfg.top_groups, dtype=torch.int32, device=dev)
+    _need(group_sum, "group_sum", (B, Hkv, cfg.hist_len // cfg.group, D), torch.float32)
+    _need(chunk_sum, "chunk_sum", (B, Hkv, cfg.hist_len // cfg.chunk, D), torch.float32)
+    _need(chunk_idx, "chunk_idx", (B, Hkv, nblk, cfg.top_chunks), torch.int32)
+    _need(group_idx, "group_idx", (B, Hkv, nblk, cfg.top_groups), torch.int32)
+    C.route(cfg, q.data_ptr(), group_sum.data_ptr(), chunk_sum.data_ptr(), chunk_idx.data_ptr(),
+            group_idx.data_ptr(), workspace.data_ptr() if workspace is not None else None, _stream(q))
+    return chunk_idx, group_idx
+
+
+def _check_layer(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx):
+    B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
+    dt = _tdtype(cfg)
+    _need(q, "q", (B, Hq, S, D), dt)
+    _need(k_hist, "k_hist", (B, Hkv, H, D), dt)
+    _need(v_hist, "v_hist", (B, Hkv, H, D), dt)
+    _need(k_seg, "k_seg", (B, Hkv, S, D), dt)
+    _need(v_seg, "v_seg", (B, Hkv, S, D), dt)
+    _need(group_idx, "group_idx", (B, Hkv, S // cfg.qblock, cfg.top_groups), torch.int32)
+
+
+def attn_fwd(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o=None, lse=None, workspace=None):
+    _check_layer(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(cfg.B, cfg.Hq, cfg.seg_len, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(cfg, q.device)
+    _need(o, "o", q.shape, q.dtype)
+    _need(lse, "lse", (cfg.B, cfg.Hq, cfg.seg_len), torch.float32)
+    C.attn_fwd(cfg, q.data_ptr(), k_hist.data_ptr(), v_hist.data_ptr(), k_seg.data_ptr(), v_seg.data_ptr(),
+               group_idx.data_ptr(), o.data_ptr(), lse.data_ptr(), workspace.data_ptr(), _stream(q))
+    return o, lse
+
+
+def attn_bwd(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq=None, dk_seg=None, dv_seg=None,
+             workspace=None):
+    _check_layer(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx)
+    _need(o, "o", q.shape, q.dtype)
+    _need(d_o, "d_o", q.shape, q.dtype)
+    _need(lse, "lse", (cfg.B, cfg.Hq, cfg.seg_len), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk_seg = torch.empty_like(k_seg) if dk_seg is None else dk_seg
+    dv_seg = torch.empty_like(v_seg) if dv_seg is None else dv_seg
+    _need(dq, "dq", q.shape, q.dtype)
+    _need(dk_seg, "dk_seg", k_seg.shape, k_seg.dtype)
+    _need(dv_seg, "dv_seg", v_seg.shape, v_seg.dtype)
+    if workspace is None:
+        workspace = new_workspace(cfg, q.device)
+    C.attn_bwd(cfg, q.data_ptr(), k_hist.data_ptr(), v_hist.data_ptr(), k_seg.data_ptr(), v_seg.data_ptr(),
+               group_idx.data_ptr(), o.data_ptr(), lse.data_ptr(), d_o.data_ptr(), dq.data_ptr(),
+               dk_seg.data_ptr(), dv_seg.data_ptr(), workspace.data_ptr(), _stream(q))
+    return dq, dk_seg, dv_seg
+
+
+def read_status(workspace: torch.Tensor) -> int:
+    return C.read_status(workspace.data_ptr(), _stream(workspace))
+
+
+class _HGAFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k_seg, v_seg, k_hist, v_hist, top_chunks, top_groups, softmax_scale):
+        cfg = make_config(q, k_hist, top_chunks, top_groups, softmax_scale)
+        ws = new_workspace(cfg, q.device)
+        with torch.no_grad():                       # routing carries no gradient
+            gs, cs = build_summaries(cfg, k_hist, workspace=ws)
+            _, gi = route(cfg, q, gs, cs, workspace=ws)
+        o, lse = attn_fwd(cfg, q, k_hist, v_hist, k_seg, v_seg, gi, workspace=ws)
+        ctx.cfg = cfg
+        ctx.save_for_backward(q, k_seg, v_seg, k_hist, v_hist, gi, o, lse, ws)
+        ctx.mark_non_differentiable(lse, gi)
+        return o, lse, gi
+
+    @staticmethod
+    def backward(ctx, d_o, _dlse, _dgi):
+        q, k_seg, v_seg, k_hist, v_hist, gi, o, lse, ws = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(ctx.cfg, q, k_hist, v_hist, k_seg, v_seg, gi, o, lse, d_o.contiguous(),
+                              workspace=ws)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def hga_attention(q, k_seg, v_seg, k_hist, v_hist, top_chunks: int, top_groups: int,
+                  softmax_scale: float | None = None):
+    """Routed HGA attention of the active segment.  Returns (o, lse, group_idx).
+
+    Differentiable in q, k_seg, v_seg; k_hist / v_hist are treated as detached history."""
+    return _HGAFunction.apply(q, k_seg, v_seg, k_hist.detach(), v_hist.detach(), top_chunks, top_groups,
+                              softmax_scale)
+
+
+class LayerStep:
+    """One full pass of the hot path (summaries, routing, forward, backward) over preallocated
+    buffers, for a fixed configuration.  Used by the benchmark and the smoke check."""
+
+    def __init__(self, cfg, device="cuda"):
+        self.cfg = cfg
+        dev = torch.device(device)
+        B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
+        dt = _tdtype(cfg)
+        nblk = S // cfg.qblock
+        self.ws = new_workspace(cfg, dev)
+        self.group_sum = torch.empty(B, Hkv, H // cfg.group, D, dtype=torch.float32, device=dev)
+        self.chunk_sum = torch.empty(B, Hkv, H // cfg.chunk, D, dtype=torch.float32, device=dev)
+        self.chunk_idx = torch.empty(B, Hkv, nblk, cfg.top_chunks, dtype=torch.int32, device=dev)
+        self.group_idx = torch.empty(B, Hkv, nblk, cfg.top_groups, dtype=torch.int32, device=dev)
+        self.o = torch.empty(B, Hq, S, D, dtype=dt, device=dev)
+        self.lse = torch.empty(B, Hq, S, dtype=torch.float32, device=dev)
+        self.dq = torch.empty(B, Hq, S, D, dtype=dt, device=dev)
+        self.dk = torch.empty(B, Hkv, S, D, dtype=dt, device=dev)
+        self.dv = torch.empty(B, Hkv, S, D, dtype=dt, device=dev)
+
+    def calls(self, x: dict, stream: int | None = None):
+        """The step as a list of (kernel name, zero-argument C-ABI call), one kernel each, in order.
+        Pointers are bound once so the timed loop does no tensor bookkeeping."""
+        cfg, ws = self.cfg, self.ws.data_ptr()
+        st = torch.cuda.current_stream(self.o.device).cuda_stream if stream is None else stream
+        p = {k: v.data_ptr() for k, v in x.items() if isinstance(v, torch.Tensor) and v.is_cuda}
+        gs, cs, ci, gi = (t.data_ptr() for t in (self.group_sum, self.chunk_sum, self.chunk_idx, self.group_idx))
+        o, lse, dq, dk, dv = (t.data_ptr() for t in (self.o, self.lse, self.dq, self.dk, self.dv))
+        return [
+            ("summaries", lambda: C.build_summaries(cfg, p["k_hist"], gs, cs, ws, st)),
+            ("route", lambda: C.route(cfg, p["q"], gs, cs, ci, gi, ws, st)),
+            ("attn_fwd", lambda: C.attn_fwd(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi, o,
+                                            lse, ws, st)),
+            ("bwd_preprocess", lambda: C.attn_bwd_preprocess(cfg, o, p["d_o"], ws, st)),
+            ("bwd_dkdv", lambda: C.attn_bwd_dkdv(cfg, p["q"], p["k_seg"], p["v_seg"], lse, p["d_o"], dk, dv, ws,
+                                                 st)),
+            ("bwd_dq", lambda: C.attn_bwd_dq(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi,
+                                             lse, p["d_o"], dq, ws, st)),
+        ]
+
+    def forward(self, x: dict) -> None:
+        for _, call in self.calls(x)[:3]:
+            call()
+
+    def backward(self, x: dict) -> None:
+        for _, call in self.calls(x)[3:]:
+            call()
+
+    def __call__(self, x: dict) -> None:
+        for _, call in self.calls(x):
+            call()
+
+
+def default_scale(D: int = 128) -> float:
+    return 1.0 / math.sqrt(D)

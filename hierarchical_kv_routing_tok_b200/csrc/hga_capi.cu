@@ -1,0 +1,208 @@
+// C ABI of the routed-HGA library (declarations and contract in include/hga.h).
+// Validates every argument on the host, then enqueues the kernels on the
+// caller's stream.  No allocation, no synchronisation (except hga_read_status).
+#include <math.h>
+#include <stdint.h>
+
+#include "hga.h"
+#include "common.cuh"
+
+namespace hga {
+cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum,
+                             int64_t n_chunks_total, cudaStream_t stream);
+cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
+                         int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S, int nch,
+                         int kc, int kg, cudaStream_t stream);
+size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
+cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
+                                 const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
+                                 int64_t H, int64_t S, int kg, float scale, int* status, cudaStream_t st);
+cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
+                                  int64_t S, cudaStream_t st);
+cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
+                                 const void* d_o, const float* delta, void* dk, void* dv, int B, int Hq, int Hkv,
+                                 int64_t H, int64_t S, int kg, float scale, cudaStream_t st);
+cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
+                               const void* vs, const int32_t* gi, const float* lse, const void* d_o,
+                               const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
+                               float scale, int* status, cudaStream_t st);
+}  // namespace hga
+
+namespace {
+
+constexpr int64_t kMaxChunks = 32768;             // routing keeps one score per chunk in smem
+constexpr size_t kMaxRouteSmem = 200 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_config(const hga_config_t* c) {
+  if (!c) return HGA_ERR_ARG;
+  if (c->B < 1 || c->Hq < 1 || c->Hkv < 1 || c->Hq % c->Hkv != 0) return HGA_ERR_ARG;
+  if (c->dtype != HGA_F32 && c->dtype != HGA_BF16) return HGA_ERR_ARG;
+  if (c->D != hga::kD || c->chunk != hga::kChunk || c->group != hga::kGroup || c->qblock != hga::kQBlock)
+    return HGA_ERR_UNSUPPORTED;
+  if (c->n_sink_tokens != 0) return HGA_ERR_UNSUPPORTED;
+  if (c->hist_len < c->chunk || c->hist_len % c->chunk != 0) return HGA_ERR_ARG;
+  if (c->seg_len < c->qblock || c->seg_len % c->qblock != 0) return HGA_ERR_ARG;
+  const int64_t nch = c->hist_len / c->chunk;
+  if (nch > kMaxChunks) return HGA_ERR_UNSUPPORTED;
+  if (c->top_chunks < 1 || c->top_chunks > nch) return HGA_ERR_ARG;
+  if (c->top_groups < 1 || (int64_t)c->top_groups > (int64_t)c->top_chunks * (c->chunk / c->group))
+    return HGA_ERR_ARG;
+  if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return HGA_ERR_ARG;
+  // grid dimensions are 32-bit
+  if ((int64_t)c->B * c->Hq * (c->seg_len / c->qblock) > INT32_MAX) return HGA_ERR_UNSUPPORTED;
+  if ((int64_t)c->B * c->Hkv * nch > (int64_t)INT32_MAX * 8) return HGA_ERR_UNSUPPORTED;
+  if (hga::route_smem_bytes(c->dtype == HGA_BF16, (int)nch, c->top_chunks, c->top_groups) > kMaxRouteSmem)
+    return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p) return HGA_ERR_ARG;
+  for (const void* p : ps)
+    if (!aligned16(p)) return HGA_ERR_ALIGN;
+  return HGA_OK;
+}
+
+float eff_scale(const hga_config_t* c) {
+  return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->D);
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
+
+// The workspace starts with the status word.
+int* status_of(void* workspace) { return static_cast<int*>(workspace); }
+
+// Backward scratch (delta) lives after the status word of the workspace.
+float* delta_of(void* workspace) {
+  return reinterpret_cast<float*>(static_cast<char*>(workspace) + hga::kStatusBytes);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hga_version(void) { return HGA_VERSION; }
+
+const char* hga_strerror(int code) {
+  switch (code) {
+    case HGA_OK: return "ok";
+    case HGA_ERR_ARG: return "invalid argument (shape, budget or null pointer)";
+    case HGA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case HGA_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case HGA_ERR_CUDA: return "CUDA launch or copy failed";
+    case HGA_ERR_TIMEOUT: return "device-side bounded wait expired";
+    case HGA_ERR_WORKSPACE: return "workspace missing";
+    default: return "unknown status";
+  }
+}
+
+int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!bytes_out) return HGA_ERR_ARG;
+  const size_t delta = (size_t)cfg->B * cfg->Hq * cfg->seg_len * sizeof(float);
+  *bytes_out = hga::kStatusBytes + ((delta + 255) & ~(size_t)255);
+  return HGA_OK;
+}
+
+int hga_build_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum, float* chunk_sum,
+                        void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({k_hist, group_sum, chunk_sum}))) return rc;
+  (void)workspace;
+  const int64_t n_chunks = (int64_t)cfg->B * cfg->Hkv * (cfg->hist_len / cfg->chunk);
+  return from_cuda(hga::launch_summaries(cfg->dtype == HGA_BF16, k_hist, group_sum, chunk_sum, n_chunks,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, const float* chunk_sum,
+              int32_t* chunk_idx, int32_t* group_idx, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, group_sum, chunk_sum, chunk_idx, group_idx}))) return rc;
+  (void)workspace;
+  return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, group_sum, chunk_sum, chunk_idx, group_idx, cfg->B,
+                                     cfg->Hq, cfg->Hkv, cfg->seg_len, (int)(cfg->hist_len / cfg->chunk),
+                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
+}
+
+int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
+                 const void* v_seg, const int32_t* group_idx, void* o, float* lse, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  const bool bf16 = cfg->dtype == HGA_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
+                                             cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
+                                             eff_scale(cfg), status_of(workspace), st));
+}
+
+int hga_attn_bwd_preprocess(const hga_config_t* cfg, const void* o, const void* d_o, void* workspace,
+                            void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({o, d_o}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  return from_cuda(hga::launch_bwd_delta_simt(cfg->dtype == HGA_BF16, o, d_o, delta_of(workspace), cfg->B, cfg->Hq,
+                                              cfg->seg_len, static_cast<cudaStream_t>(stream)));
+}
+
+int hga_attn_bwd_dkdv(const hga_config_t* cfg, const void* q, const void* k_seg, const void* v_seg, const float* lse,
+                      const void* d_o, void* dk_seg, void* dv_seg, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
+                                             dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
+                                             cfg->top_groups, eff_scale(cfg), static_cast<cudaStream_t>(stream)));
+}
+
+int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
+                    const void* v_seg, const int32_t* group_idx, const float* lse, const void* d_o, void* dq,
+                    void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
+                                           d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
+                                           cfg->seg_len, cfg->top_groups, eff_scale(cfg), status_of(workspace),
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
+                 const void* v_seg, const int32_t* group_idx, const void* o, const float* lse, const void* d_o,
+                 void* dq, void* dk_seg, void* dv_seg, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
+  if ((rc = hga_attn_bwd_dkdv(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, stream))) return rc;
+  return hga_attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream);
+}
+
+int hga_read_status(void* workspace, void* stream, int32_t* status_out) {
+  if (!workspace || !status_out) return HGA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return HGA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(v), st) != cudaSuccess) return HGA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HGA_ERR_CUDA;
+  *status_out = v;
+  return HGA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,258 @@
+// Two-level HGA routing ("Long-Context Fine-Tuning with Limited VRAM",
+// gist.science Technical Summary 2.1 "Chunk Selection" / "Group Selection";
+// pith.science review Figure 1): the query block scores every history chunk
+// summary, keeps the best top_chunks, then scores the 8 group summaries of
+// each kept chunk and keeps the best top_groups.
+//
+// One CTA per (batch, KV head, 64-query block).  The block query (mean over
+// the block's positions and the KV head's query heads) stays in shared memory,
+// scores are warp dot products against float32 summaries (L2-resident), and
+// the top-k is an exact CTA-wide radix select on order-preserving 32-bit keys
+// followed by an index-ordered compaction, so ties go to the lower index and
+// the output comes out sorted ascending.  This is not a dense contraction
+// (M = 1 per CTA), so it runs on the CUDA cores.
+#include "common.cuh"
+
+namespace hga {
+
+constexpr int kRouteThreads = 256;
+
+// Larger score -> larger key; +0 and -0 map to the same key.
+__device__ __forceinline__ uint32_t order_key(float s) {
+  if (s == 0.f) s = 0.f;
+  const uint32_t b = __float_as_uint(s);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Exclusive scan of one int per thread over the CTA; returns the block total in *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < kRouteThreads / 32 ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kRouteThreads / 32) warp_tot[lane] = t;   // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = (warp == 0 ? 0 : warp_tot[warp - 1]);
+  *total = warp_tot[kRouteThreads / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// Select the k largest keys[0..n) (ties: lower position first); write the selected
+// positions, ascending, to out[0..k).  All threads of the CTA must call it.
+__device__ void block_select_topk(const uint32_t* keys, int n, int k, int* out, int* hist,
+                                  int* scratch /* >= 8 + 4 ints */) {
+  int* warp_tot = scratch;
+  int* bcast = scratch + 8;
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kRouteThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kRouteThreads) {
+      const uint32_t key = keys[i];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns bins 255-8l .. 248-8l (descending)
+      int c[8], s = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { c[e] = hist[255 - 8 * lane - e]; s += c[e]; }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned ball = __ballot_sync(0xffffffffu, incl >= remaining);
+      const int L = __ffs(ball) - 1;               // always exists: total >= remaining
+      if (lane == L) {
+        int cum = incl - s, digit = 0, rem = remaining;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (cum + c[e] >= remaining) { digit = 255 - 8 * lane - e; rem = remaining - cum; break; }
+          cum += c[e];
+        }
+        bcast[0] = digit;
+        bcast[1] = rem;
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)bcast[0] << shift;
+    pmask |= 0xFFu << shift;
+    remaining = bcast[1];
+    __syncthreads();
+  }
+  // keys > prefix are all taken; of the keys == prefix, the first `remaining` in index order.
+  const int per = (n + kRouteThreads - 1) / kRouteThreads;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int eq = 0;
+  for (int i = lo; i < hi; ++i) eq += (keys[i] == prefix);
+  int tot;
+  int eq_before = block_exclusive_scan(eq, warp_tot, &tot);
+  int cnt = 0;
+  {
+    int e = eq_before;
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t key = keys[i];
+      if (key > prefix) ++cnt;
+      else if (key == prefix) { if (e < remaining) ++cnt; ++e; }
+    }
+  }
+  int pos = block_exclusive_scan(cnt, warp_tot, &tot);
+  {
+    int e = eq_before;
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t key = keys[i];
+      bool take = false;
+      if (key > prefix) take = true;
+      else if (key == prefix) { take = e < remaining; ++e; }
+      if (take) out[pos++] = i;
+    }
+  }
+  __syncthreads();
+}
+
+// Dot products of qb (smem, 128 floats) with `count` rows of a float32 [*, 128] table,
+// row ids given by row_of(i); one warp per row, 4 rows in flight per warp.
+template <typename RowOf>
+__device__ __forceinline__ void score_rows(const float* qb, const float* __restrict__ table, int count,
+                                           RowOf row_of, uint32_t* keys_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float4 qv = *reinterpret_cast<const float4*>(qb + 4 * lane);
+  constexpr int W = kRouteThreads / 32;
+  for (int i0 = warp; i0 < count; i0 += 4 * W) {
+    float s[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * W;
+      s[u] = 0.f;
+      if (i < count) {
+        const float4 c = __ldg(reinterpret_cast<const float4*>(table + (int64_t)row_of(i) * kD) + lane);
+        s[u] = qv.x * c.x + qv.y * c.y + qv.z * c.z + qv.w * c.w;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+      const int i = i0 + u * W;
+      if (lane == 0 && i < count) keys_out[i] = order_key(s[u]);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(
+    const T* __restrict__ q, const float* __restrict__ group_sum, const float* __restrict__ chunk_sum,
+    int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq, int Hkv, int64_t S, int nch,
+    int kc, int kg) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int N = Vec16<T>::N;
+  constexpr int LPR = kD / N;
+  constexpr int RP = kRouteThreads / LPR;       // rows reduced in parallel
+  const int nblk = (int)(S / kQBlock);
+  const int unit = blockIdx.x;                  // (b*Hkv + kh)*nblk + n
+  const int n = unit % nblk;
+  const int bkh = unit / nblk;
+  const int kh = bkh % Hkv, b = bkh / Hkv;
+  const int G = Hq / Hkv;
+
+  float* red = reinterpret_cast<float*>(smem_raw);              // [RP][128]
+  float* qb = red + RP * kD;                                      // [128]
+  int* hist = reinterpret_cast<int*>(qb + kD);                    // [256]
+  int* scratch = hist + 256;                                      // [16]
+  int* csel = scratch + 16;                                       // [kc]
+  int* gpos = csel + ((kc + 3) & ~3);                             // [kg]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(gpos + ((kg + 3) & ~3));   // [max(nch, 8kc)]
+
+  // ---- block query: mean over G heads x 64 positions
+  {
+    const int tid = threadIdx.x;
+    const int col = (tid % LPR) * N, r0 = tid / LPR;
+    float acc[N];
+#pragma unroll
+    for (int e = 0; e < N; ++e) acc[e] = 0.f;
+    const int R = G * kQBlock;
+    for (int r = r0; r < R; r += RP) {
+      const int h = kh * G + r / kQBlock;
+      const int64_t t = (int64_t)n * kQBlock + r % kQBlock;
+      float v[N];
+      Vec16<T>::load(q + (((int64_t)b * Hq + h) * S + t) * kD + col, v);
+#pragma unroll
+      for (int e = 0; e < N; ++e) acc[e] += v[e];
+    }
+#pragma unroll
+    for (int e = 0; e < N; ++e) red[r0 * kD + col + e] = acc[e];
+    __syncthreads();
+    if (tid < kD) {
+      float s = 0.f;
+      for (int r = 0; r < RP; ++r) s += red[r * kD + tid];
+      qb[tid] = s / (float)R;
+    }
+    __syncthreads();
+  }
+
+  // ---- level 1: chunks
+  const float* cs = chunk_sum + (int64_t)bkh * nch * kD;
+  score_rows(qb, cs, nch, [](int i) { return i; }, keys);
+  __syncthreads();
+  block_select_topk(keys, nch, kc, csel, hist, scratch);
+
+  // ---- level 2: the 8 groups of every selected chunk
+  const float* gs = group_sum + (int64_t)bkh * nch * (kChunk / kGroup) * kD;
+  const int ncand = kc * (kChunk / kGroup);
+  score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
+  __syncthreads();
+  block_select_topk(keys, ncand, kg, gpos, hist, scratch);
+
+  for (int i = threadIdx.x; i < kc; i += kRouteThreads) chunk_idx[(int64_t)unit * kc + i] = csel[i];
+  for (int i = threadIdx.x; i < kg; i += kRouteThreads)
+    group_idx[(int64_t)unit * kg + i] = csel[gpos[i] >> 3] * 8 + (gpos[i] & 7);
+}
+
+size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
+  const int RP = kRouteThreads / (kD / (bf16 ? 8 : 4));
+  size_t words = (size_t)RP * kD + kD + 256 + 16 + ((kc + 3) & ~3) + ((kg + 3) & ~3) +
+                 (size_t)(nch > 8 * kc ? nch : 8 * kc);
+  return words * 4;
+}
+
+cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
+                         int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S,
+                         int nch, int kc, int kg, cudaStream_t stream) {
+  const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
+  if (units == 0) return cudaSuccess;
+  const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
+  cudaError_t e;
+  if (bf16) {
+    e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<__nv_bfloat16><<<(unsigned)units, kRouteThreads, smem, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, kc,
+        kg);
+  } else {
+    e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<float><<<(unsigned)units, kRouteThreads, smem, stream>>>(
+        static_cast<const float*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, kc, kg);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hga

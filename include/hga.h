@@ -1,0 +1,183 @@
+/*
+ * hga.h -- C ABI of the B200 (sm_100a) library for routed Hierarchical Global
+ * Attention (HGA): the attention step of one transformer layer over a
+ * detached history plus an active, differentiable segment.
+ *
+ * Method: "Long-Context Fine-Tuning with Limited VRAM" (arXiv 2607.15105).
+ *   - gist.science "Technical Summary", section 2.1 "Hierarchical Global
+ *     Attention": chunk selection over per-chunk summaries, group selection
+ *     inside the chosen chunks, exact-token attention over the selected
+ *     groups only; routing runs without gradient.
+ *   - same page, section 2.2: the history K/V are detached at the segment
+ *     boundary (segment-wise backward), so only the active segment gets
+ *     gradients.
+ *   - pith.science review, Figure 1 / Figure 2 captions and the
+ *     free-parameter ledger: 64-token chunks, 8-token groups, summaries for
+ *     every closed chunk, routed tokens alongside the local window.
+ *
+ * Readings where the pages are silent (the same ones the test oracle takes):
+ * a summary is the arithmetic mean of the keys it covers; the routing query
+ * of a block is the mean of its queries over the block's positions and the
+ * query heads of one KV head (one routing per batch x KV head x block); the
+ * score is the raw dot product; only history chunks are routable; group
+ * selection is one top-k over all groups of the chosen chunks; ties go to the
+ * lower index; index lists are sorted ascending; the local window is the whole
+ * causal prefix of the active segment; one softmax spans routed and local
+ * keys; softmax scale 1/sqrt(D) unless given.
+ *
+ * Conventions for every entry point
+ *   - Memory: the caller allocates and owns every buffer, including the
+ *     workspace.  All tensor pointers are DEVICE pointers, 16-byte aligned,
+ *     contiguous, head-major: q, o, d_o, dq: [B, Hq, S, D]; k/v history:
+ *     [B, Hkv, H, D]; k/v segment, dk/dv segment: [B, Hkv, S, D].  Query head
+ *     h uses KV head h / (Hq / Hkv).  Element type: float32 or bfloat16 as
+ *     set by cfg->dtype (summaries, LSE are always float32; indices int32).
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     Every call only enqueues work and returns without synchronising.
+ *   - Return value: HGA_OK, or a negative HGA_ERR_* code.  Argument checks
+ *     happen before anything is launched; on an error nothing is launched
+ *     and no output is touched.  HGA_ERR_CUDA reports a launch failure.
+ *   - Workspace: at least hga_workspace_size() bytes of device memory.  Its
+ *     first 256 bytes hold a sticky status word; they must be zero before the
+ *     first call (cudaMemset once) and are read and cleared by
+ *     hga_read_status().  Kernels that wait on on-chip barriers give up after
+ *     a bounded time and record HGA_ERR_TIMEOUT there instead of hanging; an
+ *     attention kernel given a group index outside [0, H/8) reads that group
+ *     as zeros (never out of bounds) and records HGA_ERR_ARG there.
+ *   - Aliasing: outputs must not overlap inputs or each other.
+ *   - Thread safety: the library keeps no mutable host state; calls on
+ *     different streams with different workspaces may run concurrently.
+ */
+#ifndef HGA_H_
+#define HGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HGA_VERSION 1
+
+/* Symbols of the shared library (built with hidden default visibility). */
+#if defined(__GNUC__)
+#define HGA_API __attribute__((visibility("default")))
+#else
+#define HGA_API
+#endif
+
+enum hga_status {
+  HGA_OK = 0,
+  HGA_ERR_ARG = -1,         /* bad shape, budget or null pointer            */
+  HGA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned             */
+  HGA_ERR_UNSUPPORTED = -3, /* valid for the method, not built (D != 128 ...) */
+  HGA_ERR_CUDA = -4,        /* kernel launch failed                         */
+  HGA_ERR_TIMEOUT = -5,     /* a device-side bounded wait expired           */
+  HGA_ERR_WORKSPACE = -6    /* workspace pointer missing                    */
+};
+
+enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 };
+
+/* Problem description.  chunk = 64, group = 8, qblock = 64 and D = 128 are
+ * the only built values (pith.science free-parameter ledger: chunk 64,
+ * group 8).  hist_len must be a positive multiple of chunk (only closed
+ * chunks exist), seg_len a positive multiple of qblock.
+ * 1 <= top_chunks <= hist_len / chunk; 1 <= top_groups <= top_chunks *
+ * (chunk / group).  n_sink_tokens must be 0 (sink window not built).
+ * softmax_scale = 0 selects 1 / sqrt(D). */
+typedef struct hga_config {
+  int32_t B, Hq, Hkv, D;
+  int64_t hist_len, seg_len;
+  int32_t chunk, group, qblock;
+  int32_t top_chunks, top_groups;
+  int32_t n_sink_tokens;
+  int32_t dtype;
+  float softmax_scale;
+} hga_config_t;
+
+/* Bytes of workspace the calls below need for this configuration. */
+HGA_API int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out);
+
+/* Summaries (Technical Summary 2.1, chunk and group selection; review,
+ * Figure 1): group_sum[b,kh,j,:] = mean of history keys 8j..8j+7;
+ * chunk_sum[b,kh,i,:] = mean of history keys 64i..64i+63.
+ *   k_hist     [B, Hkv, H, D]        cfg->dtype        (in)
+ *   group_sum  [B, Hkv, H/8, D]      float32           (out)
+ *   chunk_sum  [B, Hkv, H/64, D]     float32           (out) */
+HGA_API int hga_build_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum,
+                        float* chunk_sum, void* workspace, void* stream);
+
+/* Two-level routing (Technical Summary 2.1): for each (b, kv head kh, block
+ * n) the block query qb = mean of q over the block's 64 positions and the
+ * query heads of kh; chunk scores qb . chunk_sum over all history chunks,
+ * keep the top_chunks best; group scores qb . group_sum over the 8 groups of
+ * each kept chunk, keep the top_groups best.  Scores in float32; ties to
+ * the lower index; both lists written sorted ascending.  No gradient.
+ *   q          [B, Hq, S, D]               cfg->dtype  (in)
+ *   group_sum, chunk_sum                   float32     (in, from above)
+ *   chunk_idx  [B, Hkv, S/64, top_chunks]  int32       (out)
+ *   group_idx  [B, Hkv, S/64, top_groups]  int32       (out) */
+HGA_API int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum,
+              const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx,
+              void* workspace, void* stream);
+
+/* Forward (Technical Summary 2.1 "Exact-Token Attention"; review Figure 2):
+ * query (b, h, t) of block n = t/64 attends to the exact history tokens
+ * 8j..8j+7 of every j in group_idx[b, h/G, n, :] and to the segment tokens
+ * 0..t, with one softmax over both sets:
+ *   o = softmax(scale * q K^T) V,   lse = log sum exp(scale * q K^T).
+ *   q [B,Hq,S,D]; k_hist, v_hist [B,Hkv,H,D]; k_seg, v_seg [B,Hkv,S,D]
+ *   group_idx [B,Hkv,S/64,top_groups] int32, entries in [0, H/8)
+ *   o [B,Hq,S,D] (cfg->dtype, out); lse [B,Hq,S] float32 (out, natural log) */
+HGA_API int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist,
+                 const void* v_hist, const void* k_seg, const void* v_seg,
+                 const int32_t* group_idx, void* o, float* lse, void* workspace,
+                 void* stream);
+
+/* Backward of the forward above for L with dL/do = d_o (Technical Summary
+ * 2.1: routing has no gradient; 2.2: history detached).  Produces
+ *   dq over routed and local keys; dk_seg, dv_seg from the local (segment)
+ *   pairs only, summed over the G query heads of each KV head.
+ * No gradient is produced for k_hist / v_hist.  o and lse are the forward's
+ * outputs.  dq [B,Hq,S,D], dk_seg, dv_seg [B,Hkv,S,D] in cfg->dtype (out).
+ * Uses B*Hq*S*4 bytes of workspace scratch (delta, below). */
+HGA_API int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist,
+                 const void* v_hist, const void* k_seg, const void* v_seg,
+                 const int32_t* group_idx, const void* o, const float* lse,
+                 const void* d_o, void* dq, void* dk_seg, void* dv_seg, void* workspace,
+                 void* stream);
+
+/* The three steps of hga_attn_bwd as separate calls, in this order, on one
+ * stream and one workspace (the same computation; each launches one kernel):
+ *   preprocess: delta[b,h,t] = sum_d d_o * o  -> workspace scratch
+ *               (the FlashAttention-form backward the pages cite);
+ *   dkdv:       dk_seg, dv_seg from the local causal pairs (needs delta);
+ *   dq:         dq over routed and local keys (needs delta).
+ * Arguments as for hga_attn_bwd. */
+HGA_API int hga_attn_bwd_preprocess(const hga_config_t* cfg, const void* o, const void* d_o,
+                                    void* workspace, void* stream);
+HGA_API int hga_attn_bwd_dkdv(const hga_config_t* cfg, const void* q, const void* k_seg,
+                              const void* v_seg, const float* lse, const void* d_o,
+                              void* dk_seg, void* dv_seg, void* workspace, void* stream);
+HGA_API int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist,
+                            const void* v_hist, const void* k_seg, const void* v_seg,
+                            const int32_t* group_idx, const float* lse, const void* d_o,
+                            void* dq, void* workspace, void* stream);
+
+/* Synchronises `stream`, copies the workspace status word to *status_out
+ * (HGA_OK, HGA_ERR_TIMEOUT or HGA_ERR_ARG, see Workspace above) and clears it.  Returns HGA_ERR_CUDA if the
+ * copy itself fails. */
+HGA_API int hga_read_status(void* workspace, void* stream, int32_t* status_out);
+
+/* Static text for a status code. */
+HGA_API const char* hga_strerror(int code);
+
+/* HGA_VERSION of the built library. */
+HGA_API int hga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H_ */

@@ -1,0 +1,128 @@
+"""The C-ABI library: it loads, exports every symbol include/hga.h declares, its config struct
+matches the C layout, and argument validation rejects bad calls before anything is launched
+(these calls need no GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from hierarchical_kv_routing_tok_b200 import _capi as C
+from hierarchical_kv_routing_tok_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hga.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return C.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"HGA_API\s+[\w\s\*]*?\b(hga_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    assert sorted(C.EXPORTS) == names
+    out = subprocess.run(["nm", "-D", "--defined-only", C.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (hga_\w+)", out))
+    assert set(names) <= exported
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_version_and_strerror(lib):
+    hdr = open(HEADER).read()
+    assert C.version() == int(re.search(r"#define HGA_VERSION (\d+)", hdr).group(1))
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert C.strerror(code) and C.strerror(code) != "unknown status"
+    assert C.strerror(12345) == "unknown status"
+
+
+def test_config_struct_layout_matches_c(tmp_path):
+    src = tmp_path / "layout.c"
+    fields = [n for n, _ in C.HGAConfig._fields_]
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "hga.h"\nint main(void){\n'
+                   '  printf("%zu\\n", sizeof(hga_config_t));\n'
+                   + "".join(f'  printf("%zu\\n", offsetof(hga_config_t, {f}));\n' for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    vals = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
+    assert vals[0] == ctypes.sizeof(C.HGAConfig)
+    assert vals[1:] == [getattr(C.HGAConfig, f).offset for f in fields]
+
+
+def cfg(**kw):
+    base = dict(B=1, Hq=32, Hkv=8, hist_len=14336, seg_len=2048, top_chunks=16, top_groups=64)
+    base.update(kw)
+    return C.make_config(**base)
+
+
+def test_workspace_size(lib):
+    assert C.workspace_size(cfg()) == 256 + 32 * 2048 * 4
+    assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) == 256 + 3 * 4 * 64 * 4 + (256 - 3 * 4 * 64 * 4 % 256) % 256
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=30), C.HGA_ERR_ARG),                     # Hq not a multiple of Hkv
+    (dict(B=0), C.HGA_ERR_ARG),
+    (dict(D=64), C.HGA_ERR_UNSUPPORTED),
+    (dict(chunk=32), C.HGA_ERR_UNSUPPORTED),
+    (dict(group=4), C.HGA_ERR_UNSUPPORTED),
+    (dict(qblock=128), C.HGA_ERR_UNSUPPORTED),
+    (dict(n_sink_tokens=4), C.HGA_ERR_UNSUPPORTED),
+    (dict(hist_len=14300), C.HGA_ERR_ARG),            # open chunk
+    (dict(hist_len=0), C.HGA_ERR_ARG),
+    (dict(seg_len=2000), C.HGA_ERR_ARG),
+    (dict(top_chunks=0), C.HGA_ERR_ARG),
+    (dict(top_chunks=225), C.HGA_ERR_ARG),            # more chunks than the history has
+    (dict(top_groups=129), C.HGA_ERR_ARG),            # more groups than the chosen chunks hold
+    (dict(top_groups=0), C.HGA_ERR_ARG),
+    (dict(dtype=7), C.HGA_ERR_ARG),
+    (dict(softmax_scale=-1.0), C.HGA_ERR_ARG),
+    (dict(softmax_scale=float("nan")), C.HGA_ERR_ARG),
+    (dict(hist_len=64 * 40000, top_chunks=16), C.HGA_ERR_UNSUPPORTED),
+])
+def test_config_validation(lib, kw, code):
+    with pytest.raises(C.HGAError) as e:
+        C.workspace_size(cfg(**kw))
+    assert e.value.code == code
+
+
+def test_entry_points_reject_bad_pointers_before_launch(lib):
+    c = cfg()
+    ok, odd = 1 << 20, (1 << 20) + 8             # never dereferenced: validation fails first
+    calls = {
+        "summaries": lambda p: C.build_summaries(c, p[0], p[1], p[2], ok),
+        "route": lambda p: C.route(c, p[0], p[1], p[2], p[3], p[4], ok),
+        "fwd": lambda p: C.attn_fwd(c, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7], p[8]),
+        "bwd": lambda p: C.attn_bwd(c, *p[:13]),
+    }
+    for name, call in calls.items():
+        for i in range(3):
+            ptrs = [ok] * 13
+            ptrs[i] = None
+            with pytest.raises(C.HGAError) as e:
+                call(ptrs)
+            assert e.value.code == C.HGA_ERR_ARG, name
+            ptrs[i] = odd
+            with pytest.raises(C.HGAError) as e:
+                call(ptrs)
+            assert e.value.code == C.HGA_ERR_ALIGN, name
+    with pytest.raises(C.HGAError) as e:
+        C.attn_fwd(c, ok, ok, ok, ok, ok, ok, ok, ok, None)
+    assert e.value.code == C.HGA_ERR_WORKSPACE
+    with pytest.raises(C.HGAError) as e:
+        C.attn_bwd(c, *([ok] * 12), None)
+    assert e.value.code == C.HGA_ERR_WORKSPACE
+    bad = cfg(top_chunks=300)
+    with pytest.raises(C.HGAError) as e:
+        C.route(bad, ok, ok, ok, ok, ok, ok)
+    assert e.value.code == C.HGA_ERR_ARG

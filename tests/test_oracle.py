@@ -373,16 +373,18 @@ def test_invalid_arguments_raise(oracle):
 
 
 # --------------------------------------------------------------------------- inputs used by GPU parity
-PARITY_SEEDS = {"tiny_f32": [0, 1, 2, 3, 4], "ctx4k": [0, 1], "ctx16k": [0, 2], "ctx131k": [0]}
+PARITY_SEEDS = {"tiny_f32": [0, 1, 2, 3, 4], "small_bf16": [0, 1], "ctx4k": [0, 1], "ctx16k": [0, 2],
+                "ctx131k": [0]}
+PARITY_SEEDS.update({name: [0] for name in HI.EDGE_WORKLOADS})
 MIN_GAP = 4e-6
 
 
-@pytest.mark.parametrize("name", ["tiny_f32", "ctx4k", "ctx16k"])
+@pytest.mark.parametrize("name", ["tiny_f32", "small_bf16", "ctx4k", "ctx16k", *HI.EDGE_WORKLOADS])
 def test_parity_seeds_have_routing_margins(oracle, name):
     """For the seeds the GPU parity tests use, the fp32 routing equals the fp64 routing and every
     selection boundary has a score gap >= MIN_GAP (far above fp32 rounding of these scores,
     whose magnitude is < 10), so summation order cannot flip a selection."""
-    w = HI.WORKLOADS[name]
+    w = HI.WORKLOADS.get(name) or HI.EDGE_WORKLOADS[name]
     for seed in PARITY_SEEDS[name]:
         x = HI.make_inputs(w, seed)
         r32 = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32)
