@@ -1,0 +1,441 @@
+// Routed + causal-local attention forward on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Method: "Long-Context Fine-Tuning with Limited VRAM", gist.science Technical Summary 2.1
+// ("Exact-Token Attention": only the exact K/V of the selected groups are loaded) with the
+// causal local window of the active segment (pith.science review, Figure 2 caption), one softmax
+// over both key sets, online-softmax accumulation in the FlashAttention form the pages cite.
+//
+// One CTA per (batch, KV head, 64-query block, pair of query-head pairs): its query tile is
+// hpc = 2 * NT query heads x 64 positions = NT M-tiles of 128 rows that share one routed key set,
+// so every gathered K/V byte feeds NT MMAs.  Key tiles hold 128 keys:
+//   routed tiles: 16 groups of 8 history rows, each group fetched by TMA as two 8x64 boxes
+//                 (one per 64-dim half) into its own 1 KB swizzle atoms ("group layout");
+//   local tiles:  128 consecutive segment rows, two 128x64 boxes ("tile layout").
+// Warp roles: warp 0 = TMA producer, warp 1 = TMEM owner + single-thread MMA issuer,
+// warps 4.. = one softmax warpgroup per M-tile (thread = TMEM lane = query row).
+// TMEM: S_i (128 fp32 columns, P_i packed bf16 aliased into its first 64) and O_i (128 columns).
+// Issue order S_0 S_1 | PV_0 S_0' PV_1 S_1' | ... lets softmax i work on S_i while the tensor
+// core runs the other tile's MMAs; completion of S_i(j+1) implies completion of PV_i(j), so the
+// softmax may rescale O_i (lazily, only when its row max grows by more than 2^8) right after it.
+// Every mbarrier wait is bounded; on timeout the CTA records HGA_ERR_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "tc_common.cuh"
+
+namespace hga {
+namespace tcfwd {
+
+using namespace tc;
+
+constexpr int BN = 128;                    // keys per tile
+constexpr uint32_t kHalfBytes = BN * 128;  // one 64-dim half of a tile
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;
+constexpr float kRescaleThreshold = 8.f;   // log2 units
+
+struct Params {
+  int B, Hq, Hkv, G, hpc, kg, nblk;
+  int64_t H, S;
+  float scale_log2;
+  const int32_t* group_idx;
+  __nv_bfloat16* o;
+  float* lse;
+  int* status;
+};
+
+template <int NT>
+struct Smem {
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + NT * kTileBytes;
+  static constexpr uint32_t kV = kK + 2 * kTileBytes;
+  static constexpr uint32_t kBar = kV + 2 * kTileBytes;
+  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NT], p_full[NT], o_final, mma_done
+  static constexpr int kNumBars = 1 + 8 + 2 * NT + 2;
+  static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
+  static constexpr uint32_t kBytes = kMisc + 16;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// bounded wait that ignores the abort flag (used only to drain before exit)
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status) {
+  volatile int never = 0;
+  mbar_wait(bar, parity, &never, status);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(128 + 128 * NT, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
+                  const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
+                  const __grid_constant__ CUtensorMap tm_vs, const Params p) {
+  using L = Smem<NT>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBar;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const uint32_t q_full = BAR(0);
+  auto k_full = [&](int s) { return BAR(1 + s); };
+  auto k_empty = [&](int s) { return BAR(3 + s); };
+  auto v_full = [&](int s) { return BAR(5 + s); };
+  auto v_empty = [&](int s) { return BAR(7 + s); };
+  auto s_full = [&](int i) { return BAR(9 + i); };
+  auto p_full = [&](int i) { return BAR(9 + NT + i); };
+  const uint32_t o_final = BAR(9 + 2 * NT);
+  const uint32_t mma_done = BAR(10 + 2 * NT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- unit decode: heavy (late) query blocks first
+  const int hg = p.G / p.hpc;
+  int c = blockIdx.x;
+  const int hgi = c % hg;
+  c /= hg;
+  const int bkh = c % (p.B * p.Hkv);
+  const int n = p.nblk - 1 - c / (p.B * p.Hkv);
+  const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
+  const int h0 = kh * p.G + hgi * p.hpc;
+  const int n_rt = (8 * p.kg + BN - 1) / BN;
+  const int n_lt = n / 2 + 1;
+  const int T = n_rt + n_lt;
+  const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
+  const int64_t ngr = p.H / kGroup;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    for (int i = 0; i < NT; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(p_full(i), 128);
+    }
+    mbar_init(o_final, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), NT * 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kh);
+      tma_prefetch_desc(&tm_vh);
+      tma_prefetch_desc(&tm_ks);
+      tma_prefetch_desc(&tm_vs);
+      mbar_arrive_expect_tx(q_full, NT * kTileBytes);
+      for (int t = 0; t < NT; ++t)
+        for (int j = 0; j < 2; ++j) {
+          const int64_t row = ((int64_t)b * p.Hq + h0 + 2 * t + j) * p.S + (int64_t)n * kQBlock;
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(sbase + L::kQ + t * kTileBytes + h * kHalfBytes + j * (kHalfBytes / 2), &tm_q, 64 * h,
+                        (int32_t)row, q_full);
+        }
+    }
+    int issued_k[2] = {0, 0}, issued_v[2] = {0, 0};
+    for (int j = 0; j < T; ++j) {
+      const int s = j & 1;
+      const uint32_t par = ((j >> 1) & 1) ^ 1;
+      const bool routed = j < n_rt;
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t full = kv ? v_full(s) : k_full(s);
+        const uint32_t empty = kv ? v_empty(s) : k_empty(s);
+        const uint32_t dst = sbase + (kv ? L::kV : L::kK) + s * kTileBytes;
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(empty, par, abort_flag, p.status);
+          if (ok) mbar_arrive_expect_tx(full, kTileBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) goto producer_exit;
+        if (routed) {
+          if (lane < 16) {
+            const int slot = j * 16 + lane;
+            int32_t g = gi[slot < p.kg ? slot : 0];
+            if (g < 0 || (int64_t)g >= ngr) {
+              set_status(p.status, -1);
+              g = 0;
+            }
+            const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
+            const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
+            tma_load_2d(dst + lane * 2048, m, 0, row, full);
+            tma_load_2d(dst + lane * 2048 + 1024, m, 64, row, full);
+          }
+        } else if (lane == 0) {
+          const int jl = j - n_rt;
+          const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)jl * BN);
+          const CUtensorMap* m = kv ? &tm_vs : &tm_ks;
+          tma_load_2d(dst, m, 0, row, full);
+          tma_load_2d(dst + kHalfBytes, m, 64, row, full);
+        }
+        __syncwarp();
+        if (kv) ++issued_v[s]; else ++issued_k[s];
+      }
+    }
+  producer_exit:
+    // every load this warp issued has landed before the CTA may exit
+    if (lane == 0) {
+      for (int s = 0; s < 2; ++s) {
+        if (issued_k[s]) drain_wait(k_full(s), (issued_k[s] - 1) & 1, p.status);
+        if (issued_v[s]) drain_wait(v_full(s), (issued_v[s] - 1) & 1, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, true);
+      auto issue_s = [&](int j, int i) {
+        const int s = j & 1;
+        const bool routed = j < n_rt;
+        const uint32_t sbo = routed ? 2048u : 1024u;
+        const uint32_t half_off = routed ? 1024u : kHalfBytes;
+        const uint32_t kb = sbase + L::kK + s * kTileBytes;
+        const uint32_t qb = sbase + L::kQ + i * kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off_q = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
+          const uint32_t off_k = (ks >> 2) * half_off + (ks & 3) * 32;
+          mma_ss(tmem + i * 128, smem_desc_sw128(qb + off_q, 16, 1024), smem_desc_sw128(kb + off_k, 16, sbo),
+                 idesc_qk, ks > 0);
+        }
+      };
+      auto issue_pv = [&](int j, int i) {
+        const int s = j & 1;
+        const bool routed = j < n_rt;
+        const uint32_t lbo = routed ? 1024u : kHalfBytes;   // between 64-dim halves
+        const uint32_t sbo = routed ? 2048u : 1024u;        // between 8-key groups
+        const uint32_t vb = sbase + L::kV + s * kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, smem_desc_sw128(vb + ks * 2 * sbo, lbo, sbo),
+                 idesc_pv, (j > 0 || ks > 0));
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full(0), 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < NT; ++i) {
+          issue_s(0, i);
+          mma_commit(s_full(i));
+        }
+        mma_commit(k_empty(0));
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        const int s = j & 1;
+        ok = mbar_wait(v_full(s), (j >> 1) & 1, abort_flag, p.status);
+        if (ok && j + 1 < T) ok = mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status);
+        for (int i = 0; ok && i < NT; ++i) {
+          ok = mbar_wait(p_full(i), j & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j, i);
+          if (j + 1 < T) {
+            issue_s(j + 1, i);
+            mma_commit(s_full(i));
+          }
+        }
+        if (!ok) break;
+        mma_commit(v_empty(s));
+        if (j + 1 < T) mma_commit(k_empty((j + 1) & 1));
+      }
+      if (ok) mma_commit(o_final);
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ======================= softmax / epilogue, one warpgroup per M-tile
+    const int i = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                  // row of the M-tile = TMEM lane
+    const int head = h0 + 2 * i + (r >> 6);
+    const int64_t t_pos = (int64_t)n * kQBlock + (r & 63);
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + i * 128;
+    const uint32_t tO = tmem + lane_off + NT * 128 + i * 128;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      ok = mbar_wait(s_full(i), j & 1, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const bool routed = j < n_rt;
+      int nvalid;
+      if (routed) {
+        nvalid = min(BN, 8 * p.kg - j * BN);
+      } else {
+        const int64_t u0 = (int64_t)(j - n_rt) * BN;
+        nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
+      }
+      // pass 1: row max of the scaled logits
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tS + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (cc * 32 + e < nvalid) mx = fmaxf(mx, __uint_as_float(v[e]) * p.scale_log2);
+      }
+      // lazy rescale: move the reference max only when it grows by more than 2^8
+      const bool need = mx > m + kRescaleThreshold || (m == -INFINITY && mx > -INFINITY);
+      const float mnew = need ? mx : m;
+      const float alpha = need ? ex2(m - mnew) : 1.f;   // m = -inf -> 0
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tO + cc * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tmem_st32(tO + cc * 32, v);
+        }
+      }
+      l *= alpha;
+      m = mnew;
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      // pass 2: probabilities, row sum, bf16 P into the first 64 columns of S
+      float rs = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tS + cc * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = (cc * 32 + e < nvalid) ? ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref)) : 0.f;
+          const float p1 =
+              (cc * 32 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref)) : 0.f;
+          rs += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + cc * 16, pk);
+      }
+      l += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(i));
+    }
+    if (ok) {
+      ok = mbar_wait(o_final, 0, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* dst = p.o + (((int64_t)b * p.Hq + head) * p.S + t_pos) * kD;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tO + cc * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      }
+      p.lse[((int64_t)b * p.Hq + head) * p.S + t_pos] = (m + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NT * 256);
+  }
+}
+
+}  // namespace tcfwd
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;   // resolved once; the driver symbol never changes
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D bf16 map over a [rows, 128] row-major tensor, boxes of {64 dims, box_rows rows}, 128B swizzle.
+bool make_map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool attn_fwd_tc_supported(int Hq, int Hkv) {
+  const int G = Hq / Hkv;
+  return G % 2 == 0;
+}
+
+cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
+                               const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
+                               int kg, float scale, int* status, cudaStream_t st) {
+  CUtensorMap mq, mkh, mvh, mks, mvs;
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mkh, kh, (uint64_t)B * Hkv * H, 8) ||
+      !make_map_bf16_rows(&mvh, vh, (uint64_t)B * Hkv * H, 8) ||
+      !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, tcfwd::BN) ||
+      !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, tcfwd::BN))
+    return cudaErrorInvalidValue;
+  const int G = Hq / Hkv;
+  tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), H, S,
+                  scale * 1.4426950408889634f, gi, static_cast<__nv_bfloat16*>(o), lse, status};
+  const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
+  cudaError_t e;
+  if (p.hpc == 4) {
+    const size_t smem = tcfwd::Smem<2>::kBytes + 1024;
+    e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tcfwd::fwd_tc_kernel<2><<<(unsigned)grid, 384, smem, st>>>(mq, mkh, mvh, mks, mvs, p);
+  } else {
+    const size_t smem = tcfwd::Smem<1>::kBytes + 1024;
+    e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tcfwd::fwd_tc_kernel<1><<<(unsigned)grid, 256, smem, st>>>(mq, mkh, mvh, mks, mvs, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hga

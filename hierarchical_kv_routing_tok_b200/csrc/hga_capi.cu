@@ -3,6 +3,8 @@
 // caller's stream.  No allocation, no synchronisation (except hga_read_status).
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "hga.h"
 #include "common.cuh"
@@ -17,6 +19,10 @@ size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
                                  int64_t H, int64_t S, int kg, float scale, int* status, cudaStream_t st);
+bool attn_fwd_tc_supported(int Hq, int Hkv);
+cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
+                               const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
+                               int kg, float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
@@ -71,6 +77,13 @@ float eff_scale(const hga_config_t* c) {
 }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
+
+// HGA_ATTN_PATH=cuda_cores selects the CUDA-core attention kernels for every dtype (the
+// tensor-core kernels are the default for bf16); used to cross-check the two implementations.
+bool force_cuda_cores() {
+  const char* v = getenv("HGA_ATTN_PATH");
+  return v && strcmp(v, "cuda_cores") == 0;
+}
 
 // The workspace starts with the status word.
 int* status_of(void* workspace) { return static_cast<int*>(workspace); }
@@ -139,6 +152,10 @@ int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   const bool bf16 = cfg->dtype == HGA_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bf16 && hga::attn_fwd_tc_supported(cfg->Hq, cfg->Hkv) && !force_cuda_cores())
+    return from_cuda(hga::launch_attn_fwd_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B, cfg->Hq,
+                                             cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups, eff_scale(cfg),
+                                             status_of(workspace), st));
   return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
                                              cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
                                              eff_scale(cfg), status_of(workspace), st));
