@@ -20,13 +20,15 @@ HGA_ERR_UNSUPPORTED = -3
 HGA_ERR_CUDA = -4
 HGA_ERR_TIMEOUT = -5
 HGA_ERR_WORKSPACE = -6
+HGA_ERR_TOO_LARGE = -7
+HGA_NOALLOC_MAX_ROWS = 1 << 20
 HGA_F32 = 0
 HGA_BF16 = 1
 
 #: every entry point declared in include/hga.h
 EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd",
-           "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_read_status", "hga_strerror",
-           "hga_version")
+           "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
+           "hga_read_status", "hga_strerror", "hga_version")
 
 
 class HGAConfig(ctypes.Structure):
@@ -69,6 +71,7 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd_preprocess": [C, P, P, P, P],
         "hga_attn_bwd_dkdv": [C, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_dq": [C, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_attn_bwd_noalloc": [C, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
         "hga_strerror": [ctypes.c_int],
         "hga_version": [],
@@ -138,6 +141,14 @@ def attn_bwd_dkdv(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, str
 def attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream=0) -> None:
     _call("hga_attn_bwd_dq", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq,
           workspace, stream)
+
+
+def attn_bwd_noalloc(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg,
+                     stream=0) -> None:
+    """hga_attn_bwd without a workspace: for callers that cannot allocate device memory (the
+    library's fixed per-device scratch is used instead; overlapping calls race)."""
+    _call("hga_attn_bwd_noalloc", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o,
+          dq, dk_seg, dv_seg, stream)
 
 
 def read_status(workspace, stream=0) -> int:

@@ -108,6 +108,7 @@ const char* hga_strerror(int code) {
     case HGA_ERR_CUDA: return "CUDA launch or copy failed";
     case HGA_ERR_TIMEOUT: return "device-side bounded wait expired";
     case HGA_ERR_WORKSPACE: return "workspace missing";
+    case HGA_ERR_TOO_LARGE: return "problem larger than the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }

@@ -74,7 +74,8 @@ enum hga_status {
   HGA_ERR_UNSUPPORTED = -3, /* valid for the method, not built (D != 128 ...) */
   HGA_ERR_CUDA = -4,        /* kernel launch failed                         */
   HGA_ERR_TIMEOUT = -5,     /* a device-side bounded wait expired           */
-  HGA_ERR_WORKSPACE = -6    /* workspace pointer missing                    */
+  HGA_ERR_WORKSPACE = -6,   /* workspace pointer missing                    */
+  HGA_ERR_TOO_LARGE = -7    /* beyond the fixed scratch of hga_attn_bwd_noalloc */
 };
 
 enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 };
@@ -164,6 +165,30 @@ HGA_API int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* 
                             const void* v_hist, const void* k_seg, const void* v_seg,
                             const int32_t* group_idx, const float* lse, const void* d_o,
                             void* dq, void* workspace, void* stream);
+
+/* Backward without any allocation: the same computation and kernels as
+ * hga_attn_bwd, for callers that cannot allocate device memory -- e.g. a host
+ * runtime that has handed the whole device to its own memory pool, or code that
+ * must not call cudaMalloc/cudaFree because those may synchronise the device.
+ * The paper has no counterpart of this entry point; it exists for such callers.
+ *
+ * Scratch: instead of a caller workspace it uses one fixed device array of
+ * 256 + 4 * HGA_NOALLOC_MAX_ROWS bytes (4 MiB + 256 B) that every GPU loading
+ * the library holds until the process exits.  B * Hq * S must not exceed
+ * HGA_NOALLOC_MAX_ROWS, else HGA_ERR_TOO_LARGE is returned and nothing runs.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call clears the array's status word and overwrites the
+ * rest, and all calls share it: calls that overlap on the GPU (other streams,
+ * other threads) race and corrupt each other's results -- serialise them.
+ * Device-side status (see hga_read_status) is not reported by this entry.
+ * Arguments as for hga_attn_bwd, without workspace. */
+#define HGA_NOALLOC_MAX_ROWS (1 << 20)
+HGA_API int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, const void* k_hist,
+                                 const void* v_hist, const void* k_seg, const void* v_seg,
+                                 const int32_t* group_idx, const void* o, const float* lse,
+                                 const void* d_o, void* dq, void* dk_seg, void* dv_seg,
+                                 void* stream);
 
 /* Synchronises `stream`, copies the workspace status word to *status_out
  * (HGA_OK, HGA_ERR_TIMEOUT or HGA_ERR_ARG, see Workspace above) and clears it.  Returns HGA_ERR_CUDA if the

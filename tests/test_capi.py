@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_version_and_strerror(lib):
     hdr = open(HEADER).read()
     assert C.version() == int(re.search(r"#define HGA_VERSION (\d+)", hdr).group(1))
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert C.strerror(code) and C.strerror(code) != "unknown status"
     assert C.strerror(12345) == "unknown status"
 
