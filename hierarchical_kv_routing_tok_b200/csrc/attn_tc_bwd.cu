@@ -1,0 +1,682 @@
+// Routed + causal-local attention backward on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Method: "Long-Context Fine-Tuning with Limited VRAM", gist.science Technical Summary 2.1
+// (routing carries no gradient; the gather and the exact-token attention are differentiable) and
+// 2.2 (history K/V detached at the segment boundary, so only q and the active segment's K/V
+// receive gradients), with the softmax backward in the FlashAttention form the pages cite:
+// P = exp(S - lse), dP = dO V^T, dS = P o (dP - delta), dQ = scale dS K, dK = scale dS^T Q,
+// dV = P^T dO.
+//
+// dq_tc_kernel: one CTA per (batch, KV head, query block, 4 query heads) = two M=128 query tiles
+//   sharing one routed key set, as in the forward.  Key tiles of 64 keys (routed: 8 groups of 8
+//   history rows; local: 64 segment rows) so that S_i, dP_i (64 fp32 columns each) and dQ_i
+//   (128 columns) of both tiles fit the 512 TMEM columns.  dS_i is packed to bf16 into S_i's
+//   first 32 columns and feeds dQ_i += dS_i K from TMEM.
+// dkdv_tc_kernel: one CTA per (batch, KV head, 128-key tile, query head); keys are the M
+//   dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
+//   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  Each of the G query-head
+//   CTAs of one key tile stores its float32 partial dK / dV into its own workspace slot; the last
+//   one to finish (atomic ticket) sums the G slots in head order -- so the result does not depend
+//   on which CTA finishes first -- writes the output type and resets the ticket to zero.
+// Warp roles as in the forward: warp 0 TMA, warp 1 TMEM owner + single-thread MMA issuer,
+// warps 4.. element-wise warpgroups (thread = TMEM lane = row).  All mbarrier waits are bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "tc_common.cuh"
+
+namespace hga {
+
+bool make_map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows);
+
+namespace tcbwd {
+
+using namespace tc;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kQTile = 128 * 256;      // 128 rows x 128 dims bf16
+constexpr uint32_t kQHalf = 128 * 128;
+
+// ======================================================================================== dQ
+namespace dq {
+
+constexpr int BN = 64;                      // keys per tile
+constexpr uint32_t kKVTile = BN * 256;      // 16 KB
+constexpr uint32_t kKVHalf = BN * 128;      // 8 KB (local layout)
+
+struct Params {
+  int B, Hq, Hkv, G, hpc, kg, nblk;
+  int64_t H, S;
+  float c2;       // scale * log2(e)
+  float scale;
+  const int32_t* group_idx;
+  const float* lse;
+  const float* delta;
+  __nv_bfloat16* dq;
+  int* status;
+};
+
+template <int NT>
+struct Smem {
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kDO = kQ + NT * kQTile;
+  static constexpr uint32_t kK = kDO + NT * kQTile;
+  static constexpr uint32_t kV = kK + 2 * kKVTile;
+  static constexpr uint32_t kBar = kV + 2 * kKVTile;
+  // qdo_full, kv_full[2], kv_empty[2], sd_full[NT], ds_full[NT], final, mma_done
+  static constexpr int kNumBars = 1 + 4 + 2 * NT + 2;
+  static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
+  static constexpr uint32_t kBytes = kMisc + 16;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(128 + 128 * NT, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
+                 const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                 const Params p) {
+  using L = Smem<NT>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBar;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const uint32_t qdo_full = BAR(0);
+  auto kv_full = [&](int s) { return BAR(1 + s); };
+  auto kv_empty = [&](int s) { return BAR(3 + s); };
+  auto sd_full = [&](int i) { return BAR(5 + i); };
+  auto ds_full = [&](int i) { return BAR(5 + NT + i); };
+  const uint32_t final_bar = BAR(5 + 2 * NT);
+  const uint32_t mma_done = BAR(6 + 2 * NT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int hg = p.G / p.hpc;
+  int c = blockIdx.x;
+  const int hgi = c % hg;
+  c /= hg;
+  const int bkh = c % (p.B * p.Hkv);
+  const int n = p.nblk - 1 - c / (p.B * p.Hkv);
+  const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
+  const int h0 = kh * p.G + hgi * p.hpc;
+  const int n_rt = (8 * p.kg + BN - 1) / BN;
+  const int T = n_rt + n + 1;
+  const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
+  const int64_t ngr = p.H / kGroup;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qdo_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int i = 0; i < NT; ++i) {
+      mbar_init(sd_full(i), 1);
+      mbar_init(ds_full(i), 128);
+    }
+    mbar_init(final_bar, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), NT * 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(qdo_full, 2 * NT * kQTile);
+      for (int t = 0; t < NT; ++t)
+        for (int j = 0; j < 2; ++j) {
+          const int64_t row = ((int64_t)b * p.Hq + h0 + 2 * t + j) * p.S + (int64_t)n * kQBlock;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t off = t * kQTile + h * kQHalf + j * (kQHalf / 2);
+            tma_load_2d(sbase + L::kQ + off, &tm_q, 64 * h, (int32_t)row, qdo_full);
+            tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
+          }
+        }
+    }
+    int issued[2] = {0, 0};
+    for (int j = 0; j < T; ++j) {
+      const int s = j & 1;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(kv_empty(s), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (ok) mbar_arrive_expect_tx(kv_full(s), 2 * kKVTile);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const uint32_t kd = sbase + L::kK + s * kKVTile, vd = sbase + L::kV + s * kKVTile;
+      if (j < n_rt) {
+        if (lane < 8) {
+          const int slot = j * 8 + lane;
+          int32_t g = gi[slot < p.kg ? slot : 0];
+          if (g < 0 || (int64_t)g >= ngr) {
+            set_status(p.status, -1);
+            g = 0;
+          }
+          const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
+          tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(s));
+          tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(s));
+          tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(s));
+          tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(s));
+        }
+      } else if (lane == 0) {
+        const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)(j - n_rt) * BN);
+        tma_load_2d(kd, &tm_ks, 0, row, kv_full(s));
+        tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(s));
+        tma_load_2d(vd, &tm_vs, 0, row, kv_full(s));
+        tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(s));
+      }
+      __syncwarp();
+      ++issued[s];
+    }
+    if (lane == 0)
+      for (int s = 0; s < 2; ++s)
+        if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
+  } else if (warp == 1) {
+    // ======================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
+      auto issue_sdp = [&](int j, int i) {
+        const int s = j & 1;
+        const bool routed = j < n_rt;
+        const uint32_t sbo = routed ? 2048u : 1024u;
+        const uint32_t half_off = routed ? 1024u : kKVHalf;
+        const uint32_t kb = sbase + L::kK + s * kKVTile, vb = sbase + L::kV + s * kKVTile;
+        const uint32_t qb = sbase + L::kQ + i * kQTile, db = sbase + L::kDO + i * kQTile;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
+          const uint32_t ok = (ks >> 2) * half_off + (ks & 3) * 32;
+          mma_ss(tmem + i * 128, smem_desc_sw128(qb + oq, 16, 1024), smem_desc_sw128(kb + ok, 16, sbo), idesc_n64,
+                 ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
+          const uint32_t ok = (ks >> 2) * half_off + (ks & 3) * 32;
+          mma_ss(tmem + i * 128 + 64, smem_desc_sw128(db + oq, 16, 1024), smem_desc_sw128(vb + ok, 16, sbo),
+                 idesc_n64, ks > 0);
+        }
+      };
+      auto issue_dq = [&](int j, int i) {
+        const int s = j & 1;
+        const bool routed = j < n_rt;
+        const uint32_t lbo = routed ? 1024u : kKVHalf;
+        const uint32_t sbo = routed ? 2048u : 1024u;
+        const uint32_t kb = sbase + L::kK + s * kKVTile;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, smem_desc_sw128(kb + ks * 2 * sbo, lbo, sbo),
+                 idesc_dq, (j > 0 || ks > 0));
+      };
+      bool ok = mbar_wait(qdo_full, 0, abort_flag, p.status) && mbar_wait(kv_full(0), 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < NT; ++i) {
+          issue_sdp(0, i);
+          mma_commit(sd_full(i));
+        }
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) ok = mbar_wait(kv_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status);
+        for (int i = 0; ok && i < NT; ++i) {
+          ok = mbar_wait(ds_full(i), j & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dq(j, i);
+          if (j + 1 < T) {
+            issue_sdp(j + 1, i);
+            mma_commit(sd_full(i));
+          }
+        }
+        if (!ok) break;
+        mma_commit(kv_empty(j & 1));
+      }
+      if (ok) mma_commit(final_bar);
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ======================= element-wise: dS = P o (dP - delta), one warpgroup per M-tile
+    const int i = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int head = h0 + 2 * i + (r >> 6);
+    const int64_t t_pos = (int64_t)n * kQBlock + (r & 63);
+    const int64_t row = ((int64_t)b * p.Hq + head) * p.S + t_pos;
+    const float lse2 = p.lse[row] * kLog2e;
+    const float dl = p.delta[row];
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + i * 128;
+    const uint32_t tP = tS + 64;
+    const uint32_t tQ = tmem + lane_off + NT * 128 + i * 128;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(sd_full(i), j & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      int nvalid;
+      if (j < n_rt) {
+        nvalid = min(BN, 8 * p.kg - j * BN);
+      } else {
+        const int64_t u0 = (int64_t)(j - n_rt) * BN;
+        nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[32], dv[32], pk[16];
+        tmem_ld32(tS + hh * 32, sv);
+        tmem_ld32(tP + hh * 32, dv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int cidx = hh * 32 + e;
+          const float p0 = (cidx < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
+          const float p1 = (cidx + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
+          pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
+        }
+        tmem_st16(tS + hh * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full(i));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(final_bar, 0, abort_flag, p.status));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + row * kD;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32], pk[16];
+        tmem_ld32(tQ + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NT * 256);
+  }
+}
+
+}  // namespace dq
+
+// ======================================================================================== dK, dV
+namespace dkdv {
+
+constexpr int BM = 128;                     // keys per CTA (M dimension)
+constexpr int BQ = 64;                      // queries per step
+constexpr int NS = 3;                       // Q / dO / stats stages
+constexpr uint32_t kKTile = BM * 256;       // 32 KB
+constexpr uint32_t kKHalf = BM * 128;       // 16 KB
+constexpr uint32_t kQTileB = BQ * 256;      // 16 KB
+constexpr uint32_t kQHalfB = BQ * 128;      // 8 KB
+constexpr uint32_t kStatBytes = 2 * BQ * 4; // lse[64], delta[64]
+
+struct Params {
+  int B, Hq, Hkv, G, nblk, nkt;
+  int64_t S;
+  float c2, scale;
+  const float* lse;
+  const float* delta;
+  float* dk_part;       // [G][B*Hkv*S][128] float32 partials, one slot per query head of the group
+  float* dv_part;
+  int* ticket;          // [B*Hkv][nkt]
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int* status;
+};
+
+struct Smem {
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kKTile;
+  static constexpr uint32_t kQ = kV + kKTile;
+  static constexpr uint32_t kDO = kQ + NS * kQTileB;
+  static constexpr uint32_t kStat = kDO + NS * kQTileB;
+  static constexpr uint32_t kBar = kStat + NS * kStatBytes;
+  // kv_full, q_full[NS], q_empty[NS], sd_full[2], pd_full[2], done, mma_done
+  static constexpr int kNumBars = 1 + 2 * NS + 4 + 2;
+  static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
+  static constexpr uint32_t kBytes = kMisc + 16;
+};
+
+__global__ void __launch_bounds__(384, 1)
+    dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                   const Params p) {
+  using L = Smem;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBar;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const uint32_t kv_full = BAR(0);
+  auto q_full = [&](int s) { return BAR(1 + s); };
+  auto q_empty = [&](int s) { return BAR(1 + NS + s); };
+  auto sd_full = [&](int b) { return BAR(1 + 2 * NS + b); };
+  auto pd_full = [&](int b) { return BAR(3 + 2 * NS + b); };
+  const uint32_t done = BAR(5 + 2 * NS);
+  const uint32_t mma_done = BAR(6 + 2 * NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- unit decode: key tile m (heavy = early first), batch x KV head, query head
+  int c = blockIdx.x;
+  const int hin = c % p.G;
+  c /= p.G;
+  const int bkh = c % (p.B * p.Hkv);
+  const int m = c / (p.B * p.Hkv);
+  const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
+  const int head = kh * p.G + hin;
+  const int n0 = 2 * m;                       // first query block that sees this key tile
+  const int Tq = p.nblk - n0;
+  const int64_t qrow0 = ((int64_t)b * p.Hq + head) * p.S;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(sd_full(x), 1);
+      mbar_init(pd_full(x), 128);
+    }
+    mbar_init(done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * kKTile);
+      const int32_t krow = (int32_t)((int64_t)bkh * p.S + (int64_t)m * BM);
+      tma_load_2d(sbase + L::kK, &tm_ks, 0, krow, kv_full);
+      tma_load_2d(sbase + L::kK + kKHalf, &tm_ks, 64, krow, kv_full);
+      tma_load_2d(sbase + L::kV, &tm_vs, 0, krow, kv_full);
+      tma_load_2d(sbase + L::kV + kKHalf, &tm_vs, 64, krow, kv_full);
+      int issued[NS] = {0, 0, 0};
+      for (int i = 0; i < Tq; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(q_empty(s), ((i / NS) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(q_full(s), 2 * kQTileB + kStatBytes);
+        const int64_t row = qrow0 + (int64_t)(n0 + i) * BQ;
+        tma_load_2d(sbase + L::kQ + s * kQTileB, &tm_q, 0, (int32_t)row, q_full(s));
+        tma_load_2d(sbase + L::kQ + s * kQTileB + kQHalfB, &tm_q, 64, (int32_t)row, q_full(s));
+        tma_load_2d(sbase + L::kDO + s * kQTileB, &tm_do, 0, (int32_t)row, q_full(s));
+        tma_load_2d(sbase + L::kDO + s * kQTileB + kQHalfB, &tm_do, 64, (int32_t)row, q_full(s));
+        bulk_load(sbase + L::kStat + s * kStatBytes, p.lse + row, BQ * 4, q_full(s));
+        bulk_load(sbase + L::kStat + s * kStatBytes + BQ * 4, p.delta + row, BQ * 4, q_full(s));
+        ++issued[s];
+      }
+      drain_wait(kv_full, 0, p.status);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s]) drain_wait(q_full(s), (issued[s] - 1) & 1, p.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BQ, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(BM, kD, true);
+      auto issue_sd = [&](int i, int x) {
+        const int s = i % NS;
+        const uint32_t qb = sbase + L::kQ + s * kQTileB, db = sbase + L::kDO + s * kQTileB;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t ok_ = (ks >> 2) * kKHalf + (ks & 3) * 32;
+          const uint32_t oq = (ks >> 2) * kQHalfB + (ks & 3) * 32;
+          mma_ss(tmem + x * 128, smem_desc_sw128(sbase + L::kK + ok_, 16, 1024), smem_desc_sw128(qb + oq, 16, 1024),
+                 idesc_s, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t ok_ = (ks >> 2) * kKHalf + (ks & 3) * 32;
+          const uint32_t oq = (ks >> 2) * kQHalfB + (ks & 3) * 32;
+          mma_ss(tmem + x * 128 + 64, smem_desc_sw128(sbase + L::kV + ok_, 16, 1024),
+                 smem_desc_sw128(db + oq, 16, 1024), idesc_s, ks > 0);
+        }
+      };
+      auto issue_grad = [&](int i, int x) {
+        const int s = i % NS;
+        const uint32_t qb = sbase + L::kQ + s * kQTileB, db = sbase + L::kDO + s * kQTileB;
+#pragma unroll
+        for (int ks = 0; ks < BQ / 16; ++ks) {
+          // dV += P^T dO ; dK += dS^T Q  (B operands MN-major: 64-dim halves 8 KB apart, 8 rows 1 KB apart)
+          mma_ts(tmem + 256, tmem + x * 128 + ks * 8, smem_desc_sw128(db + ks * 2048, kQHalfB, 1024), idesc_g,
+                 (i > 0 || ks > 0));
+          mma_ts(tmem + 384, tmem + x * 128 + 64 + ks * 8, smem_desc_sw128(qb + ks * 2048, kQHalfB, 1024), idesc_g,
+                 (i > 0 || ks > 0));
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
+      for (int i = 0; ok && i < 2 && i < Tq; ++i) {
+        ok = mbar_wait(q_full(i % NS), (i / NS) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sd(i, i & 1);
+        mma_commit(sd_full(i & 1));
+      }
+      for (int i = 0; ok && i < Tq; ++i) {
+        const int x = i & 1;
+        ok = mbar_wait(pd_full(x), (i >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_grad(i, x);
+        mma_commit(q_empty(i % NS));
+        if (i + 2 < Tq) {
+          ok = mbar_wait(q_full((i + 2) % NS), ((i + 2) / NS) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sd(i + 2, x);
+          mma_commit(sd_full(x));
+        }
+      }
+      if (ok) mma_commit(done);
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ======================= element-wise: P^T, dS^T (warpgroup x takes query steps i = x mod 2)
+    const int x = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;          // key row within the tile
+    const int64_t u = (int64_t)m * BM + r;      // key position in the segment
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + x * 128;
+    const uint32_t tP = tS + 64;
+    const float* stat_base = reinterpret_cast<const float*>(smem + L::kStat);
+    bool ok = true;
+    for (int i = x; i < Tq; i += 2) {
+      const int s = i % NS;
+      ok = mbar_wait(sd_full(x), (i >> 1) & 1, abort_flag, p.status);
+      if (ok) ok = mbar_wait(q_full(s), (i / NS) & 1, abort_flag, p.status);   // stats landed
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float* lse = stat_base + s * (kStatBytes / 4);
+      const float* dlt = lse + BQ;
+      const int64_t t0 = (int64_t)(n0 + i) * BQ;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[32], dv[32], pp[16], pd[16];
+        tmem_ld32(tS + hh * 32, sv);
+        tmem_ld32(tP + hh * 32, dv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int q0 = hh * 32 + e;
+          const bool v0 = u <= t0 + q0, v1 = u <= t0 + q0 + 1;
+          const float p0 = v0 ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse[q0] * kLog2e)) : 0.f;
+          const float p1 = v1 ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse[q0 + 1] * kLog2e)) : 0.f;
+          pp[e >> 1] = pack_bf16(p0, p1);
+          pd[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dlt[q0]), p1 * (__uint_as_float(dv[e + 1]) - dlt[q0 + 1]));
+        }
+        tmem_st16(tS + hh * 16, pp);
+        tmem_st16(tP + hh * 16, pd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(pd_full(x));
+    }
+    // ---- epilogue: warpgroup 0 owns dV, warpgroup 1 owns dK; store this head's float32 partial
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t tacc = tmem + lane_off + (x == 0 ? 256 : 384);
+      const size_t slot = (size_t)hin * p.B * p.Hkv * p.S * kD;
+      float* part = (x == 0 ? p.dv_part : p.dk_part) + slot + ((int64_t)bkh * p.S + u) * kD;
+      const float mul = (x == 0) ? 1.f : p.scale;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tacc + cc * 32, v);
+        tmem_wait_ld();
+        if (u < p.S) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            __stcg(reinterpret_cast<float4*>(part + cc * 32 + e),
+                   make_float4(__uint_as_float(v[e]) * mul, __uint_as_float(v[e + 1]) * mul,
+                               __uint_as_float(v[e + 2]) * mul, __uint_as_float(v[e + 3]) * mul));
+        }
+      }
+      __threadfence();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  // ---- the last of the G query-head CTAs of this key tile converts and clears it
+  if (*abort_flag) return;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    int* tk = p.ticket + (int64_t)bkh * p.nkt + m;
+    const int prev = atomicAdd(tk, 1);
+    if (prev == p.G - 1) {
+      *tk = 0;
+      *last_flag = 1;
+    }
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  const int64_t key0 = (int64_t)bkh * p.S + (int64_t)m * BM;
+  const int64_t nkeys = min((int64_t)BM, p.S - (int64_t)m * BM);
+  const size_t slot = (size_t)p.B * p.Hkv * p.S * kD;
+  for (int64_t e = (int64_t)threadIdx.x * 4; e < nkeys * kD; e += (int64_t)blockDim.x * 4) {
+    float4 ks = make_float4(0.f, 0.f, 0.f, 0.f), vs = ks;
+    for (int h = 0; h < p.G; ++h) {                 // fixed order: bitwise reproducible
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(p.dk_part + h * slot + key0 * kD + e));
+      const float4 c4 = __ldcg(reinterpret_cast<const float4*>(p.dv_part + h * slot + key0 * kD + e));
+      ks.x += a.x; ks.y += a.y; ks.z += a.z; ks.w += a.w;
+      vs.x += c4.x; vs.y += c4.y; vs.z += c4.z; vs.w += c4.w;
+    }
+    store4(p.dk + key0 * kD + e, ks);
+    store4(p.dv + key0 * kD + e, vs);
+  }
+}
+
+}  // namespace dkdv
+}  // namespace tcbwd
+
+// ------------------------------------------------------------------ host side
+size_t bwd_tc_acc_bytes(int B, int Hq, int Hkv, int64_t S) {
+  const int64_t nkt = (S + tcbwd::dkdv::BM - 1) / tcbwd::dkdv::BM;
+  const int G = Hq / Hkv;
+  return 2 * (size_t)G * B * Hkv * S * kD * sizeof(float) + (size_t)B * Hkv * nkt * sizeof(int);
+}
+
+cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
+                             const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
+                             cudaStream_t st) {
+  namespace K = tcbwd::dq;
+  CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mdo, d_o, (uint64_t)B * Hq * S, 64) ||
+      !make_map_bf16_rows(&mkh, kh, (uint64_t)B * Hkv * H, 8) ||
+      !make_map_bf16_rows(&mvh, vh, (uint64_t)B * Hkv * H, 8) ||
+      !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, K::BN) ||
+      !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
+    return cudaErrorInvalidValue;
+  const int G = Hq / Hkv;
+  K::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), H, S, scale * tcbwd::kLog2e, scale,
+              gi, lse, delta, static_cast<__nv_bfloat16*>(dq), status};
+  const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
+  cudaError_t e;
+  if (p.hpc == 4) {
+    const size_t smem = K::Smem<2>::kBytes + 1024;
+    e = cudaFuncSetAttribute(K::dq_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    K::dq_tc_kernel<2><<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
+  } else {
+    const size_t smem = K::Smem<1>::kBytes + 1024;
+    e = cudaFuncSetAttribute(K::dq_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    K::dq_tc_kernel<1><<<(unsigned)grid, 256, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
+                               const float* delta, void* dk, void* dv, void* acc, int B, int Hq, int Hkv, int64_t S,
+                               float scale, int* status, cudaStream_t st) {
+  namespace K = tcbwd::dkdv;
+  CUtensorMap mq, mdo, mks, mvs;
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, K::BQ) ||
+      !make_map_bf16_rows(&mdo, d_o, (uint64_t)B * Hq * S, K::BQ) ||
+      !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, K::BM) ||
+      !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BM))
+    return cudaErrorInvalidValue;
+  const int G = Hq / Hkv;
+  const int nkt = (int)((S + K::BM - 1) / K::BM);
+  float* dk_part = static_cast<float*>(acc);
+  float* dv_part = dk_part + (size_t)G * B * Hkv * S * kD;
+  int* ticket = reinterpret_cast<int*>(dv_part + (size_t)G * B * Hkv * S * kD);
+  K::Params p{B, Hq, Hkv, G, (int)(S / kQBlock), nkt, S, scale * tcbwd::kLog2e, scale, lse, delta, dk_part, dv_part,
+              ticket, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), status};
+  const int64_t grid = (int64_t)B * Hkv * nkt * G;
+  const size_t smem = K::Smem::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  K::dkdv_tc_kernel<<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mks, mvs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace hga

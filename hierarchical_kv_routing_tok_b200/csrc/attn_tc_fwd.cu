@@ -57,17 +57,6 @@ struct Smem {
   static constexpr uint32_t kBytes = kMisc + 16;
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// bounded wait that ignores the abort flag (used only to drain before exit)
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status) {
-  volatile int never = 0;
-  mbar_wait(bar, parity, &never, status);
-}
 
 template <int NT>
 __global__ void __launch_bounds__(128 + 128 * NT, 1)

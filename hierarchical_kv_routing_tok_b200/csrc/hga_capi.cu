@@ -23,6 +23,14 @@ bool attn_fwd_tc_supported(int Hq, int Hkv);
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
                                int kg, float scale, int* status, cudaStream_t st);
+size_t bwd_tc_acc_bytes(int B, int Hq, int Hkv, int64_t S);
+cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
+                             const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
+                             cudaStream_t st);
+cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
+                               const float* delta, void* dk, void* dv, void* acc, int B, int Hq, int Hkv, int64_t S,
+                               float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
@@ -88,12 +96,57 @@ bool force_cuda_cores() {
 // The workspace starts with the status word.
 int* status_of(void* workspace) { return static_cast<int*>(workspace); }
 
-// Backward scratch (delta) lives after the status word of the workspace.
+// Workspace layout: [status word | delta rows (float32) | dK, dV accumulators (float32) and
+// per-key-tile tickets of the tensor-core dK/dV kernel].
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t delta_bytes(const hga_config_t* c) { return (size_t)c->B * c->Hq * c->seg_len * sizeof(float); }
 float* delta_of(void* workspace) {
   return reinterpret_cast<float*>(static_cast<char*>(workspace) + hga::kStatusBytes);
 }
+size_t acc_offset(const hga_config_t* c) { return hga::kStatusBytes + round256(delta_bytes(c)); }
+void* acc_of(void* workspace, const hga_config_t* c) { return static_cast<char*>(workspace) + acc_offset(c); }
+size_t full_workspace_bytes(const hga_config_t* c) {
+  return acc_offset(c) + round256(hga::bwd_tc_acc_bytes(c->B, c->Hq, c->Hkv, c->seg_len));
+}
+
+// The tensor-core attention kernels handle bf16 with an even number of query heads per KV head.
+bool use_tc(const hga_config_t* c) {
+  return c->dtype == HGA_BF16 && hga::attn_fwd_tc_supported(c->Hq, c->Hkv) && !force_cuda_cores();
+}
+
+// dK/dV with a workspace of ws_bytes: the tensor-core kernel needs the accumulator region.
+int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const void* v_seg, const float* lse,
+                const void* d_o, void* dk_seg, void* dv_seg, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg});
+  if (rc) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (use_tc(cfg) && ws_bytes >= full_workspace_bytes(cfg))
+    return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg,
+                                             acc_of(workspace, cfg), cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
+                                             eff_scale(cfg), status_of(workspace), st));
+  return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
+                                             dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
+                                             cfg->top_groups, eff_scale(cfg), st));
+}
 
 }  // namespace
+
+// The whole backward with a workspace of ws_bytes (also used by the no-allocation entry point).
+int hga_internal_attn_bwd_ws(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist,
+                             const void* k_seg, const void* v_seg, const int32_t* group_idx, const void* o,
+                             const float* lse, const void* d_o, void* dq, void* dk_seg, void* dv_seg, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
+  if ((rc = bwd_dkdv_ws(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, ws_bytes, stream))) return rc;
+  return hga_attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream);
+}
 
 extern "C" {
 
@@ -117,8 +170,7 @@ int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out) {
   int rc = check_config(cfg);
   if (rc) return rc;
   if (!bytes_out) return HGA_ERR_ARG;
-  const size_t delta = (size_t)cfg->B * cfg->Hq * cfg->seg_len * sizeof(float);
-  *bytes_out = hga::kStatusBytes + ((delta + 255) & ~(size_t)255);
+  *bytes_out = full_workspace_bytes(cfg);
   return HGA_OK;
 }
 
@@ -153,7 +205,7 @@ int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   const bool bf16 = cfg->dtype == HGA_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (bf16 && hga::attn_fwd_tc_supported(cfg->Hq, cfg->Hkv) && !force_cuda_cores())
+  if (use_tc(cfg))
     return from_cuda(hga::launch_attn_fwd_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B, cfg->Hq,
                                              cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups, eff_scale(cfg),
                                              status_of(workspace), st));
@@ -177,12 +229,7 @@ int hga_attn_bwd_dkdv(const hga_config_t* cfg, const void* q, const void* k_seg,
                       const void* d_o, void* dk_seg, void* dv_seg, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg}))) return rc;
-  if (!workspace) return HGA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
-  return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
-                                             dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
-                                             cfg->top_groups, eff_scale(cfg), static_cast<cudaStream_t>(stream)));
+  return bwd_dkdv_ws(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, full_workspace_bytes(cfg), stream);
 }
 
 int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
@@ -193,10 +240,14 @@ int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, 
   if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq}))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (use_tc(cfg))
+    return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, delta_of(workspace),
+                                           dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
+                                           eff_scale(cfg), status_of(workspace), st));
   return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
                                            d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
-                                           cfg->seg_len, cfg->top_groups, eff_scale(cfg), status_of(workspace),
-                                           static_cast<cudaStream_t>(stream)));
+                                           cfg->seg_len, cfg->top_groups, eff_scale(cfg), status_of(workspace), st));
 }
 
 int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
@@ -204,12 +255,8 @@ int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
                  void* dq, void* dk_seg, void* dv_seg, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
-  if (!workspace) return HGA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
-  if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
-  if ((rc = hga_attn_bwd_dkdv(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, stream))) return rc;
-  return hga_attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream);
+  return hga_internal_attn_bwd_ws(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg,
+                                  workspace, full_workspace_bytes(cfg), stream);
 }
 
 int hga_read_status(void* workspace, void* stream, int32_t* status_out) {

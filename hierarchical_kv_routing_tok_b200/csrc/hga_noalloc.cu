@@ -34,6 +34,11 @@ int scratch_for_current_device(void** out) {
 
 }  // namespace
 
+int hga_internal_attn_bwd_ws(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist,
+                             const void* k_seg, const void* v_seg, const int32_t* group_idx, const void* o,
+                             const float* lse, const void* d_o, void* dq, void* dk_seg, void* dv_seg, void* workspace,
+                             size_t ws_bytes, void* stream);
+
 extern "C" int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist,
                                     const void* k_seg, const void* v_seg, const int32_t* group_idx, const void* o,
                                     const float* lse, const void* d_o, void* dq, void* dk_seg, void* dv_seg,
@@ -47,6 +52,7 @@ extern "C" int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, cons
   // the status word must start at zero; delta is fully rewritten by the first kernel
   if (cudaMemsetAsync(scratch, 0, hga::kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return HGA_ERR_CUDA;
-  return hga_attn_bwd(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg, scratch,
-                      stream);
+  // kernels that need more scratch than the fixed array holds fall back to the CUDA-core ones
+  return hga_internal_attn_bwd_ws(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg,
+                                  scratch, kScratchBytes, stream);
 }

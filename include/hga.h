@@ -37,10 +37,14 @@
  *   - Return value: HGA_OK, or a negative HGA_ERR_* code.  Argument checks
  *     happen before anything is launched; on an error nothing is launched
  *     and no output is touched.  HGA_ERR_CUDA reports a launch failure.
- *   - Workspace: at least hga_workspace_size() bytes of device memory.  Its
- *     first 256 bytes hold a sticky status word; they must be zero before the
- *     first call (cudaMemset once) and are read and cleared by
- *     hga_read_status().  Kernels that wait on on-chip barriers give up after
+ *   - Workspace: at least hga_workspace_size() bytes of device memory, zero-
+ *     filled once before its first use (cudaMemset); every successful call
+ *     leaves what must start at zero at zero again.  Layout:
+ *     a 256-byte sticky status word (read and cleared by hga_read_status()),
+ *     the backward's delta rows (B*Hq*S float32), then per-query-head float32
+ *     dK / dV partials and per-key-tile counters of the tensor-core dK/dV
+ *     kernel (the counters must start at zero; the kernel resets them).  After a call reports an error the workspace must be zero-filled
+ *     again before reuse.  Kernels that wait on on-chip barriers give up after
  *     a bounded time and record HGA_ERR_TIMEOUT there instead of hanging; an
  *     attention kernel given a group index outside [0, H/8) reads that group
  *     as zeros (never out of bounds) and records HGA_ERR_ARG there.
@@ -142,7 +146,7 @@ HGA_API int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_h
  *   pairs only, summed over the G query heads of each KV head.
  * No gradient is produced for k_hist / v_hist.  o and lse are the forward's
  * outputs.  dq [B,Hq,S,D], dk_seg, dv_seg [B,Hkv,S,D] in cfg->dtype (out).
- * Uses B*Hq*S*4 bytes of workspace scratch (delta, below). */
+ * Uses the workspace scratch described above (delta, dK/dV accumulators). */
 HGA_API int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist,
                  const void* v_hist, const void* k_seg, const void* v_seg,
                  const int32_t* group_idx, const void* o, const float* lse,

@@ -65,9 +65,17 @@ def cfg(**kw):
     return C.make_config(**base)
 
 
+def _expected_ws(B, Hq, Hkv, S):
+    r256 = lambda x: (x + 255) // 256 * 256
+    delta = B * Hq * S * 4
+    acc = 2 * Hq * B * S * 128 * 4 + B * Hkv * ((S + 127) // 128) * 4    # G fp32 dK, dV slots + tickets
+    return 256 + r256(delta) + r256(acc)
+
+
 def test_workspace_size(lib):
-    assert C.workspace_size(cfg()) == 256 + 32 * 2048 * 4
-    assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) == 256 + 3 * 4 * 64 * 4 + (256 - 3 * 4 * 64 * 4 % 256) % 256
+    assert C.workspace_size(cfg()) == _expected_ws(1, 32, 8, 2048)
+    assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) == _expected_ws(3, 4, 1, 64)
+    assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) % 256 == 0
 
 
 @pytest.mark.parametrize("kw,code", [
