@@ -44,6 +44,7 @@ namespace dq {
 constexpr int BN = 64;                      // keys per tile
 constexpr uint32_t kKVTile = BN * 256;      // 16 KB
 constexpr uint32_t kKVHalf = BN * 128;      // 8 KB (local layout)
+constexpr int KVS = 3;                      // K/V stages
 
 struct Params {
   int B, Hq, Hkv, G, hpc, kg, nblk;
@@ -62,10 +63,10 @@ struct Smem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kDO = kQ + NT * kQTile;
   static constexpr uint32_t kK = kDO + NT * kQTile;
-  static constexpr uint32_t kV = kK + 2 * kKVTile;
-  static constexpr uint32_t kBar = kV + 2 * kKVTile;
-  // qdo_full, kv_full[2], kv_empty[2], sd_full[NT], ds_full[NT], final, mma_done
-  static constexpr int kNumBars = 1 + 4 + 2 * NT + 2;
+  static constexpr uint32_t kV = kK + KVS * kKVTile;
+  static constexpr uint32_t kBar = kV + KVS * kKVTile;
+  // qdo_full, kv_full[KVS], kv_empty[KVS], sd_full[NT], ds_full[NT], final, mma_done
+  static constexpr int kNumBars = 1 + 2 * KVS + 2 * NT + 2;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
@@ -84,11 +85,11 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const uint32_t qdo_full = BAR(0);
   auto kv_full = [&](int s) { return BAR(1 + s); };
-  auto kv_empty = [&](int s) { return BAR(3 + s); };
-  auto sd_full = [&](int i) { return BAR(5 + i); };
-  auto ds_full = [&](int i) { return BAR(5 + NT + i); };
-  const uint32_t final_bar = BAR(5 + 2 * NT);
-  const uint32_t mma_done = BAR(6 + 2 * NT);
+  auto kv_empty = [&](int s) { return BAR(1 + KVS + s); };
+  auto sd_full = [&](int i) { return BAR(1 + 2 * KVS + i); };
+  auto ds_full = [&](int i) { return BAR(1 + 2 * KVS + NT + i); };
+  const uint32_t final_bar = BAR(1 + 2 * KVS + 2 * NT);
+  const uint32_t mma_done = BAR(2 + 2 * KVS + 2 * NT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KVS; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
@@ -144,12 +145,12 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
           }
         }
     }
-    int issued[2] = {0, 0};
+    int issued[KVS] = {0, 0, 0};
     for (int j = 0; j < T; ++j) {
-      const int s = j & 1;
+      const int s = j % KVS;
       int ok = 1;
       if (lane == 0) {
-        ok = mbar_wait(kv_empty(s), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
+        ok = mbar_wait(kv_empty(s), ((j / KVS) & 1) ^ 1, abort_flag, p.status);
         if (ok) mbar_arrive_expect_tx(kv_full(s), 2 * kKVTile);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       ++issued[s];
     }
     if (lane == 0)
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < KVS; ++s)
         if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
   } else if (warp == 1) {
     // ======================= MMA issuer
@@ -188,7 +189,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
       auto issue_sdp = [&](int j, int i) {
-        const int s = j & 1;
+        const int s = j % KVS;
         const bool routed = j < n_rt;
         const uint32_t sbo = routed ? 2048u : 1024u;
         const uint32_t half_off = routed ? 1024u : kKVHalf;
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         }
       };
       auto issue_dq = [&](int j, int i) {
-        const int s = j & 1;
+        const int s = j % KVS;
         const bool routed = j < n_rt;
         const uint32_t lbo = routed ? 1024u : kKVHalf;
         const uint32_t sbo = routed ? 2048u : 1024u;
@@ -229,19 +230,22 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         }
       }
       for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T) ok = mbar_wait(kv_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status);
         for (int i = 0; ok && i < NT; ++i) {
           ok = mbar_wait(ds_full(i), j & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           issue_dq(j, i);
           if (j + 1 < T) {
+            // the next K/V tile is only needed now, after this tile's first dQ MMAs are queued
+            if (i == 0) ok = mbar_wait(kv_full((j + 1) % KVS), ((j + 1) / KVS) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
             issue_sdp(j + 1, i);
             mma_commit(sd_full(i));
           }
         }
         if (!ok) break;
-        mma_commit(kv_empty(j & 1));
+        mma_commit(kv_empty(j % KVS));
       }
       if (ok) mma_commit(final_bar);
       mma_commit(mma_done);
@@ -326,7 +330,7 @@ namespace dkdv {
 
 constexpr int BM = 128;                     // keys per CTA (M dimension)
 constexpr int BQ = 64;                      // queries per step
-constexpr int NS = 3;                       // Q / dO / stats stages
+constexpr int NS = 4;                       // Q / dO / stats stages
 constexpr uint32_t kKTile = BM * 256;       // 32 KB
 constexpr uint32_t kKHalf = BM * 128;       // 16 KB
 constexpr uint32_t kQTileB = BQ * 256;      // 16 KB
@@ -428,7 +432,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_load_2d(sbase + L::kK + kKHalf, &tm_ks, 64, krow, kv_full);
       tma_load_2d(sbase + L::kV, &tm_vs, 0, krow, kv_full);
       tma_load_2d(sbase + L::kV + kKHalf, &tm_vs, 64, krow, kv_full);
-      int issued[NS] = {0, 0, 0};
+      int issued[NS] = {0, 0, 0, 0};
       for (int i = 0; i < Tq; ++i) {
         const int s = i % NS;
         if (!mbar_wait(q_empty(s), ((i / NS) & 1) ^ 1, abort_flag, p.status)) break;

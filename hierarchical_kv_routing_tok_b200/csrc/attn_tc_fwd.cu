@@ -45,14 +45,18 @@ struct Params {
   int* status;
 };
 
+constexpr int KS = 3;                      // K stages (K runs ahead of V)
+constexpr int VS = 2;                      // V stages
+
 template <int NT>
 struct Smem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + NT * kTileBytes;
-  static constexpr uint32_t kV = kK + 2 * kTileBytes;
-  static constexpr uint32_t kBar = kV + 2 * kTileBytes;
-  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NT], p_full[NT], o_final, mma_done
-  static constexpr int kNumBars = 1 + 8 + 2 * NT + 2;
+  static constexpr uint32_t kV = kK + KS * kTileBytes;
+  static constexpr uint32_t kBar = kV + VS * kTileBytes;
+  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NT], p_full[NT], o_final,
+  // mma_done
+  static constexpr int kNumBars = 1 + 2 * KS + 2 * VS + 2 * NT + 2;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
@@ -71,13 +75,13 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const uint32_t q_full = BAR(0);
   auto k_full = [&](int s) { return BAR(1 + s); };
-  auto k_empty = [&](int s) { return BAR(3 + s); };
-  auto v_full = [&](int s) { return BAR(5 + s); };
-  auto v_empty = [&](int s) { return BAR(7 + s); };
-  auto s_full = [&](int i) { return BAR(9 + i); };
-  auto p_full = [&](int i) { return BAR(9 + NT + i); };
-  const uint32_t o_final = BAR(9 + 2 * NT);
-  const uint32_t mma_done = BAR(10 + 2 * NT);
+  auto k_empty = [&](int s) { return BAR(1 + KS + s); };
+  auto v_full = [&](int s) { return BAR(1 + 2 * KS + s); };
+  auto v_empty = [&](int s) { return BAR(1 + 2 * KS + VS + s); };
+  auto s_full = [&](int i) { return BAR(1 + 2 * KS + 2 * VS + i); };
+  auto p_full = [&](int i) { return BAR(1 + 2 * KS + 2 * VS + NT + i); };
+  const uint32_t o_final = BAR(1 + 2 * KS + 2 * VS + 2 * NT);
+  const uint32_t mma_done = BAR(2 + 2 * KS + 2 * VS + 2 * NT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -100,9 +104,11 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
@@ -124,14 +130,15 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ======================= TMA producer
-    if (lane == 0) {
+  if (warp == 0 || warp == 2) {
+    // ======================= TMA producers: warp 0 loads Q and the K tiles, warp 2 the V tiles,
+    // each through its own ring of stages, so K can run ahead of V.
+    const int kv = warp == 2;
+    const int NS = kv ? VS : KS;
+    if (!kv && lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kh);
-      tma_prefetch_desc(&tm_vh);
       tma_prefetch_desc(&tm_ks);
-      tma_prefetch_desc(&tm_vs);
       mbar_arrive_expect_tx(q_full, NT * kTileBytes);
       for (int t = 0; t < NT; ++t)
         for (int j = 0; j < 2; ++j) {
@@ -141,61 +148,57 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
                         (int32_t)row, q_full);
         }
     }
-    int issued_k[2] = {0, 0}, issued_v[2] = {0, 0};
+    if (kv && lane == 0) {
+      tma_prefetch_desc(&tm_vh);
+      tma_prefetch_desc(&tm_vs);
+    }
+    int issued[KS] = {0, 0, 0};
     for (int j = 0; j < T; ++j) {
-      const int s = j & 1;
-      const uint32_t par = ((j >> 1) & 1) ^ 1;
-      const bool routed = j < n_rt;
-      for (int kv = 0; kv < 2; ++kv) {
-        const uint32_t full = kv ? v_full(s) : k_full(s);
-        const uint32_t empty = kv ? v_empty(s) : k_empty(s);
-        const uint32_t dst = sbase + (kv ? L::kV : L::kK) + s * kTileBytes;
-        int ok = 1;
-        if (lane == 0) {
-          ok = mbar_wait(empty, par, abort_flag, p.status);
-          if (ok) mbar_arrive_expect_tx(full, kTileBytes);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) goto producer_exit;
-        if (routed) {
-          if (lane < 16) {
-            const int slot = j * 16 + lane;
-            int32_t g = gi[slot < p.kg ? slot : 0];
-            if (g < 0 || (int64_t)g >= ngr) {
-              set_status(p.status, -1);
-              g = 0;
-            }
-            const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
-            const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
-            tma_load_2d(dst + lane * 2048, m, 0, row, full);
-            tma_load_2d(dst + lane * 2048 + 1024, m, 64, row, full);
+      const int s = j % NS;
+      const uint32_t full = kv ? v_full(s) : k_full(s);
+      const uint32_t empty = kv ? v_empty(s) : k_empty(s);
+      const uint32_t dst = sbase + (kv ? L::kV : L::kK) + s * kTileBytes;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(empty, ((j / NS) & 1) ^ 1, abort_flag, p.status);
+        if (ok) mbar_arrive_expect_tx(full, kTileBytes);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (j < n_rt) {
+        if (lane < 16) {
+          const int slot = j * 16 + lane;
+          int32_t g = gi[slot < p.kg ? slot : 0];
+          if (g < 0 || (int64_t)g >= ngr) {
+            set_status(p.status, -1);
+            g = 0;
           }
-        } else if (lane == 0) {
-          const int jl = j - n_rt;
-          const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)jl * BN);
-          const CUtensorMap* m = kv ? &tm_vs : &tm_ks;
-          tma_load_2d(dst, m, 0, row, full);
-          tma_load_2d(dst + kHalfBytes, m, 64, row, full);
+          const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
+          const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
+          tma_load_2d(dst + lane * 2048, m, 0, row, full);
+          tma_load_2d(dst + lane * 2048 + 1024, m, 64, row, full);
         }
-        __syncwarp();
-        if (kv) ++issued_v[s]; else ++issued_k[s];
+      } else if (lane == 0) {
+        const int jl = j - n_rt;
+        const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)jl * BN);
+        const CUtensorMap* m = kv ? &tm_vs : &tm_ks;
+        tma_load_2d(dst, m, 0, row, full);
+        tma_load_2d(dst + kHalfBytes, m, 64, row, full);
       }
+      __syncwarp();
+      ++issued[s];
     }
-  producer_exit:
     // every load this warp issued has landed before the CTA may exit
-    if (lane == 0) {
-      for (int s = 0; s < 2; ++s) {
-        if (issued_k[s]) drain_wait(k_full(s), (issued_k[s] - 1) & 1, p.status);
-        if (issued_v[s]) drain_wait(v_full(s), (issued_v[s] - 1) & 1, p.status);
-      }
-    }
+    if (lane == 0)
+      for (int s = 0; s < NS; ++s)
+        if (issued[s]) drain_wait(kv ? v_full(s) : k_full(s), (issued[s] - 1) & 1, p.status);
   } else if (warp == 1) {
     // ======================= MMA issuer (one thread)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, true);
       auto issue_s = [&](int j, int i) {
-        const int s = j & 1;
+        const int s = j % KS;
         const bool routed = j < n_rt;
         const uint32_t sbo = routed ? 2048u : 1024u;
         const uint32_t half_off = routed ? 1024u : kHalfBytes;
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         }
       };
       auto issue_pv = [&](int j, int i) {
-        const int s = j & 1;
+        const int s = j % VS;
         const bool routed = j < n_rt;
         const uint32_t lbo = routed ? 1024u : kHalfBytes;   // between 64-dim halves
         const uint32_t sbo = routed ? 2048u : 1024u;        // between 8-key groups
@@ -231,22 +234,24 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         mma_commit(k_empty(0));
       }
       for (int j = 0; ok && j < T; ++j) {
-        const int s = j & 1;
-        ok = mbar_wait(v_full(s), (j >> 1) & 1, abort_flag, p.status);
-        if (ok && j + 1 < T) ok = mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status);
+        ok = mbar_wait(v_full(j % VS), (j / VS) & 1, abort_flag, p.status);
         for (int i = 0; ok && i < NT; ++i) {
           ok = mbar_wait(p_full(i), j & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           issue_pv(j, i);
           if (j + 1 < T) {
+            // the next K tile is only needed now, after this tile's first PV is queued
+            if (i == 0) ok = mbar_wait(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
             issue_s(j + 1, i);
             mma_commit(s_full(i));
           }
         }
         if (!ok) break;
-        mma_commit(v_empty(s));
-        if (j + 1 < T) mma_commit(k_empty((j + 1) & 1));
+        mma_commit(v_empty(j % VS));
+        if (j + 1 < T) mma_commit(k_empty((j + 1) % KS));
       }
       if (ok) mma_commit(o_final);
       mma_commit(mma_done);
@@ -278,17 +283,23 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
       }
-      // pass 1: row max of the scaled logits
+      // pass 1: row max of the raw logits (the scale is positive), masking only where needed
       float mx = -INFINITY;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
         tmem_ld32(tS + cc * 32, v);
         tmem_wait_ld();
+        if (nvalid >= BN) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (cc * 32 + e < nvalid) mx = fmaxf(mx, __uint_as_float(v[e]) * p.scale_log2);
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (cc * 32 + e < nvalid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
       }
+      mx *= p.scale_log2;
       // lazy rescale: move the reference max only when it grows by more than 2^8
       const bool need = mx > m + kRescaleThreshold || (m == -INFINITY && mx > -INFINITY);
       const float mnew = need ? mx : m;
@@ -315,13 +326,23 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         tmem_ld32(tS + cc * 32, v);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (nvalid >= BN) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = (cc * 32 + e < nvalid) ? ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref)) : 0.f;
-          const float p1 =
-              (cc * 32 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref)) : 0.f;
-          rs += p0 + p1;
-          pk[e >> 1] = pack_bf16(p0, p1);
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref));
+            const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref));
+            rs += p0 + p1;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = (cc * 32 + e < nvalid) ? ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref)) : 0.f;
+            const float p1 =
+                (cc * 32 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref)) : 0.f;
+            rs += p0 + p1;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
         }
         tmem_st16(tS + cc * 16, pk);
       }

@@ -7,9 +7,10 @@
 // One CTA per (batch, KV head, 64-query block).  The block query (mean over
 // the block's positions and the KV head's query heads) stays in shared memory,
 // scores are warp dot products against float32 summaries (L2-resident), and
-// the top-k is an exact CTA-wide radix select on order-preserving 32-bit keys
-// followed by an index-ordered compaction, so ties go to the lower index and
-// the output comes out sorted ascending.  This is not a dense contraction
+// the top-k is exact: a one-pass rank selection when a level has at most 256
+// candidates, else a CTA-wide radix select on order-preserving 32-bit keys; both
+// finish with an index-ordered compaction, so ties go to the lower index and the
+// output comes out sorted ascending.  This is not a dense contraction
 // (M = 1 per CTA), so it runs on the CUDA cores.
 #include "common.cuh"
 
@@ -128,18 +129,41 @@ __device__ void block_select_topk(const uint32_t* keys, int n, int k, int* out, 
   __syncthreads();
 }
 
+// Select the k largest keys[0..n) for n <= kRouteThreads: thread i computes the rank of key i
+// (number of keys that precede it in the order "larger first, lower position first" -- compares
+// against broadcast shared-memory reads) and keeps it if rank < k; an index-ordered scan of the
+// kept flags writes the positions ascending.  One pass, two barriers.
+__device__ void block_select_topk_small(const uint32_t* keys, int n, int k, int* out, int* scratch) {
+  const int i = threadIdx.x;
+  bool take = false;
+  if (i < n) {
+    const uint32_t ki = keys[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const uint32_t kj = keys[j];
+      rank += (kj > ki) | ((kj == ki) & (j < i));
+    }
+    take = rank < k;
+  }
+  int tot;
+  const int pos = block_exclusive_scan(take ? 1 : 0, scratch, &tot);
+  if (take) out[pos] = i;
+  __syncthreads();
+}
+
 // Dot products of qb (smem, 128 floats) with `count` rows of a float32 [*, 128] table,
-// row ids given by row_of(i); one warp per row, 4 rows in flight per warp.
+// row ids given by row_of(i); one warp per row, 8 rows in flight per warp.
 template <typename RowOf>
 __device__ __forceinline__ void score_rows(const float* qb, const float* __restrict__ table, int count,
                                            RowOf row_of, uint32_t* keys_out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float4 qv = *reinterpret_cast<const float4*>(qb + 4 * lane);
   constexpr int W = kRouteThreads / 32;
-  for (int i0 = warp; i0 < count; i0 += 4 * W) {
-    float s[4];
+  constexpr int U = 8;
+  for (int i0 = warp; i0 < count; i0 += U * W) {
+    float s[U];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int i = i0 + u * W;
       s[u] = 0.f;
       if (i < count) {
@@ -148,7 +172,7 @@ __device__ __forceinline__ void score_rows(const float* qb, const float* __restr
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
       const int i = i0 + u * W;
@@ -189,13 +213,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
 #pragma unroll
     for (int e = 0; e < N; ++e) acc[e] = 0.f;
     const int R = G * kQBlock;
-    for (int r = r0; r < R; r += RP) {
-      const int h = kh * G + r / kQBlock;
-      const int64_t t = (int64_t)n * kQBlock + r % kQBlock;
-      float v[N];
-      Vec16<T>::load(q + (((int64_t)b * Hq + h) * S + t) * kD + col, v);
+    constexpr int UQ = 8;                        // loads in flight per thread
+    for (int r1 = r0; r1 < R; r1 += UQ * RP) {
+      float v[UQ][N];
 #pragma unroll
-      for (int e = 0; e < N; ++e) acc[e] += v[e];
+      for (int u = 0; u < UQ; ++u) {
+        const int r = r1 + u * RP;
+        if (r < R) {
+          const int h = kh * G + r / kQBlock;
+          const int64_t t = (int64_t)n * kQBlock + r % kQBlock;
+          Vec16<T>::load(q + (((int64_t)b * Hq + h) * S + t) * kD + col, v[u]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < N; ++e) v[u][e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UQ; ++u)
+#pragma unroll
+        for (int e = 0; e < N; ++e) acc[e] += v[u][e];
     }
 #pragma unroll
     for (int e = 0; e < N; ++e) red[r0 * kD + col + e] = acc[e];
@@ -212,14 +248,20 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   const float* cs = chunk_sum + (int64_t)bkh * nch * kD;
   score_rows(qb, cs, nch, [](int i) { return i; }, keys);
   __syncthreads();
-  block_select_topk(keys, nch, kc, csel, hist, scratch);
+  if (nch <= kRouteThreads)
+    block_select_topk_small(keys, nch, kc, csel, scratch);
+  else
+    block_select_topk(keys, nch, kc, csel, hist, scratch);
 
   // ---- level 2: the 8 groups of every selected chunk
   const float* gs = group_sum + (int64_t)bkh * nch * (kChunk / kGroup) * kD;
   const int ncand = kc * (kChunk / kGroup);
   score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
   __syncthreads();
-  block_select_topk(keys, ncand, kg, gpos, hist, scratch);
+  if (ncand <= kRouteThreads)
+    block_select_topk_small(keys, ncand, kg, gpos, scratch);
+  else
+    block_select_topk(keys, ncand, kg, gpos, hist, scratch);
 
   for (int i = threadIdx.x; i < kc; i += kRouteThreads) chunk_idx[(int64_t)unit * kc + i] = csel[i];
   for (int i = threadIdx.x; i < kg; i += kRouteThreads)
