@@ -10,8 +10,9 @@
 // dq_tc_kernel: one CTA per (batch, KV head, query block, 4 query heads) = two M=128 query tiles
 //   sharing one routed key set, as in the forward.  Key tiles of 64 keys (routed: 8 groups of 8
 //   history rows; local: 64 segment rows) so that S_i, dP_i (64 fp32 columns each) and dQ_i
-//   (128 columns) of both tiles fit the 512 TMEM columns.  dS_i is packed to bf16 into S_i's
-//   first 32 columns and feeds dQ_i += dS_i K from TMEM.
+//   (128 columns) of both tiles fit the 512 TMEM columns.  Two element-wise warpgroups per M-tile
+//   each own 32 key columns; each packs its dS to bf16 into the first 16 of its own 32 S columns,
+//   and dQ_i += dS_i K reads them from TMEM.
 // dkdv_tc_kernel: one CTA per (batch, KV head, 128-key tile, query head); keys are the M
 //   dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
 //   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  Each of the G query-head
@@ -19,7 +20,8 @@
 //   one to finish (atomic ticket) sums the G slots in head order -- so the result does not depend
 //   on which CTA finishes first -- writes the output type and resets the ticket to zero.
 // Warp roles as in the forward: warp 0 TMA, warp 1 TMEM owner + single-thread MMA issuer,
-// warps 4.. element-wise warpgroups (thread = TMEM lane = row).  All mbarrier waits are bounded.
+// warps 4.. element-wise warpgroups (thread = TMEM lane = row; two warpgroups split each tile's
+// columns so that each thread handles 32 elements per step).  All mbarrier waits are bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -72,7 +74,7 @@ struct Smem {
 };
 
 template <int NT>
-__global__ void __launch_bounds__(128 + 128 * NT, 1)
+__global__ void __launch_bounds__(128 + 256 * NT, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
     }
     for (int i = 0; i < NT; ++i) {
       mbar_init(sd_full(i), 1);
-      mbar_init(ds_full(i), 128);
+      mbar_init(ds_full(i), 256);
     }
     mbar_init(final_bar, 1);
     mbar_init(mma_done, 1);
@@ -184,42 +186,41 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       for (int s = 0; s < KVS; ++s)
         if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
   } else if (warp == 1) {
-    // ======================= MMA issuer
+    // ======================= MMA issuer (one thread).  Descriptor arrays are built before each
+    // unrolled MMA sequence from 64-bit base descriptors prepared once.
     if (lane == 0) {
       constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
+      // stage bases: stage st is st * kKVTile bytes after stage 0 (descriptor units of 16 bytes)
+      const uint64_t q0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
+      const uint64_t do0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t k_rt = smem_desc_sw128(sbase + L::kK, 16, 2048), k_lc = smem_desc_sw128(sbase + L::kK, 16, 1024);
+      const uint64_t v_rt = smem_desc_sw128(sbase + L::kV, 16, 2048), v_lc = smem_desc_sw128(sbase + L::kV, 16, 1024);
+      const uint64_t kmn_rt = smem_desc_sw128(sbase + L::kK, 1024, 2048);
+      const uint64_t kmn_lc = smem_desc_sw128(sbase + L::kK, kKVHalf, 1024);
       auto issue_sdp = [&](int j, int i) {
-        const int s = j % KVS;
-        const bool routed = j < n_rt;
-        const uint32_t sbo = routed ? 2048u : 1024u;
-        const uint32_t half_off = routed ? 1024u : kKVHalf;
-        const uint32_t kb = sbase + L::kK + s * kKVTile, vb = sbase + L::kV + s * kKVTile;
-        const uint32_t qb = sbase + L::kQ + i * kQTile, db = sbase + L::kDO + i * kQTile;
+        const bool rt = j < n_rt;
+        const uint64_t soff = (uint64_t)((j % KVS) * (kKVTile >> 4));
+        const uint32_t half_enc = rt ? (1024u >> 4) : (kKVHalf >> 4);
+        uint64_t a[8], bb[8];
+        kmajor_from_base(a, q0 + (uint64_t)(i * (kQTile >> 4)), kQHalf >> 4);
+        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, half_enc);
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
-          const uint32_t ok = (ks >> 2) * half_off + (ks & 3) * 32;
-          mma_ss(tmem + i * 128, smem_desc_sw128(qb + oq, 16, 1024), smem_desc_sw128(kb + ok, 16, sbo), idesc_n64,
-                 ks > 0);
-        }
+        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, a[ks], bb[ks], idesc_n64, ks > 0);
+        kmajor_from_base(a, do0 + (uint64_t)(i * (kQTile >> 4)), kQHalf >> 4);
+        kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, half_enc);
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t oq = (ks >> 2) * kQHalf + (ks & 3) * 32;
-          const uint32_t ok = (ks >> 2) * half_off + (ks & 3) * 32;
-          mma_ss(tmem + i * 128 + 64, smem_desc_sw128(db + oq, 16, 1024), smem_desc_sw128(vb + ok, 16, sbo),
-                 idesc_n64, ks > 0);
-        }
+        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128 + 64, a[ks], bb[ks], idesc_n64, ks > 0);
       };
       auto issue_dq = [&](int j, int i) {
-        const int s = j % KVS;
-        const bool routed = j < n_rt;
-        const uint32_t lbo = routed ? 1024u : kKVHalf;
-        const uint32_t sbo = routed ? 2048u : 1024u;
-        const uint32_t kb = sbase + L::kK + s * kKVTile;
+        const bool rt = j < n_rt;
+        const uint64_t soff = (uint64_t)((j % KVS) * (kKVTile >> 4));
+        uint64_t bb[4];
+        mnmajor_from_base<4>(bb, (rt ? kmn_rt : kmn_lc) + soff, rt ? (2 * 2048u) >> 4 : (2 * 1024u) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, smem_desc_sw128(kb + ks * 2 * sbo, lbo, sbo),
-                 idesc_dq, (j > 0 || ks > 0));
+        for (int ks = 0; ks < BN / 16; ++ks)   // dS of keys 32h..32h+31 sits in columns 32h..32h+15
+          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq,
+                 (j > 0 || ks > 0));
       };
       bool ok = mbar_wait(qdo_full, 0, abort_flag, p.status) && mbar_wait(kv_full(0), 0, abort_flag, p.status);
       if (ok) {
@@ -253,8 +254,10 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ======================= element-wise: dS = P o (dP - delta), one warpgroup per M-tile
-    const int i = (warp - 4) >> 2;
+    // ======================= element-wise: dS = P o (dP - delta); two warpgroups per M-tile,
+    // each owning 32 of the tile's 64 key columns (thread = TMEM lane = query row)
+    const int w4 = (warp - 4) >> 2;
+    const int i = w4 >> 1, hc = w4 & 1;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int head = h0 + 2 * i + (r >> 6);
@@ -278,21 +281,29 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
       }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sv[32], dv[32], pk[16];
-        tmem_ld32(tS + hh * 32, sv);
-        tmem_ld32(tP + hh * 32, dv);
-        tmem_wait_ld();
+      // one TMEM round trip per step: both loads in flight, one wait, compute, one store
+      uint32_t sv[32], dv[32], pk[16];
+      tmem_ld32(tS + 32 * hc, sv);
+      tmem_ld32(tP + 32 * hc, dv);
+      tmem_wait_ld();
+      const int c0 = 32 * hc;
+      if (nvalid >= BN) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int cidx = hh * 32 + e;
-          const float p0 = (cidx < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
-          const float p1 = (cidx + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
+          const float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2));
+          const float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2));
           pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
         }
-        tmem_st16(tS + hh * 16, pk);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = (c0 + e < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
+          const float p1 = (c0 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
+          pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
+        }
       }
+      // packed bf16 stays inside this warpgroup's own (already read) column range
+      tmem_st16(tS + 32 * hc, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_full(i));
@@ -300,11 +311,11 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(final_bar, 0, abort_flag, p.status));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + row * kD;
+      __nv_bfloat16* dst = p.dq + row * kD + 64 * hc;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32], pk[16];
-        tmem_ld32(tQ + cc * 32, v);
+        tmem_ld32(tQ + 64 * hc + cc * 32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
@@ -364,7 +375,7 @@ struct Smem {
   static constexpr uint32_t kBytes = kMisc + 16;
 };
 
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                    const Params p) {
@@ -406,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(sd_full(x), 1);
-      mbar_init(pd_full(x), 128);
+      mbar_init(pd_full(x), 256);
     }
     mbar_init(done, 1);
     mbar_init(mma_done, 1);
@@ -452,38 +463,41 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ======================= MMA issuer
+    // ======================= MMA issuer (one thread).  K and V are fixed for the CTA, so their
+    // descriptor arrays are built once; Q / dO stage descriptors come from prebuilt bases.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BQ, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(BM, kD, true);
+      uint64_t kd[8], vd[8];
+      kmajor_descs(kd, sbase + L::kK, kKHalf, 1024);
+      kmajor_descs(vd, sbase + L::kV, kKHalf, 1024);
+      // stage st is st * kQTileB bytes after stage 0 (descriptor units of 16 bytes)
+      const uint64_t q0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
+      const uint64_t do0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t qmn0 = smem_desc_sw128(sbase + L::kQ, kQHalfB, 1024);
+      const uint64_t domn0 = smem_desc_sw128(sbase + L::kDO, kQHalfB, 1024);
       auto issue_sd = [&](int i, int x) {
-        const int s = i % NS;
-        const uint32_t qb = sbase + L::kQ + s * kQTileB, db = sbase + L::kDO + s * kQTileB;
+        const uint64_t soff = (uint64_t)((i % NS) * (kQTileB >> 4));
+        uint64_t bb[8];
+        kmajor_from_base(bb, q0 + soff, kQHalfB >> 4);
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t ok_ = (ks >> 2) * kKHalf + (ks & 3) * 32;
-          const uint32_t oq = (ks >> 2) * kQHalfB + (ks & 3) * 32;
-          mma_ss(tmem + x * 128, smem_desc_sw128(sbase + L::kK + ok_, 16, 1024), smem_desc_sw128(qb + oq, 16, 1024),
-                 idesc_s, ks > 0);
-        }
+        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + x * 128, kd[ks], bb[ks], idesc_s, ks > 0);
+        kmajor_from_base(bb, do0 + soff, kQHalfB >> 4);
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t ok_ = (ks >> 2) * kKHalf + (ks & 3) * 32;
-          const uint32_t oq = (ks >> 2) * kQHalfB + (ks & 3) * 32;
-          mma_ss(tmem + x * 128 + 64, smem_desc_sw128(sbase + L::kV + ok_, 16, 1024),
-                 smem_desc_sw128(db + oq, 16, 1024), idesc_s, ks > 0);
-        }
+        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + x * 128 + 64, vd[ks], bb[ks], idesc_s, ks > 0);
       };
       auto issue_grad = [&](int i, int x) {
-        const int s = i % NS;
-        const uint32_t qb = sbase + L::kQ + s * kQTileB, db = sbase + L::kDO + s * kQTileB;
+        const uint64_t soff = (uint64_t)((i % NS) * (kQTileB >> 4));
+        // dV += P^T dO ; dK += dS^T Q  (B operands MN-major: 64-dim halves 8 KB apart, 8 rows 1 KB apart).
+        // P^T / dS^T of queries 32h..32h+31 sit in columns 32h..32h+15 of their region.
+        uint64_t b1[4], b2[4];
+        mnmajor_from_base<4>(b1, domn0 + soff, 2048u >> 4);
+        mnmajor_from_base<4>(b2, qmn0 + soff, 2048u >> 4);
 #pragma unroll
         for (int ks = 0; ks < BQ / 16; ++ks) {
-          // dV += P^T dO ; dK += dS^T Q  (B operands MN-major: 64-dim halves 8 KB apart, 8 rows 1 KB apart)
-          mma_ts(tmem + 256, tmem + x * 128 + ks * 8, smem_desc_sw128(db + ks * 2048, kQHalfB, 1024), idesc_g,
-                 (i > 0 || ks > 0));
-          mma_ts(tmem + 384, tmem + x * 128 + 64 + ks * 8, smem_desc_sw128(qb + ks * 2048, kQHalfB, 1024), idesc_g,
-                 (i > 0 || ks > 0));
+          const uint32_t acol = (ks >> 1) * 32 + (ks & 1) * 8;
+          mma_ts(tmem + 256, tmem + x * 128 + acol, b1[ks], idesc_g, (i > 0 || ks > 0));
+          mma_ts(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (i > 0 || ks > 0));
         }
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
@@ -515,8 +529,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ======================= element-wise: P^T, dS^T (warpgroup x takes query steps i = x mod 2)
-    const int x = (warp - 4) >> 2;
+    // ======================= element-wise: P^T, dS^T.  Warpgroup w4 = 0..3 takes the query steps
+    // i = w4 mod 2 and the 32 query columns 32*(w4/2) .. of each (thread = TMEM lane = key row).
+    const int w4 = (warp - 4) >> 2;
+    const int x = w4 & 1, hc = w4 >> 1;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;          // key row within the tile
     const int64_t u = (int64_t)m * BM + r;      // key position in the segment
@@ -535,38 +551,51 @@ __global__ void __launch_bounds__(384, 1)
       const float* lse = stat_base + s * (kStatBytes / 4);
       const float* dlt = lse + BQ;
       const int64_t t0 = (int64_t)(n0 + i) * BQ;
+      const bool diag = i < 2;                  // only the first two steps overlap the key tile
+      // one TMEM round trip per step: both loads in flight, one wait, compute, both stores
+      uint32_t sv[32], dv[32], pp[16], pd[16];
+      tmem_ld32(tS + 32 * hc, sv);
+      tmem_ld32(tP + 32 * hc, dv);
+      tmem_wait_ld();
+      const int q0 = 32 * hc;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sv[32], dv[32], pp[16], pd[16];
-        tmem_ld32(tS + hh * 32, sv);
-        tmem_ld32(tP + hh * 32, dv);
-        tmem_wait_ld();
+      for (int e = 0; e < 32; e += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse + q0 + e);
+        const float4 d4 = *reinterpret_cast<const float4*>(dlt + q0 + e);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+        float pr[4], dsr[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q0 = hh * 32 + e;
-          const bool v0 = u <= t0 + q0, v1 = u <= t0 + q0 + 1;
-          const float p0 = v0 ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse[q0] * kLog2e)) : 0.f;
-          const float p1 = v1 ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse[q0 + 1] * kLog2e)) : 0.f;
-          pp[e >> 1] = pack_bf16(p0, p1);
-          pd[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dlt[q0]), p1 * (__uint_as_float(dv[e + 1]) - dlt[q0 + 1]));
+        for (int f = 0; f < 4; ++f) {
+          float pv = ex2(fmaf(__uint_as_float(sv[e + f]), p.c2, -lv[f] * kLog2e));
+          if (diag && u > t0 + q0 + e + f) pv = 0.f;
+          pr[f] = pv;
+          dsr[f] = pv * (__uint_as_float(dv[e + f]) - dd[f]);
         }
-        tmem_st16(tS + hh * 16, pp);
-        tmem_st16(tP + hh * 16, pd);
+        pp[e >> 1] = pack_bf16(pr[0], pr[1]);
+        pp[(e >> 1) + 1] = pack_bf16(pr[2], pr[3]);
+        pd[e >> 1] = pack_bf16(dsr[0], dsr[1]);
+        pd[(e >> 1) + 1] = pack_bf16(dsr[2], dsr[3]);
       }
+      // packed bf16 stays inside this warpgroup's own (already read) column range
+      tmem_st16(tS + 32 * hc, pp);
+      tmem_st16(tP + 32 * hc, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(pd_full(x));
     }
-    // ---- epilogue: warpgroup 0 owns dV, warpgroup 1 owns dK; store this head's float32 partial
+    // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK;
+    // store this head's float32 partial
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
     if (ok) {
       tc_fence_after();
-      const uint32_t tacc = tmem + lane_off + (x == 0 ? 256 : 384);
+      const bool is_dk = w4 >= 2;
+      const int ch = w4 & 1;
+      const uint32_t tacc = tmem + lane_off + (is_dk ? 384 : 256) + 64 * ch;
       const size_t slot = (size_t)hin * p.B * p.Hkv * p.S * kD;
-      float* part = (x == 0 ? p.dv_part : p.dk_part) + slot + ((int64_t)bkh * p.S + u) * kD;
-      const float mul = (x == 0) ? 1.f : p.scale;
+      float* part = (is_dk ? p.dk_part : p.dv_part) + slot + ((int64_t)bkh * p.S + u) * kD + 64 * ch;
+      const float mul = is_dk ? p.scale : 1.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
         tmem_ld32(tacc + cc * 32, v);
         tmem_wait_ld();
@@ -648,12 +677,12 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
     const size_t smem = K::Smem<2>::kBytes + 1024;
     e = cudaFuncSetAttribute(K::dq_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    K::dq_tc_kernel<2><<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
+    K::dq_tc_kernel<2><<<(unsigned)grid, 640, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
   } else {
     const size_t smem = K::Smem<1>::kBytes + 1024;
     e = cudaFuncSetAttribute(K::dq_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    K::dq_tc_kernel<1><<<(unsigned)grid, 256, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
+    K::dq_tc_kernel<1><<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
   }
   return cudaGetLastError();
 }
@@ -679,7 +708,7 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  K::dkdv_tc_kernel<<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mks, mvs, p);
+  K::dkdv_tc_kernel<<<(unsigned)grid, 640, smem, st>>>(mq, mdo, mks, mvs, p);
   return cudaGetLastError();
 }
 

@@ -193,59 +193,58 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       for (int s = 0; s < NS; ++s)
         if (issued[s]) drain_wait(kv ? v_full(s) : k_full(s), (issued[s] - 1) & 1, p.status);
   } else if (warp == 1) {
-    // ======================= MMA issuer (one thread)
+    // ======================= MMA issuer (one thread).  All shared-memory descriptors are built
+    // before each unrolled MMA sequence, so the sequence issues back to back.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, true);
-      auto issue_s = [&](int j, int i) {
-        const int s = j % KS;
-        const bool routed = j < n_rt;
-        const uint32_t sbo = routed ? 2048u : 1024u;
-        const uint32_t half_off = routed ? 1024u : kHalfBytes;
-        const uint32_t kb = sbase + L::kK + s * kTileBytes;
-        const uint32_t qb = sbase + L::kQ + i * kTileBytes;
+      uint64_t qd[NT][8], kd[8], vd[8];
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off_q = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-          const uint32_t off_k = (ks >> 2) * half_off + (ks & 3) * 32;
-          mma_ss(tmem + i * 128, smem_desc_sw128(qb + off_q, 16, 1024), smem_desc_sw128(kb + off_k, 16, sbo),
-                 idesc_qk, ks > 0);
-        }
+      for (int i = 0; i < NT; ++i) kmajor_descs(qd[i], sbase + L::kQ + i * kTileBytes, kHalfBytes, 1024);
+      auto build_k = [&](int j) {
+        const bool routed = j < n_rt;
+        kmajor_descs(kd, sbase + L::kK + (j % KS) * kTileBytes, routed ? 1024u : kHalfBytes, routed ? 2048u : 1024u);
       };
-      auto issue_pv = [&](int j, int i) {
-        const int s = j % VS;
+      auto build_v = [&](int j) {
         const bool routed = j < n_rt;
-        const uint32_t lbo = routed ? 1024u : kHalfBytes;   // between 64-dim halves
-        const uint32_t sbo = routed ? 2048u : 1024u;        // between 8-key groups
-        const uint32_t vb = sbase + L::kV + s * kTileBytes;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, smem_desc_sw128(vb + ks * 2 * sbo, lbo, sbo),
-                 idesc_pv, (j > 0 || ks > 0));
-        }
+        mnmajor_descs<8>(vd, sbase + L::kV + (j % VS) * kTileBytes, routed ? 1024u : kHalfBytes,
+                         routed ? 2048u : 1024u);
       };
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full(0), 0, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
+        build_k(0);
+#pragma unroll
         for (int i = 0; i < NT; ++i) {
-          issue_s(0, i);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
           mma_commit(s_full(i));
         }
         mma_commit(k_empty(0));
       }
       for (int j = 0; ok && j < T; ++j) {
         ok = mbar_wait(v_full(j % VS), (j / VS) & 1, abort_flag, p.status);
-        for (int i = 0; ok && i < NT; ++i) {
+        if (!ok) break;
+        tc_fence_after();
+        build_v(j);
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
           ok = mbar_wait(p_full(i), j & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(j, i);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, vd[ks], idesc_pv, (j > 0 || ks > 0));
           if (j + 1 < T) {
             // the next K tile is only needed now, after this tile's first PV is queued
-            if (i == 0) ok = mbar_wait(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(j + 1, i);
+            if (i == 0) {
+              ok = mbar_wait(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+              build_k(j + 1);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
             mma_commit(s_full(i));
           }
         }
@@ -283,69 +282,60 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
       }
-      // pass 1: row max of the raw logits (the scale is positive), masking only where needed
-      float mx = -INFINITY;
+      // The whole 128-column row is loaded with one TMEM round trip and kept in registers.
+      uint32_t v[128];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+      tmem_wait_ld();
+      if (nvalid < BN) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tS + cc * 32, v);
-        tmem_wait_ld();
-        if (nvalid >= BN) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (cc * 32 + e < nvalid) mx = fmaxf(mx, __uint_as_float(v[e]));
-        }
+        for (int e = 0; e < BN; ++e)
+          if (e >= nvalid) v[e] = __float_as_uint(-INFINITY);
       }
-      mx *= p.scale_log2;
+      // row max of the raw logits (the scale is positive)
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < BN; e += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+        mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
+      }
+      const float mx = fmaxf(mx0, mx1) * p.scale_log2;
       // lazy rescale: move the reference max only when it grows by more than 2^8
       const bool need = mx > m + kRescaleThreshold || (m == -INFINITY && mx > -INFINITY);
       const float mnew = need ? mx : m;
       const float alpha = need ? ex2(m - mnew) : 1.f;   // m = -inf -> 0
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tO + cc * 32, v);
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st32(tO + cc * 32, v);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + cc * 32, o);
         }
       }
       l *= alpha;
       m = mnew;
       const float mref = (m == -INFINITY) ? 0.f : m;
-      // pass 2: probabilities, row sum, bf16 P into the first 64 columns of S
-      float rs = 0.f;
+      // probabilities (masked logits are -inf -> 0), row sum, bf16 P into the first 64 columns of S
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tS + cc * 32, v);
-        tmem_wait_ld();
         uint32_t pk[16];
-        if (nvalid >= BN) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref));
-            const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref));
-            rs += p0 + p1;
-            pk[e >> 1] = pack_bf16(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = (cc * 32 + e < nvalid) ? ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, -mref)) : 0.f;
-            const float p1 =
-                (cc * 32 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -mref)) : 0.f;
-            rs += p0 + p1;
-            pk[e >> 1] = pack_bf16(p0, p1);
-          }
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(v[cc * 32 + e]), p.scale_log2, -mref));
+          const float p1 = ex2(fmaf(__uint_as_float(v[cc * 32 + e + 1]), p.scale_log2, -mref));
+          rs0 += p0;
+          rs1 += p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
         }
         tmem_st16(tS + cc * 16, pk);
       }
+      const float rs = rs0 + rs1;
       l += rs;
       tmem_wait_st();
       tc_fence_before();

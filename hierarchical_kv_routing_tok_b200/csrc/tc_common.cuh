@@ -153,6 +153,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -188,6 +201,38 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// The 8 K-step descriptors (16 bf16 each) of a K-major [rows][128] bf16 operand stored as two
+// 128B-swizzled 64-dim halves half_bytes apart, 8-row groups sbo bytes apart.  Built once per
+// tile so that the MMA issue sequence itself does no descriptor arithmetic (which otherwise
+// dominates the single issuing thread's time).
+__device__ __forceinline__ void kmajor_descs(uint64_t (&d)[8], uint32_t saddr, uint32_t half_bytes, uint32_t sbo) {
+  const uint64_t base = smem_desc_sw128(saddr, 16, sbo);
+  const uint64_t hi = base + (uint64_t)(half_bytes >> 4);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) d[ks] = (ks < 4 ? base : hi) + (uint64_t)((ks & 3) * 2);
+}
+// The n K-step descriptors (16 rows each) of an MN-major operand: 64-element MN blocks lbo bytes
+// apart, 8-row K groups sbo bytes apart; K-step ks starts 2*ks groups in.
+template <int NK>
+__device__ __forceinline__ void mnmajor_descs(uint64_t (&d)[NK], uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  const uint64_t base = smem_desc_sw128(saddr, lbo, sbo);
+  const uint64_t step = (uint64_t)((2 * sbo) >> 4);
+#pragma unroll
+  for (int ks = 0; ks < NK; ++ks) d[ks] = base + (uint64_t)ks * step;
+}
+
+// Same as kmajor_descs, from a prebuilt base descriptor (half_enc = half_bytes >> 4).
+__device__ __forceinline__ void kmajor_from_base(uint64_t (&d)[8], uint64_t base, uint32_t half_enc) {
+  const uint64_t hi = base + (uint64_t)half_enc;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) d[ks] = (ks < 4 ? base : hi) + (uint64_t)((ks & 3) * 2);
+}
+template <int NK>
+__device__ __forceinline__ void mnmajor_from_base(uint64_t (&d)[NK], uint64_t base, uint32_t step_enc) {
+#pragma unroll
+  for (int ks = 0; ks < NK; ++ks) d[ks] = base + (uint64_t)ks * step_enc;
 }
 
 // Instruction descriptor of kind::f16: bf16 x bf16 -> f32, M x N, A K-major, B K- or MN-major.
