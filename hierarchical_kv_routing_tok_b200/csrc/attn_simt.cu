@@ -212,18 +212,41 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const T* __restrict__ q, 
 }
 
 // ------------------------------------------------------------------------------------ backward
+// delta[row] = sum_d dO[row, d] * O[row, d].  Each warp owns 8 rows and keeps all of their
+// 16-byte loads in flight at once (HBM-bound streaming kernel).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) bwd_delta_kernel(const T* __restrict__ o, const T* __restrict__ d_o,
                                                              float* __restrict__ delta, int64_t rows) {
-  const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+  constexpr int N = Vec16<T>::N;          // elements per 16-byte load
+  constexpr int LPR = kD / N;             // lanes per row
+  constexpr int RPW = 32 / LPR;           // rows per warp-wide load
+  constexpr int ROWS = 8;                 // rows per warp
+  constexpr int IT = ROWS / RPW;
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const float4 a = load4(o + row * kD + 4 * lane);
-  const float4 c = load4(d_o + row * kD + 4 * lane);
-  float s = a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+  const int64_t row0 = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * ROWS;
+  const int sub = lane / LPR, col = (lane % LPR) * N;
+  float a[IT][N], c[IT][N];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) delta[row] = s;
+  for (int it = 0; it < IT; ++it) {
+    const int64_t row = row0 + it * RPW + sub;
+    if (row < rows) {
+      Vec16<T>::load(o + row * kD + col, a[it]);
+      Vec16<T>::load(d_o + row * kD + col, c[it]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < N; ++e) a[it][e] = c[it][e] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < N; ++e) sum = fmaf(a[it][e], c[it][e], sum);
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const int64_t row = row0 + it * RPW + sub;
+    if ((lane % LPR) == 0 && row < rows) delta[row] = sum;
+  }
 }
 
 template <typename T>
@@ -392,7 +415,7 @@ cudaError_t fwd(const void* q, const void* kh, const void* vh, const void* ks, c
 template <typename T>
 cudaError_t bwd_delta(const void* o, const void* d_o, float* delta, int B, Dims dm, cudaStream_t st) {
   const int64_t rows = (int64_t)B * dm.Hq * dm.S;
-  bwd_delta_kernel<T><<<(unsigned)((rows + 7) / 8), kThreads, 0, st>>>(static_cast<const T*>(o),
+  bwd_delta_kernel<T><<<(unsigned)((rows + 63) / 64), kThreads, 0, st>>>(static_cast<const T*>(o),
                                                                        static_cast<const T*>(d_o), delta, rows);
   return cudaGetLastError();
 }

@@ -66,7 +66,7 @@ int check_config(const hga_config_t* c) {
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return HGA_ERR_ARG;
   // grid dimensions are 32-bit
   if ((int64_t)c->B * c->Hq * (c->seg_len / c->qblock) > INT32_MAX) return HGA_ERR_UNSUPPORTED;
-  if ((int64_t)c->B * c->Hkv * nch > (int64_t)INT32_MAX * 8) return HGA_ERR_UNSUPPORTED;
+  if ((int64_t)c->B * c->Hkv * nch > (int64_t)INT32_MAX) return HGA_ERR_UNSUPPORTED;   // one CTA per chunk
   if (hga::route_smem_bytes(c->dtype == HGA_BF16, (int)nch, c->top_chunks, c->top_groups) > kMaxRouteSmem)
     return HGA_ERR_UNSUPPORTED;
   return HGA_OK;

@@ -16,7 +16,8 @@
 
 namespace hga {
 
-constexpr int kRouteThreads = 256;
+constexpr int kRouteThreads = 512;
+constexpr int kScratchInts = 32;   // warp totals (16) + broadcast slots
 
 // Larger score -> larger key; +0 and -0 map to the same key.
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -55,9 +56,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 // Select the k largest keys[0..n) (ties: lower position first); write the selected
 // positions, ascending, to out[0..k).  All threads of the CTA must call it.
 __device__ void block_select_topk(const uint32_t* keys, int n, int k, int* out, int* hist,
-                                  int* scratch /* >= 8 + 4 ints */) {
+                                  int* scratch /* kScratchInts ints */) {
   int* warp_tot = scratch;
-  int* bcast = scratch + 8;
+  int* bcast = scratch + kRouteThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31;
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
@@ -130,18 +131,26 @@ __device__ void block_select_topk(const uint32_t* keys, int n, int k, int* out, 
 }
 
 // Select the k largest keys[0..n) for n <= kRouteThreads: thread i computes the rank of key i
-// (number of keys that precede it in the order "larger first, lower position first" -- compares
-// against broadcast shared-memory reads) and keeps it if rank < k; an index-ordered scan of the
-// kept flags writes the positions ascending.  One pass, two barriers.
+// (number of keys that precede it in the order "larger first, lower position first") by comparing
+// against broadcast 16-byte shared-memory reads of four keys at a time (keys[n..n4) hold 0, which
+// precedes nothing and is preceded by every score), keeps it if rank < k, and an index-ordered
+// scan of the kept flags writes the positions ascending.  One pass, two barriers.
 __device__ void block_select_topk_small(const uint32_t* keys, int n, int k, int* out, int* scratch) {
   const int i = threadIdx.x;
   bool take = false;
   if (i < n) {
     const uint32_t ki = keys[i];
+    const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+    const int n4 = (n + 3) >> 2;
     int rank = 0;
-    for (int j = 0; j < n; ++j) {
-      const uint32_t kj = keys[j];
-      rank += (kj > ki) | ((kj == ki) & (j < i));
+#pragma unroll 4
+    for (int j4 = 0; j4 < n4; ++j4) {
+      const uint4 v = k4[j4];
+      const int j = 4 * j4;
+      rank += (v.x > ki) | ((v.x == ki) & (j < i));
+      rank += (v.y > ki) | ((v.y == ki) & (j + 1 < i));
+      rank += (v.z > ki) | ((v.z == ki) & (j + 2 < i));
+      rank += (v.w > ki) | ((v.w == ki) & (j + 3 < i));
     }
     take = rank < k;
   }
@@ -182,7 +191,7 @@ __device__ __forceinline__ void score_rows(const float* qb, const float* __restr
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(
+__global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     const T* __restrict__ q, const float* __restrict__ group_sum, const float* __restrict__ chunk_sum,
     int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq, int Hkv, int64_t S, int nch,
     int kc, int kg) {
@@ -200,10 +209,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   float* red = reinterpret_cast<float*>(smem_raw);              // [RP][128]
   float* qb = red + RP * kD;                                      // [128]
   int* hist = reinterpret_cast<int*>(qb + kD);                    // [256]
-  int* scratch = hist + 256;                                      // [16]
-  int* csel = scratch + 16;                                       // [kc]
+  int* scratch = hist + 256;                                      // [kScratchInts]
+  int* csel = scratch + kScratchInts;                             // [kc]
   int* gpos = csel + ((kc + 3) & ~3);                             // [kg]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(gpos + ((kg + 3) & ~3));   // [max(nch, 8kc)]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(gpos + ((kg + 3) & ~3));   // [max(nch, 8kc) rounded to 4]
 
   // ---- block query: mean over G heads x 64 positions
   {
@@ -213,25 +222,27 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
 #pragma unroll
     for (int e = 0; e < N; ++e) acc[e] = 0.f;
     const int R = G * kQBlock;
-    constexpr int UQ = 8;                        // loads in flight per thread
+    constexpr int UQ = 8;                        // 16-byte loads in flight per thread
     for (int r1 = r0; r1 < R; r1 += UQ * RP) {
-      float v[UQ][N];
+      uint4 raw[UQ];                             // kept packed until accumulation (register budget)
 #pragma unroll
       for (int u = 0; u < UQ; ++u) {
         const int r = r1 + u * RP;
         if (r < R) {
           const int h = kh * G + r / kQBlock;
           const int64_t t = (int64_t)n * kQBlock + r % kQBlock;
-          Vec16<T>::load(q + (((int64_t)b * Hq + h) * S + t) * kD + col, v[u]);
+          raw[u] = *reinterpret_cast<const uint4*>(q + (((int64_t)b * Hq + h) * S + t) * kD + col);
         } else {
-#pragma unroll
-          for (int e = 0; e < N; ++e) v[u][e] = 0.f;
+          raw[u] = make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
-      for (int u = 0; u < UQ; ++u)
+      for (int u = 0; u < UQ; ++u) {
+        float v[N];
+        Vec16<T>::load(reinterpret_cast<const T*>(&raw[u]), v);
 #pragma unroll
-        for (int e = 0; e < N; ++e) acc[e] += v[u][e];
+        for (int e = 0; e < N; ++e) acc[e] += v[e];
+      }
     }
 #pragma unroll
     for (int e = 0; e < N; ++e) red[r0 * kD + col + e] = acc[e];
@@ -247,6 +258,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   // ---- level 1: chunks
   const float* cs = chunk_sum + (int64_t)bkh * nch * kD;
   score_rows(qb, cs, nch, [](int i) { return i; }, keys);
+  if (threadIdx.x < 4 && nch + (int)threadIdx.x < ((nch + 3) & ~3)) keys[nch + threadIdx.x] = 0u;
   __syncthreads();
   if (nch <= kRouteThreads)
     block_select_topk_small(keys, nch, kc, csel, scratch);
@@ -257,6 +269,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   const float* gs = group_sum + (int64_t)bkh * nch * (kChunk / kGroup) * kD;
   const int ncand = kc * (kChunk / kGroup);
   score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
+  if (threadIdx.x < 4 && ncand + (int)threadIdx.x < ((ncand + 3) & ~3)) keys[ncand + threadIdx.x] = 0u;
   __syncthreads();
   if (ncand <= kRouteThreads)
     block_select_topk_small(keys, ncand, kg, gpos, scratch);
@@ -270,8 +283,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
 
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
   const int RP = kRouteThreads / (kD / (bf16 ? 8 : 4));
-  size_t words = (size_t)RP * kD + kD + 256 + 16 + ((kc + 3) & ~3) + ((kg + 3) & ~3) +
-                 (size_t)(nch > 8 * kc ? nch : 8 * kc);
+  size_t words = (size_t)RP * kD + kD + 256 + kScratchInts + ((kc + 3) & ~3) + ((kg + 3) & ~3) +
+                 (size_t)(((nch > 8 * kc ? nch : 8 * kc) + 3) & ~3);
   return words * 4;
 }
 
