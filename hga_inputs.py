@@ -159,4 +159,12 @@ EDGE_WORKLOADS = {
     "dense_tiny_f32": WORKLOADS["tiny_f32"].with_(name="dense_tiny_f32", top_chunks=16, top_groups=128),
     # maximal group budget for the chosen chunks (k_g = 8 k_c), bf16
     "max_groups_bf16": WORKLOADS["small_bf16"].with_(name="max_groups_bf16", B=1, top_groups=32),
+    # two query heads per KV head (one 128-row query tile per CTA), 7 query blocks (a ragged
+    # 64-key last tile of the dK/dV kernel), 20 groups = 160 routed keys (ragged routed tiles), bf16
+    "gqa2_ragged_bf16": Workload("gqa2_ragged_bf16", 1, 4, 2, 128, 1024, 448, 3, 20, "bf16", 1.0),
+    # eight query heads per KV head (two CTAs per query block), 5 query blocks, bf16
+    "gqa8_bf16": Workload("gqa8_bf16", 1, 8, 1, 128, 512, 320, 4, 12, "bf16", 1.0),
+    # many (batch, KV head) units of short segments: as many dK/dV key tiles as SMs or more, so
+    # every CTA sums all of its KV head's query heads alone; ragged 64-key last tile, bf16
+    "wide_bf16": Workload("wide_bf16", 16, 16, 8, 128, 256, 192, 2, 8, "bf16", 1.0),
 }

@@ -13,12 +13,12 @@
 //   (128 columns) of both tiles fit the 512 TMEM columns.  Two element-wise warpgroups per M-tile
 //   each own 32 key columns; each packs its dS to bf16 into the first 16 of its own 32 S columns,
 //   and dQ_i += dS_i K reads them from TMEM.
-// dkdv_tc_kernel: one CTA per (batch, KV head, 128-key tile, query head); keys are the M
-//   dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
-//   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  Each of the G query-head
-//   CTAs of one key tile stores its float32 partial dK / dV into its own workspace slot; the last
-//   one to finish (atomic ticket) sums the G slots in head order -- so the result does not depend
-//   on which CTA finishes first -- writes the output type and resets the ticket to zero.
+// dkdv_tc_kernel: one CTA (or a cluster of two) per (batch, KV head, 128-key tile); keys are the
+//   M dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
+//   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  The G query heads of the
+//   KV head accumulate into the same TMEM dK / dV, one head after another; in a cluster of two each
+//   CTA takes G/2 heads and the two float32 tiles are added through distributed shared memory (one
+//   bulk copy each way), so no partial sums go through HBM and the result is reproducible.
 // Warp roles as in the forward: warp 0 TMA, warp 1 TMEM owner + single-thread MMA issuer,
 // warps 4.. element-wise warpgroups (thread = TMEM lane = row; two warpgroups split each tile's
 // columns so that each thread handles 32 elements per step).  All mbarrier waits are bounded.
@@ -347,16 +347,17 @@ constexpr uint32_t kKHalf = BM * 128;       // 16 KB
 constexpr uint32_t kQTileB = BQ * 256;      // 16 KB
 constexpr uint32_t kQHalfB = BQ * 128;      // 8 KB
 constexpr uint32_t kStatBytes = 2 * BQ * 4; // lse[64], delta[64]
+constexpr uint32_t kAccRow = 2 * kD * 4;    // one key's float32 dV | dK row in the reduction buffer
 
 struct Params {
-  int B, Hq, Hkv, G, nblk, nkt;
+  int B, Hq, Hkv, G;
+  int cs;               // CTAs per cluster (1 or 2): the query heads of one KV head are split over them
+  int hpc;              // query heads per CTA (G = cs * hpc), accumulated in TMEM one after another
+  int nblk, nkt;
   int64_t S;
   float c2, scale;
   const float* lse;
   const float* delta;
-  float* dk_part;       // [G][B*Hkv*S][128] float32 partials, one slot per query head of the group
-  float* dv_part;
-  int* ticket;          // [B*Hkv][nkt]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int* status;
@@ -369,11 +370,24 @@ struct Smem {
   static constexpr uint32_t kDO = kQ + NS * kQTileB;
   static constexpr uint32_t kStat = kDO + NS * kQTileB;
   static constexpr uint32_t kBar = kStat + NS * kStatBytes;
-  // kv_full, q_full[NS], q_empty[NS], sd_full[2], pd_full[2], done, mma_done
-  static constexpr int kNumBars = 1 + 2 * NS + 4 + 2;
+  // kv_full, q_full[NS], q_empty[NS], sd_full[2], pd_full[2], done, mma_done, recv
+  static constexpr int kNumBars = 1 + 2 * NS + 4 + 3;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
+  // After the main loop the K, V and Q/dO stage area holds this CTA's float32 dV | dK tile (kAcc)
+  // and, in a cluster of two, the peer's half of its tile for the rows this CTA writes (kRecv).
+  static constexpr uint32_t kAcc = 0;
+  static constexpr uint32_t kRecv = kAcc + BM * kAccRow;
+  static constexpr uint32_t kHalfBytes = (BM / 2) * kAccRow;
+  static_assert(kRecv + kHalfBytes <= kStat, "reduction buffers must not reach the stats or barriers");
 };
+
+// Byte offset of the float4 chunk c16 (0..63: dV columns 0..127, then dK) of key row r in the
+// reduction buffer.  The chunk index is XOR-swizzled by r mod 8 so that a warp writing one
+// chunk of 32 rows, and 16 threads reading consecutive chunks of one row, hit distinct banks.
+__device__ __forceinline__ uint32_t acc_off(int r, int c16) {
+  return (uint32_t)r * kAccRow + ((uint32_t)(c16 ^ (r & 7)) << 4);
+}
 
 __global__ void __launch_bounds__(640, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -392,22 +406,22 @@ __global__ void __launch_bounds__(640, 1)
   auto pd_full = [&](int b) { return BAR(3 + 2 * NS + b); };
   const uint32_t done = BAR(5 + 2 * NS);
   const uint32_t mma_done = BAR(6 + 2 * NS);
+  const uint32_t recv_bar = BAR(7 + 2 * NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- unit decode: key tile m (heavy = early first), batch x KV head, query head
-  int c = blockIdx.x;
-  const int hin = c % p.G;
-  c /= p.G;
+  // ---- unit decode: key tile m (heavy = early first), batch x KV head, rank in the cluster
+  // (the cluster's cs CTAs are consecutive blocks and share one key tile)
+  const int crank = (int)cluster_rank();
+  const int c = blockIdx.x / p.cs;
   const int bkh = c % (p.B * p.Hkv);
   const int m = c / (p.B * p.Hkv);
   const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
-  const int head = kh * p.G + hin;
+  const int head0 = kh * p.G + crank * p.hpc;
   const int n0 = 2 * m;                       // first query block that sees this key tile
-  const int Tq = p.nblk - n0;
-  const int64_t qrow0 = ((int64_t)b * p.Hq + head) * p.S;
+  const int Tq = p.nblk - n0;                 // query steps per head
+  const int NJ = p.hpc * Tq;                  // steps of this CTA: head-major, then query block
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -421,8 +435,8 @@ __global__ void __launch_bounds__(640, 1)
     }
     mbar_init(done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(recv_bar, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -444,11 +458,12 @@ __global__ void __launch_bounds__(640, 1)
       tma_load_2d(sbase + L::kV, &tm_vs, 0, krow, kv_full);
       tma_load_2d(sbase + L::kV + kKHalf, &tm_vs, 64, krow, kv_full);
       int issued[NS] = {0, 0, 0, 0};
-      for (int i = 0; i < Tq; ++i) {
-        const int s = i % NS;
-        if (!mbar_wait(q_empty(s), ((i / NS) & 1) ^ 1, abort_flag, p.status)) break;
+      for (int j = 0; j < NJ; ++j) {
+        const int s = j % NS;
+        const int t = j / Tq, i = j - t * Tq;
+        if (!mbar_wait(q_empty(s), ((j / NS) & 1) ^ 1, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(q_full(s), 2 * kQTileB + kStatBytes);
-        const int64_t row = qrow0 + (int64_t)(n0 + i) * BQ;
+        const int64_t row = ((int64_t)b * p.Hq + head0 + t) * p.S + (int64_t)(n0 + i) * BQ;
         tma_load_2d(sbase + L::kQ + s * kQTileB, &tm_q, 0, (int32_t)row, q_full(s));
         tma_load_2d(sbase + L::kQ + s * kQTileB + kQHalfB, &tm_q, 64, (int32_t)row, q_full(s));
         tma_load_2d(sbase + L::kDO + s * kQTileB, &tm_do, 0, (int32_t)row, q_full(s));
@@ -476,8 +491,8 @@ __global__ void __launch_bounds__(640, 1)
       const uint64_t do0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
       const uint64_t qmn0 = smem_desc_sw128(sbase + L::kQ, kQHalfB, 1024);
       const uint64_t domn0 = smem_desc_sw128(sbase + L::kDO, kQHalfB, 1024);
-      auto issue_sd = [&](int i, int x) {
-        const uint64_t soff = (uint64_t)((i % NS) * (kQTileB >> 4));
+      auto issue_sd = [&](int j, int x) {
+        const uint64_t soff = (uint64_t)((j % NS) * (kQTileB >> 4));
         uint64_t bb[8];
         kmajor_from_base(bb, q0 + soff, kQHalfB >> 4);
 #pragma unroll
@@ -486,8 +501,8 @@ __global__ void __launch_bounds__(640, 1)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + x * 128 + 64, vd[ks], bb[ks], idesc_s, ks > 0);
       };
-      auto issue_grad = [&](int i, int x) {
-        const uint64_t soff = (uint64_t)((i % NS) * (kQTileB >> 4));
+      auto issue_grad = [&](int j, int x) {
+        const uint64_t soff = (uint64_t)((j % NS) * (kQTileB >> 4));
         // dV += P^T dO ; dK += dS^T Q  (B operands MN-major: 64-dim halves 8 KB apart, 8 rows 1 KB apart).
         // P^T / dS^T of queries 32h..32h+31 sit in columns 32h..32h+15 of their region.
         uint64_t b1[4], b2[4];
@@ -496,30 +511,30 @@ __global__ void __launch_bounds__(640, 1)
 #pragma unroll
         for (int ks = 0; ks < BQ / 16; ++ks) {
           const uint32_t acol = (ks >> 1) * 32 + (ks & 1) * 8;
-          mma_ts(tmem + 256, tmem + x * 128 + acol, b1[ks], idesc_g, (i > 0 || ks > 0));
-          mma_ts(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (i > 0 || ks > 0));
+          mma_ts(tmem + 256, tmem + x * 128 + acol, b1[ks], idesc_g, (j > 0 || ks > 0));
+          mma_ts(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (j > 0 || ks > 0));
         }
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
-      for (int i = 0; ok && i < 2 && i < Tq; ++i) {
-        ok = mbar_wait(q_full(i % NS), (i / NS) & 1, abort_flag, p.status);
+      for (int j = 0; ok && j < 2 && j < NJ; ++j) {
+        ok = mbar_wait(q_full(j % NS), (j / NS) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        issue_sd(i, i & 1);
-        mma_commit(sd_full(i & 1));
+        issue_sd(j, j & 1);
+        mma_commit(sd_full(j & 1));
       }
-      for (int i = 0; ok && i < Tq; ++i) {
-        const int x = i & 1;
-        ok = mbar_wait(pd_full(x), (i >> 1) & 1, abort_flag, p.status);
+      for (int j = 0; ok && j < NJ; ++j) {
+        const int x = j & 1;
+        ok = mbar_wait(pd_full(x), (j >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        issue_grad(i, x);
-        mma_commit(q_empty(i % NS));
-        if (i + 2 < Tq) {
-          ok = mbar_wait(q_full((i + 2) % NS), ((i + 2) / NS) & 1, abort_flag, p.status);
+        issue_grad(j, x);
+        mma_commit(q_empty(j % NS));
+        if (j + 2 < NJ) {
+          ok = mbar_wait(q_full((j + 2) % NS), ((j + 2) / NS) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          issue_sd(i + 2, x);
+          issue_sd(j + 2, x);
           mma_commit(sd_full(x));
         }
       }
@@ -529,8 +544,8 @@ __global__ void __launch_bounds__(640, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ======================= element-wise: P^T, dS^T.  Warpgroup w4 = 0..3 takes the query steps
-    // i = w4 mod 2 and the 32 query columns 32*(w4/2) .. of each (thread = TMEM lane = key row).
+    // ======================= element-wise: P^T, dS^T.  Warpgroup w4 = 0..3 takes the steps
+    // j = w4 mod 2 and the 32 query columns 32*(w4/2) .. of each (thread = TMEM lane = key row).
     const int w4 = (warp - 4) >> 2;
     const int x = w4 & 1, hc = w4 >> 1;
     const int quarter = warp & 3;
@@ -541,10 +556,11 @@ __global__ void __launch_bounds__(640, 1)
     const uint32_t tP = tS + 64;
     const float* stat_base = reinterpret_cast<const float*>(smem + L::kStat);
     bool ok = true;
-    for (int i = x; i < Tq; i += 2) {
-      const int s = i % NS;
-      ok = mbar_wait(sd_full(x), (i >> 1) & 1, abort_flag, p.status);
-      if (ok) ok = mbar_wait(q_full(s), (i / NS) & 1, abort_flag, p.status);   // stats landed
+    for (int j = x; j < NJ; j += 2) {
+      const int s = j % NS;
+      const int i = j % Tq;
+      ok = mbar_wait(sd_full(x), (j >> 1) & 1, abort_flag, p.status);
+      if (ok) ok = mbar_wait(q_full(s), (j / NS) & 1, abort_flag, p.status);   // stats landed
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -583,31 +599,29 @@ __global__ void __launch_bounds__(640, 1)
       tc_fence_before();
       mbar_arrive(pd_full(x));
     }
-    // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK;
-    // store this head's float32 partial
+    // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK.
+    // After `done` every MMA has completed, so the K, V and Q/dO stage area is free: this CTA's
+    // float32 tile (the sum over its hpc heads) goes there for the reduction and the store.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
     if (ok) {
       tc_fence_after();
       const bool is_dk = w4 >= 2;
       const int ch = w4 & 1;
       const uint32_t tacc = tmem + lane_off + (is_dk ? 384 : 256) + 64 * ch;
-      const size_t slot = (size_t)hin * p.B * p.Hkv * p.S * kD;
-      float* part = (is_dk ? p.dk_part : p.dv_part) + slot + ((int64_t)bkh * p.S + u) * kD + 64 * ch;
       const float mul = is_dk ? p.scale : 1.f;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
         tmem_ld32(tacc + cc * 32, v);
         tmem_wait_ld();
-        if (u < p.S) {
+        const int c16 = (is_dk ? 32 : 0) + 16 * ch + 8 * cc;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            __stcg(reinterpret_cast<float4*>(part + cc * 32 + e),
-                   make_float4(__uint_as_float(v[e]) * mul, __uint_as_float(v[e + 1]) * mul,
-                               __uint_as_float(v[e + 2]) * mul, __uint_as_float(v[e + 3]) * mul));
-        }
+        for (int e = 0; e < 32; e += 4)
+          st_smem_f4(sbase + L::kAcc + acc_off(r, c16 + e / 4), __uint_as_float(v[e]) * mul,
+                     __uint_as_float(v[e + 1]) * mul, __uint_as_float(v[e + 2]) * mul,
+                     __uint_as_float(v[e + 3]) * mul);
       }
-      __threadfence();
+      fence_proxy_async_smem();   // the tile is read by a bulk copy below
     }
   }
   tc_fence_before();
@@ -616,46 +630,54 @@ __global__ void __launch_bounds__(640, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  // ---- the last of the G query-head CTAs of this key tile converts and clears it
-  if (*abort_flag) return;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    int* tk = p.ticket + (int64_t)bkh * p.nkt + m;
-    const int prev = atomicAdd(tk, 1);
-    if (prev == p.G - 1) {
-      *tk = 0;
-      *last_flag = 1;
+  // ---- reduction over the query heads of this KV head and store.  In a cluster of two, CTA
+  // `crank` writes key rows [64 crank, 64 crank + 64): after a cluster barrier (both CTAs have left
+  // their main loops, so the peer's stage area is free) each CTA pushes the peer's rows of its tile
+  // into the peer's kRecv with one bulk copy, then adds the received rows to its own.  A sum of two
+  // terms does not depend on their order, so the result is reproducible.  Every thread takes
+  // part on the error path too; a CTA that gave up leaves an arbitrary tile and the status word
+  // says so.
+  const int nrows = BM / p.cs;
+  const int r0 = crank * nrows;
+  if (p.cs == 2) {
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, L::kHalfBytes);
+    cluster_sync();
+    if (threadIdx.x == 0) {
+      const uint32_t peer = (uint32_t)(crank ^ 1);
+      bulk_copy_to_peer(dsmem_addr(sbase + L::kRecv, peer), sbase + L::kAcc + peer * L::kHalfBytes, L::kHalfBytes,
+                        dsmem_addr(recv_bar, peer));
+      bulk_commit_group();
+    }
+    drain_wait(recv_bar, 0, p.status);
+  }
+  {
+    const int r1 = (int)min((int64_t)(r0 + nrows), p.S - (int64_t)m * BM);
+    const int nitems = max(0, r1 - r0) * 32;  // per row: dV and dK, 16 chunks of 8 columns each
+    const int64_t key0 = (int64_t)bkh * p.S + (int64_t)m * BM;
+    for (int it = threadIdx.x; it < nitems; it += blockDim.x) {
+      const int pr = it & 15, is_dk = (it >> 4) & 1, rr = r0 + (it >> 5);
+      const int c16 = is_dk * 32 + 2 * pr;
+      float4 a = *reinterpret_cast<const float4*>(smem + L::kAcc + acc_off(rr, c16));
+      float4 a2 = *reinterpret_cast<const float4*>(smem + L::kAcc + acc_off(rr, c16 + 1));
+      if (p.cs == 2) {   // received rows keep the row's swizzle: (rr - r0) mod 8 == rr mod 8
+        const float4 x0 = *reinterpret_cast<const float4*>(smem + L::kRecv + acc_off(rr - r0, c16));
+        const float4 x1 = *reinterpret_cast<const float4*>(smem + L::kRecv + acc_off(rr - r0, c16 + 1));
+        a.x += x0.x; a.y += x0.y; a.z += x0.z; a.w += x0.w;
+        a2.x += x1.x; a2.y += x1.y; a2.z += x1.z; a2.w += x1.w;
+      }
+      __nv_bfloat16* dst = (is_dk ? p.dk : p.dv) + (key0 + rr) * kD + 8 * pr;
+      *reinterpret_cast<uint4*>(dst) =
+          make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(a2.x, a2.y), pack_bf16(a2.z, a2.w));
     }
   }
-  __syncthreads();
-  if (!*last_flag) return;
-  __threadfence();
-  const int64_t key0 = (int64_t)bkh * p.S + (int64_t)m * BM;
-  const int64_t nkeys = min((int64_t)BM, p.S - (int64_t)m * BM);
-  const size_t slot = (size_t)p.B * p.Hkv * p.S * kD;
-  for (int64_t e = (int64_t)threadIdx.x * 4; e < nkeys * kD; e += (int64_t)blockDim.x * 4) {
-    float4 ks = make_float4(0.f, 0.f, 0.f, 0.f), vs = ks;
-    for (int h = 0; h < p.G; ++h) {                 // fixed order: bitwise reproducible
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(p.dk_part + h * slot + key0 * kD + e));
-      const float4 c4 = __ldcg(reinterpret_cast<const float4*>(p.dv_part + h * slot + key0 * kD + e));
-      ks.x += a.x; ks.y += a.y; ks.z += a.z; ks.w += a.w;
-      vs.x += c4.x; vs.y += c4.y; vs.z += c4.z; vs.w += c4.w;
-    }
-    store4(p.dk + key0 * kD + e, ks);
-    store4(p.dv + key0 * kD + e, vs);
-  }
+  // the outgoing copy must have finished reading this CTA's shared memory before the CTA exits
+  if (p.cs == 2 && threadIdx.x == 0) bulk_wait_read_all();
 }
 
 }  // namespace dkdv
 }  // namespace tcbwd
 
 // ------------------------------------------------------------------ host side
-size_t bwd_tc_acc_bytes(int B, int Hq, int Hkv, int64_t S) {
-  const int64_t nkt = (S + tcbwd::dkdv::BM - 1) / tcbwd::dkdv::BM;
-  const int G = Hq / Hkv;
-  return 2 * (size_t)G * B * Hkv * S * kD * sizeof(float) + (size_t)B * Hkv * nkt * sizeof(int);
-}
-
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
                              int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
@@ -687,9 +709,21 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
   return cudaGetLastError();
 }
 
+// CTAs per cluster of the dK/dV kernel.  With one CTA per (batch, KV head, key tile) every CTA
+// sums all G query heads in TMEM and no reduction is needed; when that gives fewer CTAs than the GPU
+// has SMs (and G is even) the heads are split over a cluster of two.  (Clusters of four CTAs of one
+// SM each leave SMs of the graphics processing clusters idle and measured slower.)
+int dkdv_cluster_size(int B, int Hkv, int G, int nkt) {
+  if (G % 2 != 0) return 1;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  return ((int64_t)B * Hkv * nkt >= sms) ? 1 : 2;
+}
+
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
-                               const float* delta, void* dk, void* dv, void* acc, int B, int Hq, int Hkv, int64_t S,
-                               float scale, int* status, cudaStream_t st) {
+                               const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
+                               int* status, cudaStream_t st) {
   namespace K = tcbwd::dkdv;
   CUtensorMap mq, mdo, mks, mvs;
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, K::BQ) ||
@@ -698,17 +732,28 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BM))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
+  const int cs = dkdv_cluster_size(B, Hkv, G, (int)((S + K::BM - 1) / K::BM));
   const int nkt = (int)((S + K::BM - 1) / K::BM);
-  float* dk_part = static_cast<float*>(acc);
-  float* dv_part = dk_part + (size_t)G * B * Hkv * S * kD;
-  int* ticket = reinterpret_cast<int*>(dv_part + (size_t)G * B * Hkv * S * kD);
-  K::Params p{B, Hq, Hkv, G, (int)(S / kQBlock), nkt, S, scale * tcbwd::kLog2e, scale, lse, delta, dk_part, dv_part,
-              ticket, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), status};
-  const int64_t grid = (int64_t)B * Hkv * nkt * G;
+  K::Params p{B, Hq, Hkv, G, cs, G / cs, (int)(S / kQBlock), nkt, S, scale * tcbwd::kLog2e, scale, lse, delta,
+              static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), status};
+  const int64_t grid = (int64_t)B * Hkv * nkt * cs;
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  K::dkdv_tc_kernel<<<(unsigned)grid, 640, smem, st>>>(mq, mdo, mks, mvs, p);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)grid);
+  lc.blockDim = dim3(640);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, K::dkdv_tc_kernel, mq, mdo, mks, mvs, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -23,14 +23,13 @@ bool attn_fwd_tc_supported(int Hq, int Hkv);
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
                                int kg, float scale, int* status, cudaStream_t st);
-size_t bwd_tc_acc_bytes(int B, int Hq, int Hkv, int64_t S);
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
                              int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
                              cudaStream_t st);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
-                               const float* delta, void* dk, void* dv, void* acc, int B, int Hq, int Hkv, int64_t S,
-                               float scale, int* status, cudaStream_t st);
+                               const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
+                               int* status, cudaStream_t st);
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
@@ -96,25 +95,20 @@ bool force_cuda_cores() {
 // The workspace starts with the status word.
 int* status_of(void* workspace) { return static_cast<int*>(workspace); }
 
-// Workspace layout: [status word | delta rows (float32) | dK, dV accumulators (float32) and
-// per-key-tile tickets of the tensor-core dK/dV kernel].
+// Workspace layout: [status word | delta rows (float32)].
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t delta_bytes(const hga_config_t* c) { return (size_t)c->B * c->Hq * c->seg_len * sizeof(float); }
 float* delta_of(void* workspace) {
   return reinterpret_cast<float*>(static_cast<char*>(workspace) + hga::kStatusBytes);
 }
-size_t acc_offset(const hga_config_t* c) { return hga::kStatusBytes + round256(delta_bytes(c)); }
-void* acc_of(void* workspace, const hga_config_t* c) { return static_cast<char*>(workspace) + acc_offset(c); }
-size_t full_workspace_bytes(const hga_config_t* c) {
-  return acc_offset(c) + round256(hga::bwd_tc_acc_bytes(c->B, c->Hq, c->Hkv, c->seg_len));
-}
+size_t full_workspace_bytes(const hga_config_t* c) { return hga::kStatusBytes + round256(delta_bytes(c)); }
 
 // The tensor-core attention kernels handle bf16 with an even number of query heads per KV head.
 bool use_tc(const hga_config_t* c) {
   return c->dtype == HGA_BF16 && hga::attn_fwd_tc_supported(c->Hq, c->Hkv) && !force_cuda_cores();
 }
 
-// dK/dV with a workspace of ws_bytes: the tensor-core kernel needs the accumulator region.
+// dK/dV with a workspace of ws_bytes (status word and delta rows).
 int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const void* v_seg, const float* lse,
                 const void* d_o, void* dk_seg, void* dv_seg, void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg});
@@ -122,10 +116,11 @@ int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (use_tc(cfg) && ws_bytes >= full_workspace_bytes(cfg))
-    return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg,
-                                             acc_of(workspace, cfg), cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
-                                             eff_scale(cfg), status_of(workspace), st));
+  if (ws_bytes < full_workspace_bytes(cfg)) return HGA_ERR_WORKSPACE;
+  if (use_tc(cfg))
+    return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg, cfg->B,
+                                             cfg->Hq, cfg->Hkv, cfg->seg_len, eff_scale(cfg), status_of(workspace),
+                                             st));
   return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
                                              dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
                                              cfg->top_groups, eff_scale(cfg), st));

@@ -52,7 +52,7 @@ extern "C" int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, cons
   // the status word must start at zero; delta is fully rewritten by the first kernel
   if (cudaMemsetAsync(scratch, 0, hga::kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return HGA_ERR_CUDA;
-  // kernels that need more scratch than the fixed array holds fall back to the CUDA-core ones
+  // the fixed array holds the status word and B*Hq*S delta rows: the whole workspace of this problem
   return hga_internal_attn_bwd_ws(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg,
                                   scratch, kScratchBytes, stream);
 }

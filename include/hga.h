@@ -38,13 +38,10 @@
  *     happen before anything is launched; on an error nothing is launched
  *     and no output is touched.  HGA_ERR_CUDA reports a launch failure.
  *   - Workspace: at least hga_workspace_size() bytes of device memory, zero-
- *     filled once before its first use (cudaMemset); every successful call
- *     leaves what must start at zero at zero again.  Layout:
- *     a 256-byte sticky status word (read and cleared by hga_read_status()),
- *     the backward's delta rows (B*Hq*S float32), then per-query-head float32
- *     dK / dV partials and per-key-tile counters of the tensor-core dK/dV
- *     kernel (the counters must start at zero; the kernel resets them).  After a call reports an error the workspace must be zero-filled
- *     again before reuse.  Kernels that wait on on-chip barriers give up after
+ *     filled once before its first use (cudaMemset).  Layout: a 256-byte
+ *     sticky status word (must start at zero; read and cleared by
+ *     hga_read_status()), then the backward's delta rows (B*Hq*S float32,
+ *     written before they are read).  Kernels that wait on on-chip barriers give up after
  *     a bounded time and record HGA_ERR_TIMEOUT there instead of hanging; an
  *     attention kernel given a group index outside [0, H/8) reads that group
  *     as zeros (never out of bounds) and records HGA_ERR_ARG there.

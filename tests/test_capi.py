@@ -68,8 +68,7 @@ def cfg(**kw):
 def _expected_ws(B, Hq, Hkv, S):
     r256 = lambda x: (x + 255) // 256 * 256
     delta = B * Hq * S * 4
-    acc = 2 * Hq * B * S * 128 * 4 + B * Hkv * ((S + 127) // 128) * 4    # G fp32 dK, dV slots + tickets
-    return 256 + r256(delta) + r256(acc)
+    return 256 + r256(delta)
 
 
 def test_workspace_size(lib):
