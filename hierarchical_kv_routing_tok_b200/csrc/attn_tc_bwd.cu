@@ -7,12 +7,11 @@
 // P = exp(S - lse), dP = dO V^T, dS = P o (dP - delta), dQ = scale dS K, dK = scale dS^T Q,
 // dV = P^T dO.
 //
-// dq_tc_kernel: one CTA per (batch, KV head, query block, 4 query heads) = two M=128 query tiles
-//   sharing one routed key set, as in the forward.  Key tiles of 64 keys (routed: 8 groups of 8
-//   history rows; local: 64 segment rows) so that S_i, dP_i (64 fp32 columns each) and dQ_i
-//   (128 columns) of both tiles fit the 512 TMEM columns.  Two element-wise warpgroups per M-tile
-//   each own 32 key columns; each packs its dS to bf16 into the first 16 of its own 32 S columns,
-//   and dQ_i += dS_i K reads them from TMEM.
+// dq_tc_kernel: one CTA per (batch, KV head, query block, pair of query heads) = one M=128 query
+//   tile.  Key tiles of 128 keys (routed: 16 groups of 8 history rows; local: 128 segment rows), so
+//   that every MMA has N = 128.  TMEM: S double-buffered, dP, dQ (4 x 128 columns).  The
+//   element-wise warps load S(j) and dP(j) once, release dP for dP(j+1), and pack bf16 dS(j) into
+//   S(j)'s columns, from which dQ += dS K reads it.
 // dkdv_tc_kernel: one CTA (or a cluster of two) per (batch, KV head, 128-key tile); keys are the
 //   M dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
 //   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  The G query heads of the
@@ -20,8 +19,8 @@
 //   CTA takes G/2 heads and the two float32 tiles are added through distributed shared memory (one
 //   bulk copy each way), so no partial sums go through HBM and the result is reproducible.
 // Warp roles as in the forward: warp 0 TMA, warp 1 TMEM owner + single-thread MMA issuer,
-// warps 4.. element-wise warpgroups (thread = TMEM lane = row; two warpgroups split each tile's
-// columns so that each thread handles 32 elements per step).  All mbarrier waits are bounded.
+// warps 4..19 four element-wise warpgroups (thread = TMEM lane = row; the warpgroups split a
+// tile's columns so that each thread handles 32 elements per step).  All mbarrier waits are bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -43,13 +42,15 @@ constexpr uint32_t kQHalf = 128 * 128;
 // ======================================================================================== dQ
 namespace dq {
 
-constexpr int BN = 64;                      // keys per tile
-constexpr uint32_t kKVTile = BN * 256;      // 16 KB
-constexpr uint32_t kKVHalf = BN * 128;      // 8 KB (local layout)
-constexpr int KVS = 3;                      // K/V stages
+constexpr int BN = 128;                     // keys per tile (the N of S = Q K^T and dP = dO V^T)
+constexpr uint32_t kKVTile = BN * 256;      // 32 KB
+constexpr uint32_t kKVHalf = BN * 128;      // 16 KB (local layout)
+constexpr int KS = 3;                       // K stages (a K tile lives until its dQ MMAs are done)
+constexpr int VS = 2;                       // V stages (a V tile lives until its dP MMAs are done)
+constexpr int kEWWarps = 16;                // four element-wise warpgroups
 
 struct Params {
-  int B, Hq, Hkv, G, hpc, kg, nblk;
+  int B, Hq, Hkv, G, kg, nblk;
   int64_t H, S;
   float c2;       // scale * log2(e)
   float scale;
@@ -60,72 +61,81 @@ struct Params {
   int* status;
 };
 
-template <int NT>
 struct Smem {
   static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kDO = kQ + NT * kQTile;
-  static constexpr uint32_t kK = kDO + NT * kQTile;
-  static constexpr uint32_t kV = kK + KVS * kKVTile;
-  static constexpr uint32_t kBar = kV + KVS * kKVTile;
-  // qdo_full, kv_full[KVS], kv_empty[KVS], sd_full[NT], ds_full[NT], final, mma_done
-  static constexpr int kNumBars = 1 + 2 * KVS + 2 * NT + 2;
+  static constexpr uint32_t kDO = kQ + kQTile;
+  static constexpr uint32_t kK = kDO + kQTile;
+  static constexpr uint32_t kV = kK + KS * kKVTile;
+  static constexpr uint32_t kBar = kV + VS * kKVTile;
+  // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], sd_full, dp_free, ds_full, final, mma_done
+  static constexpr int kNumBars = 1 + 2 * KS + VS + 5;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
+static_assert(Smem::kBytes + 1024 <= 227 * 1024, "dq shared memory exceeds the per-CTA limit");
 
-template <int NT>
-__global__ void __launch_bounds__(128 + 256 * NT, 1)
+// One CTA per (batch, KV head, query block, pair of query heads): a single M=128 tile whose rows
+// 0-63 are the block's queries of head h0 and rows 64-127 those of head h0+1.  Key tiles of 128:
+// the routed groups of the block (16 groups per tile) then the causal segment prefix.
+// TMEM: S in two buffers (columns 0 and 128), dP (256), dQ (384).  Per tile j the MMA thread
+// issues dP(j+1) and S(j+1) as soon as the element-wise warps have loaded S(j), dP(j) into
+// registers, and dQ(j) += dS(j) K(j) when they have written dS(j) (bf16, packed into S(j)'s
+// columns).
+__global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                  const Params p) {
-  using L = Smem<NT>;
+  using L = Smem;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBar;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const uint32_t qdo_full = BAR(0);
-  auto kv_full = [&](int s) { return BAR(1 + s); };
-  auto kv_empty = [&](int s) { return BAR(1 + KVS + s); };
-  auto sd_full = [&](int i) { return BAR(1 + 2 * KVS + i); };
-  auto ds_full = [&](int i) { return BAR(1 + 2 * KVS + NT + i); };
-  const uint32_t final_bar = BAR(1 + 2 * KVS + 2 * NT);
-  const uint32_t mma_done = BAR(2 + 2 * KVS + 2 * NT);
+  auto kv_full = [&](int s) { return BAR(1 + s); };          // K(j) and V(j) of tile j, slot j mod KS
+  auto k_empty = [&](int s) { return BAR(1 + KS + s); };
+  auto v_empty = [&](int s) { return BAR(1 + 2 * KS + s); };
+  const uint32_t sd_full = BAR(1 + 2 * KS + VS);
+  const uint32_t dp_free = BAR(2 + 2 * KS + VS);
+  const uint32_t ds_full = BAR(3 + 2 * KS + VS);
+  const uint32_t final_bar = BAR(4 + 2 * KS + VS);
+  const uint32_t mma_done = BAR(5 + 2 * KS + VS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int hg = p.G / p.hpc;
+  // ---- unit decode: query block (heavy = late first), batch x KV head, head pair
+  const int hp = p.G / 2;
   int c = blockIdx.x;
-  const int hgi = c % hg;
-  c /= hg;
+  const int hpi = c % hp;
+  c /= hp;
   const int bkh = c % (p.B * p.Hkv);
   const int n = p.nblk - 1 - c / (p.B * p.Hkv);
   const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
-  const int h0 = kh * p.G + hgi * p.hpc;
-  const int n_rt = (8 * p.kg + BN - 1) / BN;
-  const int T = n_rt + n + 1;
+  const int h0 = kh * p.G + 2 * hpi;
+  const int n_rt = (8 * p.kg + BN - 1) / BN;                     // routed tiles
+  const int T = n_rt + ((n + 1) * kQBlock + BN - 1) / BN;        // + causal-prefix tiles
   const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
   const int64_t ngr = p.H / kGroup;
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
-    for (int s = 0; s < KVS; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(k_empty(s), 1);
     }
-    for (int i = 0; i < NT; ++i) {
-      mbar_init(sd_full(i), 1);
-      mbar_init(ds_full(i), 256);
-    }
+    for (int s = 0; s < VS; ++s) mbar_init(v_empty(s), 1);
+    mbar_init(sd_full, 1);
+    mbar_init(dp_free, kEWWarps);
+    mbar_init(ds_full, kEWWarps);
     mbar_init(final_bar, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), NT * 256);
+    tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -134,160 +144,168 @@ __global__ void __launch_bounds__(128 + 256 * NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ======================= TMA producer
+    // ======================= TMA producer: Q, dO once; then K(j), V(j) per tile into their rings
     if (lane == 0) {
-      mbar_arrive_expect_tx(qdo_full, 2 * NT * kQTile);
-      for (int t = 0; t < NT; ++t)
-        for (int j = 0; j < 2; ++j) {
-          const int64_t row = ((int64_t)b * p.Hq + h0 + 2 * t + j) * p.S + (int64_t)n * kQBlock;
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t off = t * kQTile + h * kQHalf + j * (kQHalf / 2);
-            tma_load_2d(sbase + L::kQ + off, &tm_q, 64 * h, (int32_t)row, qdo_full);
-            tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
-          }
+      mbar_arrive_expect_tx(qdo_full, 2 * kQTile);
+      for (int jh = 0; jh < 2; ++jh) {
+        const int64_t row = ((int64_t)b * p.Hq + h0 + jh) * p.S + (int64_t)n * kQBlock;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t off = h * kQHalf + jh * (kQHalf / 2);
+          tma_load_2d(sbase + L::kQ + off, &tm_q, 64 * h, (int32_t)row, qdo_full);
+          tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
         }
+      }
     }
-    int issued[KVS] = {0, 0, 0};
+    int issued[KS] = {0, 0, 0};
     for (int j = 0; j < T; ++j) {
-      const int s = j % KVS;
+      const int ks = j % KS, vs = j % VS;
       int ok = 1;
       if (lane == 0) {
-        ok = mbar_wait(kv_empty(s), ((j / KVS) & 1) ^ 1, abort_flag, p.status);
-        if (ok) mbar_arrive_expect_tx(kv_full(s), 2 * kKVTile);
+        ok = mbar_wait(k_empty(ks), ((j / KS) & 1) ^ 1, abort_flag, p.status) &&
+             mbar_wait(v_empty(vs), ((j / VS) & 1) ^ 1, abort_flag, p.status);
+        if (ok) mbar_arrive_expect_tx(kv_full(ks), 2 * kKVTile);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const uint32_t kd = sbase + L::kK + s * kKVTile, vd = sbase + L::kV + s * kKVTile;
+      const uint32_t kd = sbase + L::kK + ks * kKVTile, vd = sbase + L::kV + vs * kKVTile;
       if (j < n_rt) {
-        if (lane < 8) {
-          const int slot = j * 8 + lane;
+        // 16 routed groups, one per lane: two 8-row x 64-column boxes each of K and V
+        if (lane < 16) {
+          const int slot = j * 16 + lane;
           int32_t g = gi[slot < p.kg ? slot : 0];
           if (g < 0 || (int64_t)g >= ngr) {
             set_status(p.status, -1);
             g = 0;
           }
           const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
-          tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(s));
-          tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(s));
-          tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(s));
-          tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(s));
+          tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
+          tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
+          tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(ks));
+          tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(ks));
         }
       } else if (lane == 0) {
         const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)(j - n_rt) * BN);
-        tma_load_2d(kd, &tm_ks, 0, row, kv_full(s));
-        tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(s));
-        tma_load_2d(vd, &tm_vs, 0, row, kv_full(s));
-        tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(s));
+        tma_load_2d(kd, &tm_ks, 0, row, kv_full(ks));
+        tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(ks));
+        tma_load_2d(vd, &tm_vs, 0, row, kv_full(ks));
+        tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(ks));
       }
       __syncwarp();
-      ++issued[s];
+      ++issued[ks];
     }
-    if (lane == 0)
-      for (int s = 0; s < KVS; ++s)
-        if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
-  } else if (warp == 1) {
-    // ======================= MMA issuer (one thread).  Descriptor arrays are built before each
-    // unrolled MMA sequence from 64-bit base descriptors prepared once.
     if (lane == 0) {
-      constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, BN, false);
+      drain_wait(qdo_full, 0, p.status);
+      for (int s = 0; s < KS; ++s)
+        if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer: the whole warp runs the loop (warp-uniform descriptors
+    // and waits) and one elected lane issues each tcgen05 instruction.  Q and dO are fixed for
+    // the CTA, so their descriptor arrays are built once; K / V stage descriptors come from
+    // prebuilt bases.
+    {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
-      // stage bases: stage st is st * kKVTile bytes after stage 0 (descriptor units of 16 bytes)
-      const uint64_t q0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
-      const uint64_t do0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+      uint64_t qa[8], da[8];
+      kmajor_descs(qa, sbase + L::kQ, kQHalf, 1024);
+      kmajor_descs(da, sbase + L::kDO, kQHalf, 1024);
+      // routed tiles: group g at g * 2048 bytes, 64-column halves 1024 apart; local tiles: halves
+      // kKVHalf apart, 8-row groups 1024 apart.  Stage st is st * kKVTile bytes after stage 0.
       const uint64_t k_rt = smem_desc_sw128(sbase + L::kK, 16, 2048), k_lc = smem_desc_sw128(sbase + L::kK, 16, 1024);
       const uint64_t v_rt = smem_desc_sw128(sbase + L::kV, 16, 2048), v_lc = smem_desc_sw128(sbase + L::kV, 16, 1024);
       const uint64_t kmn_rt = smem_desc_sw128(sbase + L::kK, 1024, 2048);
       const uint64_t kmn_lc = smem_desc_sw128(sbase + L::kK, kKVHalf, 1024);
-      auto issue_sdp = [&](int j, int i) {
+      auto issue_s = [&](int j) {   // S(j) = Q K(j)^T into S buffer j mod 2
         const bool rt = j < n_rt;
-        const uint64_t soff = (uint64_t)((j % KVS) * (kKVTile >> 4));
-        const uint32_t half_enc = rt ? (1024u >> 4) : (kKVHalf >> 4);
-        uint64_t a[8], bb[8];
-        kmajor_from_base(a, q0 + (uint64_t)(i * (kQTile >> 4)), kQHalf >> 4);
-        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, half_enc);
+        const uint64_t soff = (uint64_t)((j % KS) * (kKVTile >> 4));
+        uint64_t bb[8];
+        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, a[ks], bb[ks], idesc_n64, ks > 0);
-        kmajor_from_base(a, do0 + (uint64_t)(i * (kQTile >> 4)), kQHalf >> 4);
-        kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, half_enc);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128 + 64, a[ks], bb[ks], idesc_n64, ks > 0);
+        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + (j & 1) * 128, qa[ks], bb[ks], idesc_s, ks > 0);
       };
-      auto issue_dq = [&](int j, int i) {
+      auto issue_dp = [&](int j) {  // dP(j) = dO V(j)^T
         const bool rt = j < n_rt;
-        const uint64_t soff = (uint64_t)((j % KVS) * (kKVTile >> 4));
-        uint64_t bb[4];
-        mnmajor_from_base<4>(bb, (rt ? kmn_rt : kmn_lc) + soff, rt ? (2 * 2048u) >> 4 : (2 * 1024u) >> 4);
+        const uint64_t soff = (uint64_t)((j % VS) * (kKVTile >> 4));
+        uint64_t bb[8];
+        kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)   // dS of keys 32h..32h+31 sits in columns 32h..32h+15
-          mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq,
-                 (j > 0 || ks > 0));
+        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + 256, da[ks], bb[ks], idesc_s, ks > 0);
       };
-      bool ok = mbar_wait(qdo_full, 0, abort_flag, p.status) && mbar_wait(kv_full(0), 0, abort_flag, p.status);
-      if (ok) {
+      auto issue_dq = [&](int j) {  // dQ += dS(j) K(j); dS of keys 32w..32w+31 sits in columns 32w..32w+15
+        const bool rt = j < n_rt;
+        const uint64_t soff = (uint64_t)((j % KS) * (kKVTile >> 4));
+        uint64_t bb[8];
+        mnmajor_from_base<8>(bb, (rt ? kmn_rt : kmn_lc) + soff, rt ? (2 * 2048u) >> 4 : (2 * 1024u) >> 4);
+        const uint32_t sb = tmem + (j & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_w(tmem + 384, sb + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq, (j > 0 || ks > 0));
+      };
+      // Per tile j: once the element-wise warps hold S(j), dP(j) in registers, dP(j+1) and S(j+1)
+      // (the other S buffer, whose dS(j-1) dQ(j-1) has already read); once they have written
+      // dS(j), dQ(j) += dS(j) K(j).
+      auto issue_sdp = [&](int j) {   // K(j), V(j) have landed
         tc_fence_after();
-        for (int i = 0; i < NT; ++i) {
-          issue_sdp(0, i);
-          mma_commit(sd_full(i));
-        }
-      }
+        issue_dp(j);
+        issue_s(j);
+        mma_commit_w(sd_full);
+        mma_commit_w(v_empty(j % VS));
+      };
+      bool ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status);
+      if (ok) issue_sdp(0);
       for (int j = 0; ok && j < T; ++j) {
-        for (int i = 0; ok && i < NT; ++i) {
-          ok = mbar_wait(ds_full(i), j & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dq(j, i);
-          if (j + 1 < T) {
-            // the next K/V tile is only needed now, after this tile's first dQ MMAs are queued
-            if (i == 0) ok = mbar_wait(kv_full((j + 1) % KVS), ((j + 1) / KVS) & 1, abort_flag, p.status);
-            if (!ok) break;
-            tc_fence_after();
-            issue_sdp(j + 1, i);
-            mma_commit(sd_full(i));
-          }
-        }
+        // the next tile's K/V usually landed long ago: check that before the wait on the
+        // element-wise warps, so nothing but that wait sits between it and the next MMAs
+        if (j + 1 < T) ok = mbar_wait_w(kv_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
+        if (ok) ok = mbar_wait_w(dp_free, j & 1, abort_flag, p.status);
         if (!ok) break;
-        mma_commit(kv_empty(j % KVS));
+        if (j + 1 < T) issue_sdp(j + 1);
+        ok = mbar_wait_w(ds_full, j & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dq(j);
+        mma_commit_w(k_empty(j % KS));
       }
-      if (ok) mma_commit(final_bar);
-      mma_commit(mma_done);
+      if (ok) mma_commit_w(final_bar);
+      mma_commit_w(mma_done);
       drain_wait(mma_done, 0, p.status);
     }
-    __syncwarp();
   } else if (warp >= 4) {
-    // ======================= element-wise: dS = P o (dP - delta); two warpgroups per M-tile,
-    // each owning 32 of the tile's 64 key columns (thread = TMEM lane = query row)
-    const int w4 = (warp - 4) >> 2;
-    const int i = w4 >> 1, hc = w4 & 1;
+    // ======================= element-wise: dS = P o (dP - delta), P = exp2(S c2 - lse log2 e).
+    // Thread = TMEM lane = row of the M tile; warpgroup w owns key columns 32w .. 32w+31.
+    const int w = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int head = h0 + 2 * i + (r >> 6);
+    const int head = h0 + (r >> 6);
     const int64_t t_pos = (int64_t)n * kQBlock + (r & 63);
     const int64_t row = ((int64_t)b * p.Hq + head) * p.S + t_pos;
     const float lse2 = p.lse[row] * kLog2e;
     const float dl = p.delta[row];
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + i * 128;
-    const uint32_t tP = tS + 64;
-    const uint32_t tQ = tmem + lane_off + NT * 128 + i * 128;
+    const int c0 = 32 * w;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(sd_full(i), j & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(sd_full, j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      int nvalid;
+      const uint32_t tS = tmem + lane_off + (j & 1) * 128 + c0;
+      // one TMEM round trip: both loads in flight, one wait; then dP is free for dP(j+1)
+      uint32_t sv[32], dv[32], pk[16];
+      tmem_ld32(tS, sv);
+      tmem_ld32(tmem + lane_off + 256 + c0, dv);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dp_free);
+      int nvalid;   // valid key columns of this tile for this row
       if (j < n_rt) {
         nvalid = min(BN, 8 * p.kg - j * BN);
       } else {
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
       }
-      // one TMEM round trip per step: both loads in flight, one wait, compute, one store
-      uint32_t sv[32], dv[32], pk[16];
-      tmem_ld32(tS + 32 * hc, sv);
-      tmem_ld32(tP + 32 * hc, dv);
-      tmem_wait_ld();
-      const int c0 = 32 * hc;
-      if (nvalid >= BN) {
+      if (nvalid >= c0 + 32) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2));
@@ -302,35 +320,32 @@ __global__ void __launch_bounds__(128 + 256 * NT, 1)
           pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
         }
       }
-      // packed bf16 stays inside this warpgroup's own (already read) column range
-      tmem_st16(tS + 32 * hc, pk);
+      // packed bf16 dS stays inside this warpgroup's own (already read) column range
+      tmem_st16(tS, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full(i));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(final_bar, 0, abort_flag, p.status));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + row * kD + 64 * hc;
+      uint32_t v[32], pk[16];
+      tmem_ld32(tmem + lane_off + 384 + c0, v);
+      tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32], pk[16];
-        tmem_ld32(tQ + 64 * hc + cc * 32, v);
-        tmem_wait_ld();
+      for (int e = 0; e < 32; e += 2)
+        pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale);
+      uint4* d4 = reinterpret_cast<uint4*>(p.dq + row * kD + c0);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-      }
+      for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NT * 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -478,9 +493,11 @@ __global__ void __launch_bounds__(640, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ======================= MMA issuer (one thread).  K and V are fixed for the CTA, so their
-    // descriptor arrays are built once; Q / dO stage descriptors come from prebuilt bases.
-    if (lane == 0) {
+    // ======================= MMA issuer: the whole warp runs the loop (warp-uniform descriptors
+    // and waits) and one elected lane issues each tcgen05 instruction.  K and V are fixed for the
+    // CTA, so their descriptor arrays are built once; Q / dO stage descriptors come from prebuilt
+    // bases.
+    {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BQ, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(BM, kD, true);
       uint64_t kd[8], vd[8];
@@ -496,10 +513,10 @@ __global__ void __launch_bounds__(640, 1)
         uint64_t bb[8];
         kmajor_from_base(bb, q0 + soff, kQHalfB >> 4);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + x * 128, kd[ks], bb[ks], idesc_s, ks > 0);
+        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + x * 128, kd[ks], bb[ks], idesc_s, ks > 0);
         kmajor_from_base(bb, do0 + soff, kQHalfB >> 4);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + x * 128 + 64, vd[ks], bb[ks], idesc_s, ks > 0);
+        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + x * 128 + 64, vd[ks], bb[ks], idesc_s, ks > 0);
       };
       auto issue_grad = [&](int j, int x) {
         const uint64_t soff = (uint64_t)((j % NS) * (kQTileB >> 4));
@@ -511,38 +528,37 @@ __global__ void __launch_bounds__(640, 1)
 #pragma unroll
         for (int ks = 0; ks < BQ / 16; ++ks) {
           const uint32_t acol = (ks >> 1) * 32 + (ks & 1) * 8;
-          mma_ts(tmem + 256, tmem + x * 128 + acol, b1[ks], idesc_g, (j > 0 || ks > 0));
-          mma_ts(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (j > 0 || ks > 0));
+          mma_ts_w(tmem + 256, tmem + x * 128 + acol, b1[ks], idesc_g, (j > 0 || ks > 0));
+          mma_ts_w(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (j > 0 || ks > 0));
         }
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
+      bool ok = mbar_wait_w(kv_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < 2 && j < NJ; ++j) {
-        ok = mbar_wait(q_full(j % NS), (j / NS) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(q_full(j % NS), (j / NS) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         issue_sd(j, j & 1);
-        mma_commit(sd_full(j & 1));
+        mma_commit_w(sd_full(j & 1));
       }
       for (int j = 0; ok && j < NJ; ++j) {
         const int x = j & 1;
-        ok = mbar_wait(pd_full(x), (j >> 1) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(pd_full(x), (j >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         issue_grad(j, x);
-        mma_commit(q_empty(j % NS));
+        mma_commit_w(q_empty(j % NS));
         if (j + 2 < NJ) {
-          ok = mbar_wait(q_full((j + 2) % NS), ((j + 2) / NS) & 1, abort_flag, p.status);
+          ok = mbar_wait_w(q_full((j + 2) % NS), ((j + 2) / NS) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           issue_sd(j + 2, x);
-          mma_commit(sd_full(x));
+          mma_commit_w(sd_full(x));
         }
       }
-      if (ok) mma_commit(done);
-      mma_commit(mma_done);
+      if (ok) mma_commit_w(done);
+      mma_commit_w(mma_done);
       drain_wait(mma_done, 0, p.status);
     }
-    __syncwarp();
   } else if (warp >= 4) {
     // ======================= element-wise: P^T, dS^T.  Warpgroup w4 = 0..3 takes the steps
     // j = w4 mod 2 and the 32 query columns 32*(w4/2) .. of each (thread = TMEM lane = key row).
@@ -691,21 +707,13 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  K::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), H, S, scale * tcbwd::kLog2e, scale,
-              gi, lse, delta, static_cast<__nv_bfloat16*>(dq), status};
-  const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
-  cudaError_t e;
-  if (p.hpc == 4) {
-    const size_t smem = K::Smem<2>::kBytes + 1024;
-    e = cudaFuncSetAttribute(K::dq_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    K::dq_tc_kernel<2><<<(unsigned)grid, 640, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
-  } else {
-    const size_t smem = K::Smem<1>::kBytes + 1024;
-    e = cudaFuncSetAttribute(K::dq_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    K::dq_tc_kernel<1><<<(unsigned)grid, 384, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
-  }
+  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), H, S, scale * tcbwd::kLog2e, scale, gi, lse, delta,
+              static_cast<__nv_bfloat16*>(dq), status};
+  const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / 2);
+  const size_t smem = K::Smem::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(K::dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  K::dq_tc_kernel<<<(unsigned)grid, 128 + 32 * K::kEWWarps, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
   return cudaGetLastError();
 }
 

@@ -193,9 +193,10 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       for (int s = 0; s < NS; ++s)
         if (issued[s]) drain_wait(kv ? v_full(s) : k_full(s), (issued[s] - 1) & 1, p.status);
   } else if (warp == 1) {
-    // ======================= MMA issuer (one thread).  All shared-memory descriptors are built
-    // before each unrolled MMA sequence, so the sequence issues back to back.
-    if (lane == 0) {
+    // ======================= MMA issuer: the whole warp runs the loop (warp-uniform descriptors
+    // and waits) and one elected lane issues each tcgen05 instruction.  All shared-memory
+    // descriptors are built before each unrolled MMA sequence, so the sequence issues back to back.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kD, true);
       uint64_t qd[NT][8], kd[8], vd[8];
@@ -210,53 +211,52 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         mnmajor_descs<8>(vd, sbase + L::kV + (j % VS) * kTileBytes, routed ? 1024u : kHalfBytes,
                          routed ? 2048u : 1024u);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full(0), 0, abort_flag, p.status);
+      bool ok = mbar_wait_w(q_full, 0, abort_flag, p.status) && mbar_wait_w(k_full(0), 0, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
         build_k(0);
 #pragma unroll
         for (int i = 0; i < NT; ++i) {
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
-          mma_commit(s_full(i));
+          for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
+          mma_commit_w(s_full(i));
         }
-        mma_commit(k_empty(0));
+        mma_commit_w(k_empty(0));
       }
       for (int j = 0; ok && j < T; ++j) {
-        ok = mbar_wait(v_full(j % VS), (j / VS) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(v_full(j % VS), (j / VS) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         build_v(j);
 #pragma unroll
         for (int i = 0; i < NT; ++i) {
-          ok = mbar_wait(p_full(i), j & 1, abort_flag, p.status);
+          ok = mbar_wait_w(p_full(i), j & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, vd[ks], idesc_pv, (j > 0 || ks > 0));
+            mma_ts_w(tmem + NT * 128 + i * 128, tmem + i * 128 + ks * 8, vd[ks], idesc_pv, (j > 0 || ks > 0));
           if (j + 1 < T) {
             // the next K tile is only needed now, after this tile's first PV is queued
             if (i == 0) {
-              ok = mbar_wait(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
+              ok = mbar_wait_w(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
               if (!ok) break;
               tc_fence_after();
               build_k(j + 1);
             }
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
-            mma_commit(s_full(i));
+            for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + i * 128, qd[i][ks], kd[ks], idesc_qk, ks > 0);
+            mma_commit_w(s_full(i));
           }
         }
         if (!ok) break;
-        mma_commit(v_empty(j % VS));
-        if (j + 1 < T) mma_commit(k_empty((j + 1) % KS));
+        mma_commit_w(v_empty(j % VS));
+        if (j + 1 < T) mma_commit_w(k_empty((j + 1) % KS));
       }
-      if (ok) mma_commit(o_final);
-      mma_commit(mma_done);
+      if (ok) mma_commit_w(o_final);
+      mma_commit_w(mma_done);
       drain_wait(mma_done, 0, p.status);
     }
-    __syncwarp();
   } else if (warp >= 4) {
     // ======================= softmax / epilogue, one warpgroup per M-tile
     const int i = (warp - 4) >> 2;
