@@ -136,13 +136,19 @@ class ClockSampler:
 
 
 def dist_setup():
+    """One process per GPU (torchrun env).  NCCL where CUDA is present; gloo otherwise, which is
+    all the CPU-only reference arm needs."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -153,9 +159,12 @@ def barrier(world):
 
 
 def all_max(v: float, world: int, device) -> float:
+    """Max of v over the ranks (device times are reported as the slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
+    if dist.get_backend() != "nccl":
+        device = "cpu"
     t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
