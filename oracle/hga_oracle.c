@@ -22,8 +22,10 @@
  * Where the pages leave a step open, the reading taken is stated next to the
  * code (summary = arithmetic mean; block query = mean over the block's
  * queries and the query heads of one KV head; ties go to the lower index;
- * only history chunks are routable; one joint softmax over routed and causal
- * local keys; scale 1/sqrt(D) unless given).
+ * only history chunks are routable; the fixed sink window is the first
+ * n_sink history tokens, whole chunks, always attended and never routed; one
+ * joint softmax over sink, routed and causal local keys; scale 1/sqrt(D)
+ * unless given).
  *
  * Layout of every tensor: contiguous [B, heads, tokens, D] in float64.
  * Arithmetic: float64 throughout, except that the routing functions accept
@@ -160,12 +162,13 @@ int hgo_topk(int64_t n, const double* score, int64_t k, int64_t* sel, double* ga
 /* chunk_gap, group_gap [B,Hkv,nblk]: score gap at the selection boundary.   */
 /* ------------------------------------------------------------------------ */
 int hgo_route(int64_t B, int64_t Hkv, int64_t nblk, int64_t D, int64_t nch, int64_t gpc,
-              int64_t kc, int64_t kg, int32_t prec,
+              int64_t nsc, int64_t kc, int64_t kg, int32_t prec,
               const double* qb, const double* gs, const double* cs,
               int32_t* chunk_idx, int32_t* group_idx, double* chunk_gap, double* group_gap)
 {
     if (B < 0 || Hkv <= 0 || nblk < 0 || D <= 0 || nch < 1 || gpc < 1) return -1;
-    if (kc < 1 || kc > nch || kg < 1 || kg > kc * gpc) return -1;
+    if (nsc < 0 || nsc >= nch) return -1;
+    if (kc < 1 || kc > nch - nsc || kg < 1 || kg > kc * gpc) return -1;
     if (prec != 32 && prec != 64) return -1;
     const int64_t ngr = nch * gpc;
     scored_t* items = (scored_t*)malloc((size_t)(nch > kc * gpc ? nch : kc * gpc) * sizeof(scored_t));
@@ -177,15 +180,17 @@ int hgo_route(int64_t B, int64_t Hkv, int64_t nblk, int64_t D, int64_t nch, int6
         for (int64_t n = 0; n < nblk && rc == 0; ++n) {
             const int64_t u = bh * nblk + n;
             const double* qv = qb + u * D;
-            /* level 1: every history chunk */
-            for (int64_t i = 0; i < nch; ++i) {
+            /* level 1: every history chunk outside the sink window (the sink's nsc
+             * chunks are attended anyway; [TS] 2.1: chunks are selected "alongside
+             * fixed sink and local windows") */
+            for (int64_t i = nsc; i < nch; ++i) {
                 const double* cv = cs + (bh * nch + i) * D;
                 double acc = 0.0;
                 for (int64_t d = 0; d < D; ++d) acc = rnd(acc + rnd(qv[d] * cv[d], prec), prec);
-                items[i].s = acc;
-                items[i].i = i;
+                items[i - nsc].s = acc;
+                items[i - nsc].i = i;
             }
-            rc = select_topk(items, nch, kc, csel, &chunk_gap[u]);
+            rc = select_topk(items, nch - nsc, kc, csel, &chunk_gap[u]);
             if (rc) break;
             /* level 2: the gpc groups of every selected chunk */
             int64_t nc = 0;
@@ -218,11 +223,14 @@ int hgo_route(int64_t B, int64_t Hkv, int64_t nblk, int64_t D, int64_t nch, int6
 /* the active segment; one joint softmax over routed and local keys.        */
 /*                                                                            */
 /* Key set of query (b, h, t), t in block n = t / qblock, kh = h / G:         */
+/*   the sink window: history tokens 0 .. nsink-1                             */
 /*   history tokens group*j .. group*j+group-1 for j in group_idx[b,kh,n,:]  */
 /*   active-segment tokens u = 0 .. t                                        */
+/* Routed groups never lie in the sink (routing excludes it); a group index  */
+/* that does is an invalid argument, as one out of range is.                 */
 /* ------------------------------------------------------------------------ */
 typedef struct {
-    int64_t B, Hq, Hkv, H, S, D, qblock, group, kg;
+    int64_t B, Hq, Hkv, H, S, D, qblock, group, kg, nsink;
     double scale;
     const double *q, *k_hist, *v_hist, *k_seg, *v_seg;
     const int32_t* group_idx;
@@ -236,6 +244,11 @@ static int64_t key_set(const layer_t* L, int64_t b, int64_t h, int64_t t,
     const int64_t G = L->Hq / L->Hkv, kh = h / G, n = t / L->qblock;
     const int32_t* gi = L->group_idx + ((b * L->Hkv + kh) * (L->S / L->qblock) + n) * L->kg;
     int64_t m = 0;
+    for (int64_t pos = 0; pos < L->nsink; ++pos) {
+        kr[m] = L->k_hist + ((b * L->Hkv + kh) * L->H + pos) * L->D;
+        vr[m] = L->v_hist + ((b * L->Hkv + kh) * L->H + pos) * L->D;
+        ++m;
+    }
     for (int64_t r = 0; r < L->kg; ++r)
         for (int64_t e = 0; e < L->group; ++e) {
             const int64_t pos = (int64_t)gi[r] * L->group + e;
@@ -283,23 +296,29 @@ static int check_layer(const layer_t* L)
 {
     if (L->B < 0 || L->Hq <= 0 || L->Hkv <= 0 || L->Hq % L->Hkv) return -1;
     if (L->H < 0 || L->S <= 0 || L->D <= 0 || L->qblock <= 0 || L->S % L->qblock) return -1;
-    if (L->group <= 0 || L->H % L->group || L->kg < 0 || L->kg * L->group > L->H) return -1;
+    if (L->group <= 0 || L->H % L->group || L->kg < 0) return -1;
+    if (L->nsink < 0 || L->nsink % L->group || L->nsink + L->kg * L->group > L->H) return -1;
+    /* every routed group index must name a history group outside the sink */
+    const int64_t ngr = L->H / L->group, nsg = L->nsink / L->group;
+    const int64_t nidx = L->B * L->Hkv * (L->S / L->qblock) * L->kg;
+    for (int64_t i = 0; i < nidx; ++i)
+        if (L->group_idx[i] < nsg || L->group_idx[i] >= ngr) return -1;
     return 0;
 }
 
 /* Forward.  rows: list of nrows row ids r = (b*Hq + h)*S + t, or NULL for all
  * B*Hq*S rows in order.  o [nrows, D], lse [nrows]. */
 int hgo_attn_fwd(int64_t B, int64_t Hq, int64_t Hkv, int64_t H, int64_t S, int64_t D,
-                 int64_t qblock, int64_t group, int64_t kg, double scale,
+                 int64_t qblock, int64_t group, int64_t kg, int64_t nsink, double scale,
                  const double* q, const double* k_hist, const double* v_hist,
                  const double* k_seg, const double* v_seg, const int32_t* group_idx,
                  int64_t nrows, const int64_t* rows, double* o, double* lse)
 {
-    layer_t L = {B, Hq, Hkv, H, S, D, qblock, group, kg, scale,
+    layer_t L = {B, Hq, Hkv, H, S, D, qblock, group, kg, nsink, scale,
                  q, k_hist, v_hist, k_seg, v_seg, group_idx};
     if (check_layer(&L)) return -1;
     if (!rows) nrows = B * Hq * S;
-    const int64_t maxk = kg * group + S;
+    const int64_t maxk = nsink + kg * group + S;
     const double** kr = (const double**)malloc((size_t)maxk * sizeof(double*));
     const double** vr = (const double**)malloc((size_t)maxk * sizeof(double*));
     double* p = (double*)malloc((size_t)maxk * sizeof(double));
@@ -328,19 +347,19 @@ int hgo_attn_fwd(int64_t B, int64_t Hq, int64_t Hkv, int64_t H, int64_t S, int64
  * keys (nkeys, or NULL = all B*Hkv*S): active-segment key ids
  *   r = (b*Hkv + kh)*S + u; dk, dv [nkeys, D]. */
 int hgo_attn_bwd(int64_t B, int64_t Hq, int64_t Hkv, int64_t H, int64_t S, int64_t D,
-                 int64_t qblock, int64_t group, int64_t kg, double scale,
+                 int64_t qblock, int64_t group, int64_t kg, int64_t nsink, double scale,
                  const double* q, const double* k_hist, const double* v_hist,
                  const double* k_seg, const double* v_seg, const int32_t* group_idx,
                  const double* d_o,
                  int64_t nrows, const int64_t* rows, double* dq,
                  int64_t nkeys, const int64_t* keys, double* dk, double* dv)
 {
-    layer_t L = {B, Hq, Hkv, H, S, D, qblock, group, kg, scale,
+    layer_t L = {B, Hq, Hkv, H, S, D, qblock, group, kg, nsink, scale,
                  q, k_hist, v_hist, k_seg, v_seg, group_idx};
     if (check_layer(&L)) return -1;
     if (!rows) nrows = B * Hq * S;
     if (!keys) nkeys = B * Hkv * S;
-    const int64_t G = Hq / Hkv, maxk = kg * group + S, nall = B * Hq * S;
+    const int64_t G = Hq / Hkv, maxk = nsink + kg * group + S, nall = B * Hq * S;
     const double** kr = (const double**)malloc((size_t)maxk * sizeof(double*));
     const double** vr = (const double**)malloc((size_t)maxk * sizeof(double*));
     double* p = (double*)malloc((size_t)maxk * sizeof(double));

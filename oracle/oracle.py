@@ -49,10 +49,10 @@ def _load():
         lib.hgo_span_means.argtypes = [_i64, _i64, _i64, _i64, _i64, _i32, _p, _p]
         lib.hgo_block_query.argtypes = [_i64, _i64, _i64, _i64, _i64, _i64, _i32, _p, _p]
         lib.hgo_topk.argtypes = [_i64, _p, _i64, _p, _p]
-        lib.hgo_route.argtypes = [_i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i32,
+        lib.hgo_route.argtypes = [_i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i32,
                                   _p, _p, _p, _p, _p, _p, _p]
-        lib.hgo_attn_fwd.argtypes = [_i64] * 9 + [_dbl] + [_p] * 6 + [_i64, _p, _p, _p]
-        lib.hgo_attn_bwd.argtypes = ([_i64] * 9 + [_dbl] + [_p] * 7
+        lib.hgo_attn_fwd.argtypes = [_i64] * 10 + [_dbl] + [_p] * 6 + [_i64, _p, _p, _p]
+        lib.hgo_attn_bwd.argtypes = ([_i64] * 10 + [_dbl] + [_p] * 7
                                      + [_i64, _p, _p, _i64, _p, _p, _p])
         for f in (lib.hgo_span_means, lib.hgo_block_query, lib.hgo_topk, lib.hgo_route,
                   lib.hgo_attn_fwd, lib.hgo_attn_bwd):
@@ -114,9 +114,10 @@ def topk(score, k: int):
     return sel, float(gap[0])
 
 
-def route(qb, gs, cs, top_chunks: int, top_groups: int, prec: int = 64):
+def route(qb, gs, cs, top_chunks: int, top_groups: int, prec: int = 64, n_sink_chunks: int = 0):
     """Two-level routing from summaries.  Returns chunk_idx, group_idx (int32, ascending) and the
-    score gaps at the chunk and group selection boundaries, each [B,Hkv,nblk]."""
+    score gaps at the chunk and group selection boundaries, each [B,Hkv,nblk].  The first
+    ``n_sink_chunks`` chunks (the fixed sink window) are not routable."""
     qb, gs, cs = _f64(qb), _f64(gs), _f64(cs)
     B, Hkv, nblk, D = qb.shape
     nch = cs.shape[2]
@@ -125,19 +126,22 @@ def route(qb, gs, cs, top_chunks: int, top_groups: int, prec: int = 64):
     gi = np.empty((B, Hkv, nblk, top_groups), dtype=np.int32)
     cgap = np.empty((B, Hkv, nblk))
     ggap = np.empty((B, Hkv, nblk))
-    _check(_load().hgo_route(B, Hkv, nblk, D, nch, gpc, top_chunks, top_groups, prec,
+    _check(_load().hgo_route(B, Hkv, nblk, D, nch, gpc, n_sink_chunks, top_chunks, top_groups, prec,
                              _ptr(qb), _ptr(gs), _ptr(cs), _ptr(ci), _ptr(gi), _ptr(cgap), _ptr(ggap)),
            "route")
     return ci, gi, cgap, ggap
 
 
 def route_from_inputs(q, k_hist, Hkv: int, top_chunks: int, top_groups: int, chunk: int = 64,
-                      group: int = 8, qblock: int = 64, prec: int = 32) -> dict:
-    """Summaries, block query and routing in one call (decisions taken in ``prec`` bits)."""
+                      group: int = 8, qblock: int = 64, prec: int = 32, n_sink: int = 0) -> dict:
+    """Summaries, block query and routing in one call (decisions taken in ``prec`` bits);
+    ``n_sink`` sink tokens (a multiple of ``chunk``) are excluded from routing."""
+    if n_sink % chunk:
+        raise ValueError("n_sink must be a multiple of the chunk size")
     gs = group_summaries(k_hist, group, prec)
     cs = chunk_summaries(k_hist, chunk, prec)
     qb = block_query(q, Hkv, qblock, prec)
-    ci, gi, cgap, ggap = route(qb, gs, cs, top_chunks, top_groups, prec)
+    ci, gi, cgap, ggap = route(qb, gs, cs, top_chunks, top_groups, prec, n_sink // chunk)
     return dict(group_sum=gs, chunk_sum=cs, qb=qb, chunk_idx=ci, group_idx=gi,
                 chunk_gap=cgap, group_gap=ggap)
 
@@ -151,8 +155,8 @@ def _layer(q, k_hist, v_hist, k_seg, v_seg, group_idx):
 
 
 def attn_fwd(q, k_hist, v_hist, k_seg, v_seg, group_idx, scale: float | None = None,
-             group: int = 8, qblock: int = 64, rows=None):
-    """Routed + causal-local attention forward.  Returns (o, lse).
+             group: int = 8, qblock: int = 64, rows=None, n_sink: int = 0):
+    """Sink + routed + causal-local attention forward.  Returns (o, lse).
 
     rows=None: o [B,Hq,S,D], lse [B,Hq,S].  rows = array of flat row ids (b*Hq+h)*S+t:
     o [len(rows), D], lse [len(rows)]."""
@@ -167,14 +171,14 @@ def attn_fwd(q, k_hist, v_hist, k_seg, v_seg, group_idx, scale: float | None = N
     else:
         r = np.ascontiguousarray(rows, dtype=np.int64)
         o = np.empty((r.size, D)); lse = np.empty(r.size); rp = _ptr(r); nr = r.size
-    _check(_load().hgo_attn_fwd(B, Hq, Hkv, H, S, D, qblock, group, kg, scale,
+    _check(_load().hgo_attn_fwd(B, Hq, Hkv, H, S, D, qblock, group, kg, n_sink, scale,
                                 _ptr(q), _ptr(kh), _ptr(vh), _ptr(ks), _ptr(vs), _ptr(gi),
                                 nr, rp, _ptr(o), _ptr(lse)), "attn_fwd")
     return o, lse
 
 
 def attn_bwd(q, k_hist, v_hist, k_seg, v_seg, group_idx, d_o, scale: float | None = None,
-             group: int = 8, qblock: int = 64, rows=None, keys=None):
+             group: int = 8, qblock: int = 64, rows=None, keys=None, n_sink: int = 0):
     """Gradients (dq, dk_seg, dv_seg) of sum(o * d_o); history K/V and routing get none.
 
     rows/keys select flat ids (b*Hq+h)*S+t for dq and (b*Hkv+kh)*S+u for dk/dv; None = all."""
@@ -194,7 +198,7 @@ def attn_bwd(q, k_hist, v_hist, k_seg, v_seg, group_idx, d_o, scale: float | Non
     else:
         kk = np.ascontiguousarray(keys, dtype=np.int64)
         dk = np.empty((kk.size, D)); dv = np.empty((kk.size, D)); kp = _ptr(kk); nk = kk.size
-    _check(_load().hgo_attn_bwd(B, Hq, Hkv, H, S, D, qblock, group, kg, scale,
+    _check(_load().hgo_attn_bwd(B, Hq, Hkv, H, S, D, qblock, group, kg, n_sink, scale,
                                 _ptr(q), _ptr(kh), _ptr(vh), _ptr(ks), _ptr(vs), _ptr(gi), _ptr(do),
                                 nr, rp, _ptr(dq), nk, kp, _ptr(dk), _ptr(dv)), "attn_bwd")
     return dq, dk, dv

@@ -177,11 +177,12 @@ def _small_layer(seed, B=1, Hq=4, Hkv=2, D=16, H=256, S=128):
                 k_seg=t(B, Hkv, S, D), v_seg=t(B, Hkv, S, D), d_o=t(B, Hq, S, D))
 
 
-def _mask_from_groups(group_idx, B, Hq, Hkv, H, S, group=8, qblock=64):
-    """Boolean [B, Hq, S, H+S]: history position p visible to query t iff p // group is one of
-    the block's routed groups; segment key u visible iff u <= t."""
+def _mask_from_groups(group_idx, B, Hq, Hkv, H, S, group=8, qblock=64, n_sink=0):
+    """Boolean [B, Hq, S, H+S]: history position p visible to query t iff p < n_sink or p // group
+    is one of the block's routed groups; segment key u visible iff u <= t."""
     G = Hq // Hkv
     m = torch.zeros(B, Hq, S, H + S, dtype=torch.bool)
+    m[:, :, :, :n_sink] = True
     gi = torch.as_tensor(np.asarray(group_idx), dtype=torch.long)
     for b, h in itertools.product(range(B), range(Hq)):
         for n in range(S // qblock):
@@ -207,15 +208,16 @@ def _sdpa_reference(x, mask, scale):
     return o.detach(), lse, q.grad, ks.grad, vs.grad
 
 
-def _check_against_sdpa(oracle, x, group_idx, H, S):
+def _check_against_sdpa(oracle, x, group_idx, H, S, n_sink=0):
     B, Hq = x["q"].shape[:2]
     Hkv = x["k_hist"].shape[1]
     scale = 1 / math.sqrt(x["q"].shape[-1])
-    mask = _mask_from_groups(group_idx, B, Hq, Hkv, H, S)
+    mask = _mask_from_groups(group_idx, B, Hq, Hkv, H, S, n_sink=n_sink)
     o_ref, lse_ref, dq_ref, dk_ref, dv_ref = _sdpa_reference(x, mask, scale)
-    o, lse = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], group_idx)
+    o, lse = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], group_idx,
+                             n_sink=n_sink)
     dq, dk, dv = oracle.attn_bwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"],
-                                 group_idx, x["d_o"])
+                                 group_idx, x["d_o"], n_sink=n_sink)
     for a, b in [(o, o_ref), (lse, lse_ref), (dq, dq_ref), (dk, dk_ref), (dv, dv_ref)]:
         np.testing.assert_allclose(a, b.numpy(), rtol=1e-10, atol=1e-10)
 
@@ -240,6 +242,51 @@ def test_routed_attention_equals_masked_dense_attention(oracle):
     rand_gi = np.stack([np.sort(torch.randperm(H // 8, generator=g)[:3].numpy())
                         for _ in range(2 * (S // 64))]).reshape(1, 2, S // 64, 3).astype(np.int32)
     _check_against_sdpa(oracle, x, rand_gi, H, S)
+
+
+def test_sink_window_dense_equivalence_with_full_budget(oracle):
+    """Sink of two chunks + every other chunk and group routed: HGA == dense causal attention
+    over [history | segment]; the sink chunks are never routed."""
+    H, S, ns = 256, 128, 128
+    x = _small_layer(5, H=H, S=S)
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], 2, (H - ns) // 64, (H - ns) // 8, prec=64, n_sink=ns)
+    assert (r["chunk_idx"] >= ns // 64).all()
+    assert (r["group_idx"] == np.arange(ns // 8, H // 8)).all()
+    _check_against_sdpa(oracle, x, r["group_idx"], H, S, n_sink=ns)
+
+
+def test_sink_window_equals_masked_dense_attention(oracle):
+    """Sink tokens are visible to every query, next to the routed groups and the causal prefix."""
+    H, S, ns = 256, 128, 64
+    x = _small_layer(6, H=H, S=S)
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], 2, 2, 5, prec=64, n_sink=ns)
+    assert (r["chunk_idx"] >= 1).all() and (r["group_idx"] >= ns // 8).all()
+    _check_against_sdpa(oracle, x, r["group_idx"], H, S, n_sink=ns)
+    # the sink changes the output (it is attended, not ignored)
+    o0, _ = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
+    o1, _ = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"],
+                            n_sink=ns)
+    assert np.abs(o0 - o1).max() > 1e-3
+
+
+def test_route_brute_force_with_sink(oracle):
+    """With n_sink_chunks sink chunks the chunk set is the best kc-subset of the other chunks."""
+    rng = np.random.default_rng(8)
+    B, Hkv, nblk, D, nch, gpc, nsc, kc, kg = 1, 1, 3, 8, 7, 4, 2, 2, 3
+    for _ in range(10):
+        qb = rng.standard_normal((B, Hkv, nblk, D))
+        gs = rng.standard_normal((B, Hkv, nch * gpc, D))
+        cs = rng.standard_normal((B, Hkv, nch, D))
+        cs[..., :nsc, :] += 10 * qb[..., :1, :]        # sink chunks would win if they were routable
+        ci, gi, _, _ = oracle.route(qb, gs, cs, kc, kg, 64, n_sink_chunks=nsc)
+        for n in range(nblk):
+            sc = cs[0, 0] @ qb[0, 0, n]
+            best_c = max(itertools.combinations(range(nsc, nch), kc), key=lambda c: sc[list(c)].sum())
+            assert list(ci[0, 0, n]) == sorted(best_c)
+            cand = [c * gpc + r for c in best_c for r in range(gpc)]
+            sg = gs[0, 0] @ qb[0, 0, n]
+            best_g = max(itertools.combinations(cand, kg), key=lambda c: sg[list(c)].sum())
+            assert list(gi[0, 0, n]) == sorted(best_g)
 
 
 def test_gradients_match_finite_differences(oracle):
@@ -370,6 +417,16 @@ def test_invalid_arguments_raise(oracle):
         oracle.route(qb, gs, cs, 3, 4)          # k_c > number of chunks
     with pytest.raises(ValueError):
         oracle.route(qb, gs, cs, 1, 9)          # k_g > groups of the chosen chunks
+    with pytest.raises(ValueError):
+        oracle.route(qb, gs, cs, 2, 4, n_sink_chunks=1)   # k_c > chunks outside the sink
+    with pytest.raises(ValueError):
+        oracle.route(qb, gs, cs, 1, 4, n_sink_chunks=2)   # the sink covers every chunk
+    x = _small_layer(0, H=128, S=64)
+    gi = np.array([[[[3, 9]], [[8, 9]]]], dtype=np.int32)
+    with pytest.raises(ValueError):                        # group 3 lies in a 64-token sink
+        oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], gi, n_sink=64)
+    with pytest.raises(ValueError):                        # group 16 is beyond the history
+        oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], gi + 7)
 
 
 # --------------------------------------------------------------------------- inputs used by GPU parity
