@@ -207,6 +207,28 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3) -> float:
+    """Mean device time (ms) of one whole layer step of workload w, L2 flushed before each step."""
+    x = {k: v.to(dev) for k, v in HI.make_inputs(w, seed).items() if k != "needles"}
+    cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    step = H.LayerStep(cfg, dev)
+    calls = step.calls(x, stream.cuda_stream)
+    for _ in range(warmup):
+        for _, c in calls:
+            c()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush_l2()
+        e0.record(stream)
+        for _, c in calls:
+            c()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if H.read_status(step.ws) != 0:
+        raise RuntimeError(f"device status word set while timing {w.name}")
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+
+
 def _config(w, args):
     return {"workload": f"{w.name}: routed HGA layer, B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, "
                         f"history={w.hist_len}, segment={w.seg_len}, chunk=64, group=8, qblock=64, "
@@ -228,6 +250,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-positions", action="store_true",
+                    help="skip timing the 16K layer's earlier segment positions")
     args = ap.parse_args()
     w = HI.WORKLOADS[args.workload]
     world, rank, local = dist_setup()
@@ -287,6 +311,19 @@ def main():
     value = tokens / t_step
     if H.read_status(step.ws) != 0:
         raise RuntimeError("device status word set during the timed region")
+
+    # the same layer at the earlier segment positions of a 16K sequence (history 2048 / 6144 /
+    # 10240 / 14336): attention work per token is flat, only summaries and chunk scoring grow
+    # (timed alike: events at step boundaries only, so these read a little below ms_per_step,
+    # whose timed steps also record an event after every kernel for the per-kernel times)
+    positions = None
+    if w.name == "ctx16k" and not args.no_positions:
+        positions = {}
+        for pname in ("ctx4k", "ctx8k", "ctx12k", "ctx16k"):
+            pw = HI.WORKLOADS[pname]
+            ms = all_max(_time_layer(H, pw, args.seed + rank, dev, stream, flush_l2), world, dev)
+            positions[f"history_{pw.hist_len}"] = {"ms_per_step": ms,
+                                                   "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
 
     # roofline of the dominant kernel
     wm = work_model(w)
@@ -359,6 +396,8 @@ def main():
                 "config": _config(w, args), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": K * len(calls), "clocks": clk.summary(),
                 "kernels_per_step": names}
+        if positions:
+            line["segment_positions"] = positions
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

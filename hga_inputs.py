@@ -13,6 +13,8 @@ Figure 1 caption; segment 2048 tokens as the TBPTT segment length there):
                  top-4 chunks / top-8 groups, float32, chunk offsets of scale 1.
 * ``ctx4k``      4096 context = 2048 history + 2048 segment, top-16 / top-64, bf16.
 * ``ctx16k``     16384 context = 14336 history + 2048 segment, top-16 / top-64, bf16.
+* ``ctx8k``, ``ctx12k``  the same layer at history 6144 / 10240 (earlier segment positions of
+                 the 16K sequence; ``ctx4k`` is the one at history 2048).
 * ``ctx131k``    131072 context = 129024 history + 2048 segment, top-32 / top-128,
                  bf16, forward only, 64 planted needle groups.
 * ``ctx16k_b4``  the 16K layer at batch 4 (tiered-history workload shape).
@@ -57,6 +59,7 @@ class Workload:
     needles: int = 0
     needle_q: float = 1.0
     needle_k: float = 32.0
+    n_sink: int = 0            # sink-window tokens at the start of the history (multiple of chunk)
 
     @property
     def torch_dtype(self):
@@ -82,6 +85,9 @@ WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", 1, 4, 1, 128, 1024, 256, 4, 8, "f32", 1.0),
     "ctx4k": Workload("ctx4k", 1, 32, 8, 128, 2048, 2048, 16, 64, "bf16", 0.5),
     "ctx16k": Workload("ctx16k", 1, 32, 8, 128, 14336, 2048, 16, 64, "bf16", 0.5),
+    # the 16K layer's earlier segment positions (history 6144 and 10240; 2048 is ctx4k)
+    "ctx8k": Workload("ctx8k", 1, 32, 8, 128, 6144, 2048, 16, 64, "bf16", 0.5),
+    "ctx12k": Workload("ctx12k", 1, 32, 8, 128, 10240, 2048, 16, 64, "bf16", 0.5),
     "ctx131k": Workload("ctx131k", 1, 32, 8, 128, 129024, 2048, 32, 128, "bf16", 0.5,
                         backward=False, needles=64),
     "ctx16k_b4": Workload("ctx16k_b4", 4, 32, 8, 128, 14336, 2048, 16, 64, "bf16", 0.5),
@@ -162,6 +168,11 @@ EDGE_WORKLOADS = {
     # two query heads per KV head (one 128-row query tile per CTA), 7 query blocks (a ragged
     # 64-key last tile of the dK/dV kernel), 20 groups = 160 routed keys (ragged routed tiles), bf16
     "gqa2_ragged_bf16": Workload("gqa2_ragged_bf16", 1, 4, 2, 128, 1024, 448, 3, 20, "bf16", 1.0),
+    # sink windows: two chunks (float32), one chunk (bf16, four query heads per KV head) and one
+    # chunk with two query heads per KV head and a ragged routed tile (bf16)
+    "sink_f32": WORKLOADS["tiny_f32"].with_(name="sink_f32", n_sink=128),
+    "sink_bf16": WORKLOADS["small_bf16"].with_(name="sink_bf16", n_sink=64),
+    "sink_gqa2_bf16": Workload("sink_gqa2_bf16", 1, 4, 2, 128, 1024, 448, 3, 20, "bf16", 1.0, n_sink=128),
     # eight query heads per KV head (two CTAs per query block), 5 query blocks, bf16
     "gqa8_bf16": Workload("gqa8_bf16", 1, 8, 1, 128, 512, 320, 4, 12, "bf16", 1.0),
     # many (batch, KV head) units of short segments: as many dK/dV key tiles as SMs or more, so

@@ -37,14 +37,15 @@ def _need(t: torch.Tensor, name: str, shape, dtype) -> None:
 
 
 def make_config(q: torch.Tensor, k_hist: torch.Tensor, top_chunks: int, top_groups: int,
-                softmax_scale: float | None = None) -> C.HGAConfig:
-    """Configuration from q [B,Hq,S,D] and k_hist [B,Hkv,H,D]."""
+                softmax_scale: float | None = None, n_sink_tokens: int = 0) -> C.HGAConfig:
+    """Configuration from q [B,Hq,S,D] and k_hist [B,Hkv,H,D]; ``n_sink_tokens`` (a multiple of 64)
+    history tokens at the start form the sink window every query attends."""
     if q.dtype not in _DT:
         raise ValueError(f"unsupported dtype {q.dtype}")
     B, Hq, S, D = q.shape
     Hkv, H = k_hist.shape[1], k_hist.shape[2]
     return C.make_config(B, Hq, Hkv, H, S, top_chunks, top_groups, dtype=_DT[q.dtype], D=D,
-                         softmax_scale=float(softmax_scale or 0.0))
+                         softmax_scale=float(softmax_scale or 0.0), n_sink_tokens=n_sink_tokens)
 
 
 def _tdtype(cfg) -> torch.dtype:

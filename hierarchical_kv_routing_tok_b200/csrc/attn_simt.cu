@@ -98,28 +98,27 @@ __device__ __forceinline__ float half_warp_sum(float v) {
 
 struct Dims {
   int Hq, Hkv, G, kg, nblk;
+  int nsg;              // sink groups at the start of every block's history key list
   int64_t H, S;
   float scale;
   int* status;          // workspace status word (HGA_ERR_ARG recorded for an out-of-range group index)
 };
 
-// Source row of key r of the key list of block n of KV head (b, kh): the first 8*kg keys are
-// routed history tokens, then segment tokens 0.. (the caller masks u > t).
-// A group index outside [0, H/8) is never dereferenced: the key reads as zeros and the status
-// word records HGA_ERR_ARG (-1).
+// Source row of key r of the key list of block n of KV head (b, kh): the first 8*(nsg + kg) keys
+// are history tokens (the sink window, then the routed groups), then segment tokens 0.. (the
+// caller masks u > t).  A routed group index outside [nsg, H/8) is never dereferenced: the key
+// reads as zeros and the status word records HGA_ERR_ARG (-1).
 template <typename T>
 __device__ __forceinline__ const T* key_row(const T* hist, const T* seg, const int32_t* gi, const Dims& dm,
                                             int64_t r, int64_t n_keys) {
   if (r >= n_keys) return nullptr;
-  if (r < 8 * dm.kg) {
-    const int32_t g = gi[r >> 3];
-    if (g < 0 || (int64_t)g >= dm.H / kGroup) {
-      set_status(dm.status, -1);
-      return nullptr;
-    }
+  const int64_t n_hist = 8LL * (dm.nsg + dm.kg);
+  if (r < n_hist) {
+    const int32_t g = routed_group(gi, (int)(r >> 3), dm.nsg, dm.kg, dm.H / kGroup, dm.status);
+    if (g < 0) return nullptr;
     return hist + ((int64_t)g * kGroup + (r & 7)) * kD;
   }
-  return seg + (r - 8 * dm.kg) * kD;
+  return seg + (r - n_hist) * kD;
 }
 
 // ------------------------------------------------------------------------------------ forward
@@ -148,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const T* __restrict__ q, 
   const T* ks_base = k_seg + bkh * dm.S * kD;
   const T* vs_base = v_seg + bkh * dm.S * kD;
   const int32_t* gi = group_idx + (bkh * dm.nblk + n) * dm.kg;
-  const int64_t n_route = 8LL * dm.kg;
+  const int64_t n_route = 8LL * (dm.nsg + dm.kg);
   const int64_t n_keys = n_route + (int64_t)(n + 1) * BM;
   const float qmul = dm.scale * kLog2e;
 
@@ -277,7 +276,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(const T* __restrict__ 
   const T* ks_base = k_seg + bkh * dm.S * kD;
   const T* vs_base = v_seg + bkh * dm.S * kD;
   const int32_t* gi = group_idx + (bkh * dm.nblk + n) * dm.kg;
-  const int64_t n_route = 8LL * dm.kg;
+  const int64_t n_route = 8LL * (dm.nsg + dm.kg);
   const int64_t n_keys = n_route + (int64_t)(n + 1) * BM;
 
   load_tile<T>(Qs, [&](int r) { return q + (row0 + r) * kD; }, dm.scale * kLog2e);
@@ -448,15 +447,15 @@ cudaError_t bwd_dq(const void* q, const void* kh, const void* vh, const void* ks
 
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
-                                 int64_t H, int64_t S, int kg, float scale, int* status, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), H, S, scale, status};
+                                 int64_t H, int64_t S, int kg, int nsg, float scale, int* status, cudaStream_t st) {
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, scale, status};
   return bf16 ? simt::fwd<__nv_bfloat16>(q, kh, vh, ks, vs, gi, o, lse, B, dm, st)
               : simt::fwd<float>(q, kh, vh, ks, vs, gi, o, lse, B, dm, st);
 }
 
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st) {
-  simt::Dims dm{Hq, 1, Hq, 0, (int)(S / kQBlock), 0, S, 0.f, nullptr};
+  simt::Dims dm{Hq, 1, Hq, 0, (int)(S / kQBlock), 0, 0, S, 0.f, nullptr};
   return bf16 ? simt::bwd_delta<__nv_bfloat16>(o, d_o, delta, B, dm, st)
               : simt::bwd_delta<float>(o, d_o, delta, B, dm, st);
 }
@@ -464,7 +463,7 @@ cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, flo
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
                                  const void* d_o, const float* delta, void* dk, void* dv, int B, int Hq, int Hkv,
                                  int64_t H, int64_t S, int kg, float scale, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), H, S, scale, nullptr};
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), 0, H, S, scale, nullptr};
   return bf16 ? simt::bwd_dkdv<__nv_bfloat16>(q, ks, vs, lse, d_o, delta, dk, dv, B, dm, st)
               : simt::bwd_dkdv<float>(q, ks, vs, lse, d_o, delta, dk, dv, B, dm, st);
 }
@@ -472,8 +471,8 @@ cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const
 cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                const void* vs, const int32_t* gi, const float* lse, const void* d_o,
                                const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
-                               float scale, int* status, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), H, S, scale, status};
+                               int nsg, float scale, int* status, cudaStream_t st) {
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, scale, status};
   return bf16 ? simt::bwd_dq<__nv_bfloat16>(q, kh, vh, ks, vs, gi, lse, d_o, delta, dq, B, dm, st)
               : simt::bwd_dq<float>(q, kh, vh, ks, vs, gi, lse, d_o, delta, dq, B, dm, st);
 }

@@ -51,6 +51,7 @@ constexpr int kEWWarps = 16;                // four element-wise warpgroups
 
 struct Params {
   int B, Hq, Hkv, G, kg, nblk;
+  int nsg;        // sink groups at the start of every block's history key list
   int64_t H, S;
   float c2;       // scale * log2(e)
   float scale;
@@ -114,7 +115,8 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   const int n = p.nblk - 1 - c / (p.B * p.Hkv);
   const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
   const int h0 = kh * p.G + 2 * hpi;
-  const int n_rt = (8 * p.kg + BN - 1) / BN;                     // routed tiles
+  const int n_hist = 8 * (p.nsg + p.kg);                         // sink + routed history keys
+  const int n_rt = (n_hist + BN - 1) / BN;                        // history tiles
   const int T = n_rt + ((n + 1) * kQBlock + BN - 1) / BN;        // + causal-prefix tiles
   const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
   const int64_t ngr = p.H / kGroup;
@@ -172,11 +174,8 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         // 16 routed groups, one per lane: two 8-row x 64-column boxes each of K and V
         if (lane < 16) {
           const int slot = j * 16 + lane;
-          int32_t g = gi[slot < p.kg ? slot : 0];
-          if (g < 0 || (int64_t)g >= ngr) {
-            set_status(p.status, -1);
-            g = 0;
-          }
+          int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
+          if (g < 0) g = 0;
           const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
           tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
           tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       if (lane == 0) mbar_arrive(dp_free);
       int nvalid;   // valid key columns of this tile for this row
       if (j < n_rt) {
-        nvalid = min(BN, 8 * p.kg - j * BN);
+        nvalid = min(BN, n_hist - j * BN);
       } else {
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
@@ -696,7 +695,7 @@ __global__ void __launch_bounds__(640, 1)
 // ------------------------------------------------------------------ host side
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, int nsg, float scale, int* status,
                              cudaStream_t st) {
   namespace K = tcbwd::dq;
   CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
@@ -707,7 +706,7 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), H, S, scale * tcbwd::kLog2e, scale, gi, lse, delta,
+  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, scale * tcbwd::kLog2e, scale, gi, lse, delta,
               static_cast<__nv_bfloat16*>(dq), status};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / 2);
   const size_t smem = K::Smem::kBytes + 1024;

@@ -37,6 +37,7 @@ constexpr float kRescaleThreshold = 8.f;   // log2 units
 
 struct Params {
   int B, Hq, Hkv, G, hpc, kg, nblk;
+  int nsg;        // sink groups at the start of every block's history key list
   int64_t H, S;
   float scale_log2;
   const int32_t* group_idx;
@@ -96,7 +97,8 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
   const int n = p.nblk - 1 - c / (p.B * p.Hkv);
   const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
   const int h0 = kh * p.G + hgi * p.hpc;
-  const int n_rt = (8 * p.kg + BN - 1) / BN;
+  const int n_hist = 8 * (p.nsg + p.kg);                 // sink + routed history keys
+  const int n_rt = (n_hist + BN - 1) / BN;
   const int n_lt = n / 2 + 1;
   const int T = n_rt + n_lt;
   const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
@@ -168,11 +170,8 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       if (j < n_rt) {
         if (lane < 16) {
           const int slot = j * 16 + lane;
-          int32_t g = gi[slot < p.kg ? slot : 0];
-          if (g < 0 || (int64_t)g >= ngr) {
-            set_status(p.status, -1);
-            g = 0;
-          }
+          int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
+          if (g < 0) g = 0;
           const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
           const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
           tma_load_2d(dst + lane * 2048, m, 0, row, full);
@@ -277,7 +276,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       const bool routed = j < n_rt;
       int nvalid;
       if (routed) {
-        nvalid = min(BN, 8 * p.kg - j * BN);
+        nvalid = min(BN, n_hist - j * BN);
       } else {
         const int64_t u0 = (int64_t)(j - n_rt) * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
@@ -412,7 +411,7 @@ bool attn_fwd_tc_supported(int Hq, int Hkv) {
 
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int kg, float scale, int* status, cudaStream_t st) {
+                               int kg, int nsg, float scale, int* status, cudaStream_t st) {
   CUtensorMap mq, mkh, mvh, mks, mvs;
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mkh, kh, (uint64_t)B * Hkv * H, 8) ||
       !make_map_bf16_rows(&mvh, vh, (uint64_t)B * Hkv * H, 8) ||
@@ -420,7 +419,7 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, tcfwd::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), H, S,
+  tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), nsg, H, S,
                   scale * 1.4426950408889634f, gi, static_cast<__nv_bfloat16*>(o), lse, status};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
   cudaError_t e;

@@ -62,4 +62,21 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// History group read by slot `slot` of a block's history key list: the nsg groups of the sink
+// window (groups 0..nsg-1) come first, then the block's kg routed groups gi[0..kg).  Slots past the
+// list (tile padding) read group 0.  A routed index outside [nsg, ngr) is never dereferenced: it
+// records HGA_ERR_ARG (-1) in the status word and -1 is returned.
+__device__ __forceinline__ int32_t routed_group(const int32_t* gi, int slot, int nsg, int kg, int64_t ngr,
+                                                int* status) {
+  if (slot < nsg) return slot;
+  const int r = slot - nsg;
+  if (r >= kg) return 0;
+  const int32_t g = gi[r];
+  if (g < nsg || (int64_t)g >= ngr) {
+    set_status(status, -1);
+    return -1;
+  }
+  return g;
+}
+
 }  // namespace hga

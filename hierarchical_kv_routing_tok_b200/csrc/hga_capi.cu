@@ -14,18 +14,18 @@ cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, fl
                              int64_t n_chunks_total, cudaStream_t stream);
 cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
                          int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S, int nch,
-                         int kc, int kg, cudaStream_t stream);
+                         int nsc, int kc, int kg, cudaStream_t stream);
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
-                                 int64_t H, int64_t S, int kg, float scale, int* status, cudaStream_t st);
+                                 int64_t H, int64_t S, int kg, int nsg, float scale, int* status, cudaStream_t st);
 bool attn_fwd_tc_supported(int Hq, int Hkv);
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int kg, float scale, int* status, cudaStream_t st);
+                               int kg, int nsg, float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, float scale, int* status,
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, int nsg, float scale, int* status,
                              cudaStream_t st);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
                                const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
@@ -38,7 +38,7 @@ cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const
 cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                const void* vs, const int32_t* gi, const float* lse, const void* d_o,
                                const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
-                               float scale, int* status, cudaStream_t st);
+                               int nsg, float scale, int* status, cudaStream_t st);
 }  // namespace hga
 
 namespace {
@@ -54,12 +54,15 @@ int check_config(const hga_config_t* c) {
   if (c->dtype != HGA_F32 && c->dtype != HGA_BF16) return HGA_ERR_ARG;
   if (c->D != hga::kD || c->chunk != hga::kChunk || c->group != hga::kGroup || c->qblock != hga::kQBlock)
     return HGA_ERR_UNSUPPORTED;
-  if (c->n_sink_tokens != 0) return HGA_ERR_UNSUPPORTED;
   if (c->hist_len < c->chunk || c->hist_len % c->chunk != 0) return HGA_ERR_ARG;
   if (c->seg_len < c->qblock || c->seg_len % c->qblock != 0) return HGA_ERR_ARG;
   const int64_t nch = c->hist_len / c->chunk;
   if (nch > kMaxChunks) return HGA_ERR_UNSUPPORTED;
-  if (c->top_chunks < 1 || c->top_chunks > nch) return HGA_ERR_ARG;
+  // the sink window: whole chunks at the start of the history, at least one chunk left to route
+  if (c->n_sink_tokens < 0 || c->n_sink_tokens % c->chunk != 0 || c->n_sink_tokens >= c->hist_len)
+    return HGA_ERR_ARG;
+  const int64_t nsc = c->n_sink_tokens / c->chunk;
+  if (c->top_chunks < 1 || c->top_chunks > nch - nsc) return HGA_ERR_ARG;
   if (c->top_groups < 1 || (int64_t)c->top_groups > (int64_t)c->top_chunks * (c->chunk / c->group))
     return HGA_ERR_ARG;
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return HGA_ERR_ARG;
@@ -78,6 +81,9 @@ int check_ptrs(std::initializer_list<const void*> ps) {
     if (!aligned16(p)) return HGA_ERR_ALIGN;
   return HGA_OK;
 }
+
+// Groups of the sink window, attended by every query ahead of the routed groups.
+int sink_groups(const hga_config_t* c) { return (int)(c->n_sink_tokens / c->group); }
 
 float eff_scale(const hga_config_t* c) {
   return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->D);
@@ -188,7 +194,8 @@ int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, co
   (void)workspace;
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, group_sum, chunk_sum, chunk_idx, group_idx, cfg->B,
                                      cfg->Hq, cfg->Hkv, cfg->seg_len, (int)(cfg->hist_len / cfg->chunk),
-                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
+                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
@@ -202,11 +209,11 @@ int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (use_tc(cfg))
     return from_cuda(hga::launch_attn_fwd_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B, cfg->Hq,
-                                             cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups, eff_scale(cfg),
-                                             status_of(workspace), st));
+                                             cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups, sink_groups(cfg),
+                                             eff_scale(cfg), status_of(workspace), st));
   return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
                                              cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
-                                             eff_scale(cfg), status_of(workspace), st));
+                                             sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
 }
 
 int hga_attn_bwd_preprocess(const hga_config_t* cfg, const void* o, const void* d_o, void* workspace,
@@ -239,10 +246,11 @@ int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, 
   if (use_tc(cfg))
     return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, delta_of(workspace),
                                            dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
-                                           eff_scale(cfg), status_of(workspace), st));
+                                           sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
   return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
                                            d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
-                                           cfg->seg_len, cfg->top_groups, eff_scale(cfg), status_of(workspace), st));
+                                           cfg->seg_len, cfg->top_groups, sink_groups(cfg), eff_scale(cfg),
+                                           status_of(workspace), st));
 }
 
 int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,

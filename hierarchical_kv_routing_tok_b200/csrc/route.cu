@@ -194,7 +194,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     const T* __restrict__ q, const float* __restrict__ group_sum, const float* __restrict__ chunk_sum,
     int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq, int Hkv, int64_t S, int nch,
-    int kc, int kg) {
+    int nsc, int kc, int kg) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int N = Vec16<T>::N;
   constexpr int LPR = kD / N;
@@ -255,15 +255,21 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     __syncthreads();
   }
 
-  // ---- level 1: chunks
+  // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
+  // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
   const float* cs = chunk_sum + (int64_t)bkh * nch * kD;
-  score_rows(qb, cs, nch, [](int i) { return i; }, keys);
-  if (threadIdx.x < 4 && nch + (int)threadIdx.x < ((nch + 3) & ~3)) keys[nch + threadIdx.x] = 0u;
+  const int nc1 = nch - nsc;
+  score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
+  if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
   __syncthreads();
-  if (nch <= kRouteThreads)
-    block_select_topk_small(keys, nch, kc, csel, scratch);
+  if (nc1 <= kRouteThreads)
+    block_select_topk_small(keys, nc1, kc, csel, scratch);
   else
-    block_select_topk(keys, nch, kc, csel, hist, scratch);
+    block_select_topk(keys, nc1, kc, csel, hist, scratch);
+  if (nsc) {
+    for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] += nsc;
+    __syncthreads();
+  }
 
   // ---- level 2: the 8 groups of every selected chunk
   const float* gs = group_sum + (int64_t)bkh * nch * (kChunk / kGroup) * kD;
@@ -290,7 +296,7 @@ size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
 
 cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
                          int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S,
-                         int nch, int kc, int kg, cudaStream_t stream) {
+                         int nch, int nsc, int kc, int kg, cudaStream_t stream) {
   const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
   if (units == 0) return cudaSuccess;
   const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
@@ -299,13 +305,13 @@ cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const
     e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     route_kernel<__nv_bfloat16><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, kc,
-        kg);
+        static_cast<const __nv_bfloat16*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc,
+        kc, kg);
   } else {
     e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     route_kernel<float><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const float*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, kc, kg);
+        static_cast<const float*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
   }
   return cudaGetLastError();
 }

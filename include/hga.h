@@ -22,8 +22,10 @@
  * score is the raw dot product; only history chunks are routable; group
  * selection is one top-k over all groups of the chosen chunks; ties go to the
  * lower index; index lists are sorted ascending; the local window is the whole
- * causal prefix of the active segment; one softmax spans routed and local
- * keys; softmax scale 1/sqrt(D) unless given.
+ * causal prefix of the active segment; the fixed sink window (section 2.1,
+ * "alongside fixed sink and local windows") is the first n_sink_tokens history
+ * tokens, whole chunks, attended by every query and never routed; one softmax
+ * spans sink, routed and local keys; softmax scale 1/sqrt(D) unless given.
  *
  * Conventions for every entry point
  *   - Memory: the caller allocates and owns every buffer, including the
@@ -44,7 +46,8 @@
  *     written before they are read).  Kernels that wait on on-chip barriers give up after
  *     a bounded time and record HGA_ERR_TIMEOUT there instead of hanging; an
  *     attention kernel given a group index outside [0, H/8) reads that group
- *     as zeros (never out of bounds) and records HGA_ERR_ARG there.
+ *     as zeros (never out of bounds) and records HGA_ERR_ARG there; so does a
+ *     routed index inside the sink window.
  *   - Aliasing: outputs must not overlap inputs or each other.
  *   - Thread safety: the library keeps no mutable host state; calls on
  *     different streams with different workspaces may run concurrently.
@@ -85,8 +88,11 @@ enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 };
  * the only built values (pith.science free-parameter ledger: chunk 64,
  * group 8).  hist_len must be a positive multiple of chunk (only closed
  * chunks exist), seg_len a positive multiple of qblock.
- * 1 <= top_chunks <= hist_len / chunk; 1 <= top_groups <= top_chunks *
- * (chunk / group).  n_sink_tokens must be 0 (sink window not built).
+ * n_sink_tokens: 0 <= n_sink_tokens < hist_len, a multiple of chunk; the
+ * first n_sink_tokens history tokens are attended by every query and their
+ * chunks are not routable, so 1 <= top_chunks <= (hist_len - n_sink_tokens) /
+ * chunk; 1 <= top_groups <= top_chunks * (chunk / group).  group_idx passed to
+ * the attention calls holds routed groups only (all >= n_sink_tokens / group).
  * softmax_scale = 0 selects 1 / sqrt(D). */
 typedef struct hga_config {
   int32_t B, Hq, Hkv, D;

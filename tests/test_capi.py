@@ -84,7 +84,10 @@ def test_workspace_size(lib):
     (dict(chunk=32), C.HGA_ERR_UNSUPPORTED),
     (dict(group=4), C.HGA_ERR_UNSUPPORTED),
     (dict(qblock=128), C.HGA_ERR_UNSUPPORTED),
-    (dict(n_sink_tokens=4), C.HGA_ERR_UNSUPPORTED),
+    (dict(n_sink_tokens=4), C.HGA_ERR_ARG),           # sink not a whole number of chunks
+    (dict(n_sink_tokens=-64), C.HGA_ERR_ARG),
+    (dict(n_sink_tokens=14336), C.HGA_ERR_ARG),       # sink covers the whole history
+    (dict(n_sink_tokens=13312, top_chunks=17), C.HGA_ERR_ARG),  # k_c > the 16 chunks left to route
     (dict(hist_len=14300), C.HGA_ERR_ARG),            # open chunk
     (dict(hist_len=0), C.HGA_ERR_ARG),
     (dict(seg_len=2000), C.HGA_ERR_ARG),
@@ -101,6 +104,11 @@ def test_config_validation(lib, kw, code):
     with pytest.raises(C.HGAError) as e:
         C.workspace_size(cfg(**kw))
     assert e.value.code == code
+
+
+def test_sink_window_config_accepted(lib):
+    assert C.workspace_size(cfg(n_sink_tokens=64)) == _expected_ws(1, 32, 8, 2048)
+    assert C.workspace_size(cfg(n_sink_tokens=13312, top_chunks=16)) == _expected_ws(1, 32, 8, 2048)
 
 
 def test_entry_points_reject_bad_pointers_before_launch(lib):

@@ -35,7 +35,7 @@ def _wl(name):
 def run_gpu(hga, w, x, backward=True, group_idx=None):
     """Whole hot path on cuda:0 through the C ABI; returns CPU copies of every output."""
     xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
-    cfg = hga.make_config(xd["q"], xd["k_hist"], w.top_chunks, w.top_groups)
+    cfg = hga.make_config(xd["q"], xd["k_hist"], w.top_chunks, w.top_groups, n_sink_tokens=w.n_sink)
     step = hga.LayerStep(cfg)
     step.forward(xd)
     if group_idx is not None:          # attention on a given routing (routing-independent check)
@@ -70,13 +70,14 @@ def test_full_path_matches_oracle(hga, oracle, name):
     np.testing.assert_allclose(g["gs"].numpy(), gs, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(g["cs"].numpy(), cs, rtol=1e-5, atol=1e-6)
     # routing: bit-exact against the oracle deciding in float32
-    r = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32)
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32,
+                                 n_sink=w.n_sink)
     assert np.array_equal(g["ci"].numpy(), r["chunk_idx"])
     assert np.array_equal(g["gi"].numpy(), r["group_idx"])
     # forward / backward
     args = (x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
-    o, lse = oracle.attn_fwd(*args)
-    dq, dk, dv = oracle.attn_bwd(*args, x["d_o"])
+    o, lse = oracle.attn_fwd(*args, n_sink=w.n_sink)
+    dq, dk, dv = oracle.attn_bwd(*args, x["d_o"], n_sink=w.n_sink)
     tol = TOL[w.dtype]
     errs = dict(o=maxerr(g["o"], o), dq=maxerr(g["dq"], dq), dk=maxerr(g["dk"], dk), dv=maxerr(g["dv"], dv))
     assert max(errs.values()) <= tol, errs

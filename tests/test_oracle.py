@@ -444,8 +444,10 @@ def test_parity_seeds_have_routing_margins(oracle, name):
     w = HI.WORKLOADS.get(name) or HI.EDGE_WORKLOADS[name]
     for seed in PARITY_SEEDS[name]:
         x = HI.make_inputs(w, seed)
-        r32 = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32)
-        r64 = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=64)
+        r32 = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32,
+                                       n_sink=w.n_sink)
+        r64 = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=64,
+                                       n_sink=w.n_sink)
         assert np.array_equal(r32["chunk_idx"], r64["chunk_idx"])
         assert np.array_equal(r32["group_idx"], r64["group_idx"])
         assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
