@@ -251,7 +251,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-positions", action="store_true",
-                    help="skip timing the 16K layer's earlier segment positions")
+                    help="skip timing the 16K layer at its earlier segment positions and other budgets")
     args = ap.parse_args()
     w = HI.WORKLOADS[args.workload]
     world, rank, local = dist_setup()
@@ -324,6 +324,15 @@ def main():
             ms = all_max(_time_layer(H, pw, args.seed + rank, dev, stream, flush_l2), world, dev)
             positions[f"history_{pw.hist_len}"] = {"ms_per_step": ms,
                                                    "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
+    # routing-budget sweep of the same layer (the pages vary the routed chunk count from 8 to 32)
+    budgets = None
+    if w.name == "ctx16k" and not args.no_positions:
+        budgets = {}
+        for pname in ("ctx16k_kc8", "ctx16k", "ctx16k_kc32"):
+            pw = HI.WORKLOADS[pname]
+            ms = all_max(_time_layer(H, pw, args.seed + rank, dev, stream, flush_l2), world, dev)
+            budgets[f"top_chunks_{pw.top_chunks}_top_groups_{pw.top_groups}"] = {
+                "ms_per_step": ms, "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
 
     # roofline of the dominant kernel
     wm = work_model(w)
@@ -398,6 +407,8 @@ def main():
                 "kernels_per_step": names}
         if positions:
             line["segment_positions"] = positions
+        if budgets:
+            line["routing_budget_sweep"] = budgets
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

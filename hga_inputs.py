@@ -15,6 +15,8 @@ Figure 1 caption; segment 2048 tokens as the TBPTT segment length there):
 * ``ctx16k``     16384 context = 14336 history + 2048 segment, top-16 / top-64, bf16.
 * ``ctx8k``, ``ctx12k``  the same layer at history 6144 / 10240 (earlier segment positions of
                  the 16K sequence; ``ctx4k`` is the one at history 2048).
+* ``ctx16k_kc8``, ``ctx16k_kc32``  the 16K layer with routing budgets 8 / 32 and 32 / 128
+                 (the pages' sweep of the routed chunk count from 8 to 32).
 * ``ctx131k``    131072 context = 129024 history + 2048 segment, top-32 / top-128,
                  bf16, forward only, 64 planted needle groups.
 * ``ctx16k_b4``  the 16K layer at batch 4 (tiered-history workload shape).
@@ -88,6 +90,9 @@ WORKLOADS = {
     # the 16K layer's earlier segment positions (history 6144 and 10240; 2048 is ctx4k)
     "ctx8k": Workload("ctx8k", 1, 32, 8, 128, 6144, 2048, 16, 64, "bf16", 0.5),
     "ctx12k": Workload("ctx12k", 1, 32, 8, 128, 10240, 2048, 16, 64, "bf16", 0.5),
+    # routing-budget sweep of the 16K layer (k_c = 8 and 32 with k_g = 4 k_c; 16 / 64 is ctx16k)
+    "ctx16k_kc8": Workload("ctx16k_kc8", 1, 32, 8, 128, 14336, 2048, 8, 32, "bf16", 0.5),
+    "ctx16k_kc32": Workload("ctx16k_kc32", 1, 32, 8, 128, 14336, 2048, 32, 128, "bf16", 0.5),
     "ctx131k": Workload("ctx131k", 1, 32, 8, 128, 129024, 2048, 32, 128, "bf16", 0.5,
                         backward=False, needles=64),
     "ctx16k_b4": Workload("ctx16k_b4", 4, 32, 8, 128, 14336, 2048, 16, 64, "bf16", 0.5),

@@ -152,7 +152,8 @@ def _sampled_rows(w, n, seed):
     return np.array(sorted(set(ids)), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name,seed", [("ctx4k", 0), ("ctx4k", 1), ("ctx16k", 0), ("ctx16k", 2)])
+@pytest.mark.parametrize("name,seed", [("ctx4k", 0), ("ctx4k", 1), ("ctx16k", 0), ("ctx16k", 2),
+                                       ("ctx16k_kc8", 0), ("ctx16k_kc32", 0)])
 def test_full_size_layer_sampled(hga, oracle, name, seed):
     w = HI.WORKLOADS[name]
     x = HI.make_inputs(w, seed)
