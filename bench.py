@@ -229,6 +229,37 @@ def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3) -> float:
     return sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
 
 
+def _time_tiered(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=2) -> dict:
+    """The layer of workload w with its history K/V in pinned host memory (TieredLayerStep), and the
+    same layer with the history resident in device memory, both timed per step on the device."""
+    x = HI.make_inputs(w, seed)
+    xd = {k: x[k].to(dev) for k in ("q", "k_seg", "v_seg", "d_o")}
+    kh, vh = x["k_hist"].pin_memory(), x["v_hist"].pin_memory()
+    cfg = H.make_config(xd["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    # summaries are built when the history is written, while its keys are still on the device
+    gs, cs = H.build_summaries(cfg, x["k_hist"].to(dev))
+    step = H.TieredLayerStep(cfg, kh, vh, gs, cs, dev)
+    for _ in range(warmup):
+        step(xd)
+    step.wait(timeout_s=60)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush_l2()
+        e0.record(stream)
+        step(xd)
+        e1.record(stream)
+    step.wait(timeout_s=60)
+    ms = all_max(sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps, world, dev)
+    nbytes = step.gather_bytes()
+    resident_ms = all_max(_time_layer(H, w, seed, dev, stream, flush_l2), world, dev)
+    tokens = w.B * w.seg_len * world
+    return {"workload": f"{w.name}: the 16K layer at batch {w.B}, history K/V ({2 * kh.numel() * kh.element_size() >> 20}"
+                        " MiB) in pinned host memory, summaries in device memory",
+            "ms_per_step": ms, "tokens_per_s": tokens / (ms * 1e-3),
+            "gather_bytes_per_step": nbytes, "host_link_GBps": nbytes / (ms * 1e-3) / 1e9,
+            "resident_ms_per_step": resident_ms, "resident_tokens_per_s": tokens / (resident_ms * 1e-3)}
+
+
 def _config(w, args):
     return {"workload": f"{w.name}: routed HGA layer, B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, "
                         f"history={w.hist_len}, segment={w.seg_len}, chunk=64, group=8, qblock=64, "
@@ -250,6 +281,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tiered", action="store_true", help="skip the tiered-history (batch 4) measurement")
     ap.add_argument("--no-positions", action="store_true",
                     help="skip timing the 16K layer at its earlier segment positions and other budgets")
     args = ap.parse_args()
@@ -334,6 +366,12 @@ def main():
             budgets[f"top_chunks_{pw.top_chunks}_top_groups_{pw.top_groups}"] = {
                 "ms_per_step": ms, "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
 
+    # tiered-history variant of the 16K layer at batch 4: history K/V in pinned host memory, the
+    # summaries in device memory, the routed groups gathered per batch element on a side stream
+    tiered = None
+    if w.name == "ctx16k" and not args.no_tiered:
+        tiered = _time_tiered(H, HI.WORKLOADS["ctx16k_b4"], args.seed + rank, dev, stream, flush_l2, world)
+
     # roofline of the dominant kernel
     wm = work_model(w)
     pk = _peaks()
@@ -409,6 +447,8 @@ def main():
             line["segment_positions"] = positions
         if budgets:
             line["routing_budget_sweep"] = budgets
+        if tiered:
+            line["tiered_history"] = tiered
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -3,12 +3,14 @@
 The hot path of one attention layer over a detached history plus an active
 segment ("Long-Context Fine-Tuning with Limited VRAM"): key summaries, two-level
 top-k routing, and routed + causal-local attention forward and backward, all in
-the CUDA library ``libhga.so`` behind the C ABI of ``include/hga.h``.
+the CUDA library ``libhga.so`` behind the C ABI of ``include/hga.h``; with the
+history K/V either in device memory (``LayerStep``) or in pinned host memory
+(``TieredLayerStep``).
 """
 from . import _capi
 from ._capi import HGAConfig, HGAError, load
-from .api import (LayerStep, attn_bwd, attn_fwd, build_summaries, hga_attention, make_config,
+from .api import (LayerStep, TieredLayerStep, attn_bwd, attn_fwd, build_summaries, hga_attention, make_config,
                   new_workspace, read_status, route)
 
-__all__ = ["HGAConfig", "HGAError", "LayerStep", "attn_bwd", "attn_fwd", "build_summaries", "hga_attention",
-           "load", "make_config", "new_workspace", "read_status", "route", "_capi"]
+__all__ = ["HGAConfig", "HGAError", "LayerStep", "TieredLayerStep", "attn_bwd", "attn_fwd", "build_summaries",
+           "hga_attention", "load", "make_config", "new_workspace", "read_status", "route", "_capi"]

@@ -28,6 +28,7 @@ HGA_BF16 = 1
 #: every entry point declared in include/hga.h
 EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
+           "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
            "hga_read_status", "hga_strerror", "hga_version")
 
 
@@ -72,6 +73,9 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd_dkdv": [C, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_dq": [C, P, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_noalloc": [C, P, P, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_tier_cache_config": [C, C],
+        "hga_tier_plan": [C, P, P, P, P, P, P],
+        "hga_tier_gather": [C, P, P, P, P, P, P, P],
         "hga_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
         "hga_strerror": [ctypes.c_int],
         "hga_version": [],
@@ -149,6 +153,21 @@ def attn_bwd_noalloc(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_
     library's fixed per-device scratch is used instead; overlapping calls race)."""
     _call("hga_attn_bwd_noalloc", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o,
           dq, dk_seg, dv_seg, stream)
+
+
+def tier_cache_config(cfg) -> HGAConfig:
+    """Configuration of the attention calls over the compact history cache of a tiered step."""
+    out = HGAConfig()
+    _call("hga_tier_cache_config", ctypes.byref(cfg), ctypes.byref(out))
+    return out
+
+
+def tier_plan(cfg, group_idx, used_groups, n_used, compact_idx, workspace, stream=0) -> None:
+    _call("hga_tier_plan", ctypes.byref(cfg), group_idx, used_groups, n_used, compact_idx, workspace, stream)
+
+
+def tier_gather(cfg, k_hist, v_hist, used_groups, n_used, k_cache, v_cache, stream=0) -> None:
+    _call("hga_tier_gather", ctypes.byref(cfg), k_hist, v_hist, used_groups, n_used, k_cache, v_cache, stream)
 
 
 def read_status(workspace, stream=0) -> int:

@@ -13,6 +13,7 @@ gradients.
 from __future__ import annotations
 
 import math
+import time
 
 import torch
 
@@ -223,6 +224,104 @@ class LayerStep:
     def __call__(self, x: dict) -> None:
         for _, call in self.calls(x):
             call()
+
+
+class TieredLayerStep:
+    """One layer step with the detached history K/V in pinned host memory (tiered storage,
+    "Technical Summary" 2.2): the summaries and the routing stay in device memory; per step only
+    the K/V of the routed groups are gathered into a compact device cache.  The gather runs one
+    batch element at a time on a side stream, so the copy of element b+1 over the host link
+    overlaps the forward and backward of element b on the caller's stream.
+
+    k_hist_host / v_hist_host: pinned CPU tensors [B, Hkv, H, D] (``pin_memory=True``);
+    group_sum / chunk_sum: the device summaries of that history (built when it was written)."""
+
+    def __init__(self, cfg, k_hist_host, v_hist_host, group_sum, chunk_sum, device="cuda"):
+        dev = torch.device(device)
+        B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
+        dt = _tdtype(cfg)
+        for name, t in (("k_hist_host", k_hist_host), ("v_hist_host", v_hist_host)):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError(f"{name} must be pinned host memory")
+            if tuple(t.shape) != (B, Hkv, H, D) or t.dtype != dt or not t.is_contiguous():
+                raise ValueError(f"{name}: expected contiguous {dt} {(B, Hkv, H, D)}, got {t.dtype} "
+                                 f"{tuple(t.shape)}")
+        self.cfg, self.dev = cfg, dev
+        self.ccfg = C.tier_cache_config(cfg)
+        self.cfg1 = C.make_config(1, Hq, Hkv, H, S, cfg.top_chunks, cfg.top_groups, dtype=cfg.dtype, D=D,
+                                  softmax_scale=cfg.softmax_scale, n_sink_tokens=cfg.n_sink_tokens)
+        self.ccfg1 = C.tier_cache_config(self.cfg1)
+        self.cap = self.ccfg.hist_len // cfg.group
+        nblk = S // cfg.qblock
+        self.k_host, self.v_host = k_hist_host, v_hist_host
+        self.group_sum, self.chunk_sum = group_sum, chunk_sum
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.chunk_idx = torch.empty(B, Hkv, nblk, cfg.top_chunks, **i32)
+        self.group_idx = torch.empty(B, Hkv, nblk, cfg.top_groups, **i32)
+        self.compact_idx = torch.empty(B, Hkv, nblk, cfg.top_groups, **i32)
+        self.used_groups = torch.empty(B, Hkv, self.cap, **i32)
+        self.n_used = torch.empty(B * Hkv, **i32)
+        self.k_cache = torch.empty(B, Hkv, self.cap * cfg.group, D, dtype=dt, device=dev)
+        self.v_cache = torch.empty_like(self.k_cache)
+        self.ws = new_workspace(cfg, dev)
+        self.ws1 = [new_workspace(self.cfg1, dev) for _ in range(B)]
+        self.o = torch.empty(B, Hq, S, D, dtype=dt, device=dev)
+        self.lse = torch.empty(B, Hq, S, dtype=torch.float32, device=dev)
+        self.dq = torch.empty_like(self.o)
+        self.dk = torch.empty(B, Hkv, S, D, dtype=dt, device=dev)
+        self.dv = torch.empty_like(self.dk)
+        self.side = torch.cuda.Stream(dev)
+        self.planned = torch.cuda.Event()
+        self.gathered = [torch.cuda.Event() for _ in range(B)]
+        self.done = torch.cuda.Event()
+
+    def __call__(self, x: dict, backward: bool = True) -> None:
+        """Enqueue one step (routing, plan, per-element gather + forward [+ backward]) for
+        x = {q, k_seg, v_seg[, d_o]} on the current stream; returns without synchronising."""
+        cfg, c1 = self.cfg, self.ccfg1
+        main = torch.cuda.current_stream(self.dev)
+        st, side = main.cuda_stream, self.side.cuda_stream
+        ws = self.ws.data_ptr()
+        C.route(cfg, x["q"].data_ptr(), self.group_sum.data_ptr(), self.chunk_sum.data_ptr(),
+                self.chunk_idx.data_ptr(), self.group_idx.data_ptr(), ws, st)
+        C.tier_plan(cfg, self.group_idx.data_ptr(), self.used_groups.data_ptr(), self.n_used.data_ptr(),
+                    self.compact_idx.data_ptr(), ws, st)
+        self.planned.record(main)
+        self.side.wait_event(self.planned)
+        for b in range(cfg.B):
+            C.tier_gather(self.cfg1, self.k_host[b].data_ptr(), self.v_host[b].data_ptr(),
+                          self.used_groups[b].data_ptr(), self.n_used[b * cfg.Hkv:].data_ptr(),
+                          self.k_cache[b].data_ptr(), self.v_cache[b].data_ptr(), side)
+            self.gathered[b].record(self.side)
+        for b in range(cfg.B):
+            main.wait_event(self.gathered[b])
+            w1 = self.ws1[b].data_ptr()
+            q, ks, vs = x["q"][b].data_ptr(), x["k_seg"][b].data_ptr(), x["v_seg"][b].data_ptr()
+            kc, vc, gi = self.k_cache[b].data_ptr(), self.v_cache[b].data_ptr(), self.compact_idx[b].data_ptr()
+            o, lse = self.o[b].data_ptr(), self.lse[b].data_ptr()
+            C.attn_fwd(c1, q, kc, vc, ks, vs, gi, o, lse, w1, st)
+            if backward:
+                C.attn_bwd(c1, q, kc, vc, ks, vs, gi, o, lse, x["d_o"][b].data_ptr(), self.dq[b].data_ptr(),
+                           self.dk[b].data_ptr(), self.dv[b].data_ptr(), w1, st)
+        self.done.record(main)
+
+    def wait(self, timeout_s: float = 30.0) -> None:
+        """Host-side wait for the last enqueued step with a deadline: raises TimeoutError instead of
+        blocking forever if the host link or the device stalls; raises on a device status error."""
+        deadline = time.monotonic() + timeout_s
+        while not self.done.query():
+            if time.monotonic() > deadline:
+                raise TimeoutError(f"tiered layer step not finished after {timeout_s} s")
+            time.sleep(50e-6)
+        for w in [self.ws, *self.ws1]:
+            code = read_status(w)
+            if code != 0:
+                raise C.HGAError("tiered step (device status)", code)
+
+    def gather_bytes(self) -> int:
+        """Bytes of history K/V the last step copied into the cache (K and V)."""
+        esz = 2 if self.cfg.dtype == C.HGA_BF16 else 4
+        return int(self.n_used.sum().item()) * self.cfg.group * self.cfg.D * esz * 2
 
 
 def default_scale(D: int = 128) -> float:

@@ -39,6 +39,13 @@ cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const v
                                const void* vs, const int32_t* gi, const float* lse, const void* d_o,
                                const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
                                int nsg, float scale, int* status, cudaStream_t st);
+size_t tier_plan_smem_bytes(int ngr);
+cudaError_t launch_tier_plan(const int32_t* group_idx, int BHkv, int nblk, int kg, int nsg, int ngr, int cap,
+                             int32_t* used_groups, int32_t* n_used, int32_t* compact_idx, int* status,
+                             cudaStream_t st);
+cudaError_t launch_tier_gather(bool bf16, const void* kh, const void* vh, const int32_t* used_groups,
+                               const int32_t* n_used, int BHkv, int64_t H, int cap, void* kc, void* vc,
+                               cudaStream_t st);
 }  // namespace hga
 
 namespace {
@@ -84,6 +91,15 @@ int check_ptrs(std::initializer_list<const void*> ps) {
 
 // Groups of the sink window, attended by every query ahead of the routed groups.
 int sink_groups(const hga_config_t* c) { return (int)(c->n_sink_tokens / c->group); }
+
+// int32 index arrays are read and written with 4-byte accesses: non-null and 4-byte aligned.
+int check_idx(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p) return HGA_ERR_ARG;
+  for (const void* p : ps)
+    if (reinterpret_cast<uintptr_t>(p) & 3u) return HGA_ERR_ALIGN;
+  return HGA_OK;
+}
 
 float eff_scale(const hga_config_t* c) {
   return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->D);
@@ -132,6 +148,40 @@ int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const
                                              cfg->top_groups, eff_scale(cfg), st));
 }
 
+// Groups of the compact history cache of a tiered step: every group a step can route to (the
+// sink groups plus k_g per query block, at most the whole history), rounded up to whole chunks, and
+// at least enough whole chunks for the sink and k_g routed groups (so the cache is a valid history
+// for a configuration whose routing budget is ceil(k_g / 8) chunks).
+int64_t tier_cap_groups(const hga_config_t* c) {
+  const int64_t gpc = c->chunk / c->group, ngr = c->hist_len / c->group, nsg = c->n_sink_tokens / c->group;
+  const int64_t nblk = c->seg_len / c->qblock;
+  int64_t cap = nsg + nblk * c->top_groups;
+  if (cap > ngr) cap = ngr;
+  const int64_t least = nsg + gpc * ((c->top_groups + gpc - 1) / gpc);
+  if (cap < least) cap = least;
+  cap = (cap + gpc - 1) / gpc * gpc;
+  return cap < ngr ? cap : ngr;
+}
+
+// Device-accessible address of a buffer of `bytes` bytes that is either device memory or pinned
+// host memory mapped into the device's address space (both ends checked); nullptr otherwise.
+const void* device_view(const void* p, size_t bytes) {
+  const char* ends[2] = {static_cast<const char*>(p), static_cast<const char*>(p) + (bytes ? bytes - 1 : 0)};
+  const void* dev = nullptr;
+  for (int i = 0; i < 2; ++i) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, ends[i]) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeHost && a.type != cudaMemoryTypeManaged) ||
+        a.devicePointer == nullptr)
+      return nullptr;
+    if (i == 0) dev = a.devicePointer;
+  }
+  return dev;
+}
+
 }  // namespace
 
 // The whole backward with a workspace of ws_bytes (also used by the no-allocation entry point).
@@ -141,7 +191,8 @@ int hga_internal_attn_bwd_ws(const hga_config_t* cfg, const void* q, const void*
                              size_t ws_bytes, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
+  if ((rc = check_idx({group_idx}))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
@@ -190,7 +241,8 @@ int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, co
               int32_t* chunk_idx, int32_t* group_idx, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, group_sum, chunk_sum, chunk_idx, group_idx}))) return rc;
+  if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
+  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   (void)workspace;
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, group_sum, chunk_sum, chunk_idx, group_idx, cfg->B,
                                      cfg->Hq, cfg->Hkv, cfg->seg_len, (int)(cfg->hist_len / cfg->chunk),
@@ -202,7 +254,8 @@ int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
                  const void* v_seg, const int32_t* group_idx, void* o, float* lse, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse}))) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, o, lse}))) return rc;
+  if ((rc = check_idx({group_idx}))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   const bool bf16 = cfg->dtype == HGA_BF16;
@@ -239,7 +292,8 @@ int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, 
                     void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq}))) return rc;
+  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, lse, d_o, dq}))) return rc;
+  if ((rc = check_idx({group_idx}))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -260,6 +314,47 @@ int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
   if (rc) return rc;
   return hga_internal_attn_bwd_ws(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, dk_seg, dv_seg,
                                   workspace, full_workspace_bytes(cfg), stream);
+}
+
+int hga_tier_cache_config(const hga_config_t* cfg, hga_config_t* cache_cfg) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!cache_cfg) return HGA_ERR_ARG;
+  *cache_cfg = *cfg;
+  cache_cfg->hist_len = tier_cap_groups(cfg) * cfg->group;
+  cache_cfg->top_chunks = (cfg->top_groups + (cfg->chunk / cfg->group) - 1) / (cfg->chunk / cfg->group);
+  return check_config(cache_cfg);
+}
+
+int hga_tier_plan(const hga_config_t* cfg, const int32_t* group_idx, int32_t* used_groups, int32_t* n_used,
+                  int32_t* compact_idx, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_idx({group_idx, used_groups, n_used, compact_idx}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  const int64_t ngr = cfg->hist_len / cfg->group;
+  if (hga::tier_plan_smem_bytes((int)ngr) > 200 * 1024) return HGA_ERR_UNSUPPORTED;
+  return from_cuda(hga::launch_tier_plan(group_idx, cfg->B * cfg->Hkv, (int)(cfg->seg_len / cfg->qblock),
+                                         cfg->top_groups, sink_groups(cfg), (int)ngr, (int)tier_cap_groups(cfg),
+                                         used_groups, n_used, compact_idx, status_of(workspace),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int hga_tier_gather(const hga_config_t* cfg, const void* k_hist, const void* v_hist, const int32_t* used_groups,
+                    const int32_t* n_used, void* k_cache, void* v_cache, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({k_hist, v_hist, k_cache, v_cache}))) return rc;
+  if ((rc = check_idx({used_groups, n_used}))) return rc;
+  const size_t esz = cfg->dtype == HGA_BF16 ? 2 : 4;
+  const size_t hist_bytes = (size_t)cfg->B * cfg->Hkv * cfg->hist_len * cfg->D * esz;
+  const void* kh = device_view(k_hist, hist_bytes);
+  const void* vh = device_view(v_hist, hist_bytes);
+  if (!kh || !vh) return HGA_ERR_ARG;        // pageable host memory cannot be read by the device
+  return from_cuda(hga::launch_tier_gather(cfg->dtype == HGA_BF16, kh, vh, used_groups, n_used, cfg->B * cfg->Hkv,
+                                           cfg->hist_len, (int)tier_cap_groups(cfg), k_cache, v_cache,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int hga_read_status(void* workspace, void* stream, int32_t* status_out) {

@@ -29,7 +29,8 @@
  *
  * Conventions for every entry point
  *   - Memory: the caller allocates and owns every buffer, including the
- *     workspace.  All tensor pointers are DEVICE pointers, 16-byte aligned,
+ *     workspace.  All tensor pointers are DEVICE pointers, 16-byte aligned
+ *     (int32 index arrays: 4-byte aligned),
  *     contiguous, head-major: q, o, d_o, dq: [B, Hq, S, D]; k/v history:
  *     [B, Hkv, H, D]; k/v segment, dk/dv segment: [B, Hkv, S, D].  Query head
  *     h uses KV head h / (Hq / Hkv).  Element type: float32 or bfloat16 as
@@ -196,6 +197,51 @@ HGA_API int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, const v
                                  const int32_t* group_idx, const void* o, const float* lse,
                                  const void* d_o, void* dq, void* dk_seg, void* dv_seg,
                                  void* stream);
+
+/* ---------------------------------------------------------------- tiered history
+ * Tiered storage ("Technical Summary" 2.2, "Tiered Memory Hierarchy"; pith.science
+ * review, Figure 2 caption): the detached history K/V stay in host memory, the
+ * summaries in device memory, and a layer step brings into device memory only the
+ * exact K/V of the groups its routing selected.  Per step, after hga_route:
+ *   1. hga_tier_plan: per (batch, KV head) the ascending list of every history group
+ *      any block routed to (sink groups included), and each block's routed indices
+ *      rewritten as positions in that list;
+ *   2. hga_tier_gather: those groups' K/V rows copied from the history into a
+ *      compact cache [B, Hkv, cap*8, D] in device memory;
+ *   3. hga_attn_fwd / hga_attn_bwd with the configuration from
+ *      hga_tier_cache_config, the cache as k_hist / v_hist and the rewritten
+ *      indices as group_idx.  Positions keep the order of the group indices, so
+ *      the results equal those over the full history bit for bit.
+ * The cache holds cap groups per (batch, KV head): cap = min(H/8, sink groups +
+ * (S/64) * top_groups), raised to at least the sink plus ceil(top_groups/8)
+ * chunks, rounded up to whole chunks (cache_cfg->hist_len = 8 * cap). */
+
+/* *cache_cfg = cfg with hist_len = 8 * cap and top_chunks = ceil(top_groups / 8):
+ * the configuration of the attention calls over the compact cache. */
+HGA_API int hga_tier_cache_config(const hga_config_t* cfg, hga_config_t* cache_cfg);
+
+/* group_idx [B, Hkv, S/64, top_groups] (device, from hga_route with cfg) ->
+ * used_groups [B, Hkv, cap] (ascending; entries past n_used unspecified),
+ * n_used [B*Hkv], compact_idx [B, Hkv, S/64, top_groups] (all device int32).
+ * A routed index outside [n_sink_tokens/8, H/8) is left out of the list, maps to
+ * position 0 and records HGA_ERR_ARG in the workspace status word.  Asynchronous
+ * on `stream`; needs the workspace only for its status word. */
+HGA_API int hga_tier_plan(const hga_config_t* cfg, const int32_t* group_idx,
+                          int32_t* used_groups, int32_t* n_used, int32_t* compact_idx,
+                          void* workspace, void* stream);
+
+/* Copies the K and V rows of used_groups[b, kh, 0 .. n_used) from k_hist / v_hist
+ * [B, Hkv, H, D] into k_cache / v_cache [B, Hkv, cap*8, D] (device), group
+ * position p to cache rows 8p .. 8p+7.  k_hist / v_hist may be device memory or
+ * pinned host memory mapped into the device address space (cudaHostAlloc, or
+ * cudaHostRegister with cudaHostRegisterMapped): the SMs read it over the host
+ * link.  Pageable host memory is rejected with HGA_ERR_ARG before any launch (the
+ * device cannot read it).  Cache rows past 8 * n_used are not written.
+ * Asynchronous on `stream`: a side stream lets the copy of one batch element
+ * overlap the attention of another. */
+HGA_API int hga_tier_gather(const hga_config_t* cfg, const void* k_hist, const void* v_hist,
+                            const int32_t* used_groups, const int32_t* n_used, void* k_cache,
+                            void* v_cache, void* stream);
 
 /* Synchronises `stream`, copies the workspace status word to *status_out
  * (HGA_OK, HGA_ERR_TIMEOUT or HGA_ERR_ARG, see Workspace above) and clears it.  Returns HGA_ERR_CUDA if the

@@ -111,6 +111,21 @@ def test_sink_window_config_accepted(lib):
     assert C.workspace_size(cfg(n_sink_tokens=13312, top_chunks=16)) == _expected_ws(1, 32, 8, 2048)
 
 
+def test_tier_cache_config(lib):
+    """The compact history cache holds every group a step can route to, in whole chunks."""
+    c = C.tier_cache_config(cfg())                                  # 32 blocks x 64 > 1792 groups
+    assert (c.hist_len, c.top_chunks, c.top_groups) == (14336, 8, 64)
+    c = C.tier_cache_config(cfg(hist_len=129024, top_chunks=32, top_groups=128))
+    assert c.hist_len == 32 * 128 * 8 and c.top_chunks == 16     # 4096 groups of 16128
+    c = C.tier_cache_config(cfg(seg_len=64, top_chunks=4, top_groups=20))
+    assert c.hist_len == 24 * 8                                    # 20 groups -> 3 whole chunks
+    c = C.tier_cache_config(cfg(seg_len=128, top_chunks=4, top_groups=20, n_sink_tokens=128))
+    assert c.hist_len == (16 + 40) * 8 and c.n_sink_tokens == 128   # sink + 2 blocks x 20
+    c = C.tier_cache_config(cfg(seg_len=64, top_chunks=2, top_groups=1))
+    assert c.hist_len == 64 and c.top_chunks == 1                  # at least one chunk
+    assert C.workspace_size(c) > 0                                   # a valid configuration
+
+
 def test_entry_points_reject_bad_pointers_before_launch(lib):
     c = cfg()
     ok, odd = 1 << 20, (1 << 20) + 8             # never dereferenced: validation fails first
