@@ -146,6 +146,31 @@ def route_from_inputs(q, k_hist, Hkv: int, top_chunks: int, top_groups: int, chu
                 chunk_gap=cgap, group_gap=ggap)
 
 
+def route_causal_from_inputs(q, k_hist, Hkv: int, top_chunks: int, top_groups: int, q_prev=None,
+                             chunk: int = 64, group: int = 8, qblock: int = 64, prec: int = 32,
+                             n_sink: int = 0) -> dict:
+    """Strictly causal routing (the variant the pages name as future work, Technical Summary
+    section 5 "Causal Leakage"; reading: block n is routed with the block query of block n-1, so
+    its routing depends on no token at or after the start of block n).  Block 0 uses the block
+    query of ``q_prev`` [B, Hq, qblock, D] (the previous segment's last query block), or a zero
+    query if ``q_prev`` is None."""
+    if n_sink % chunk:
+        raise ValueError("n_sink must be a multiple of the chunk size")
+    gs = group_summaries(k_hist, group, prec)
+    cs = chunk_summaries(k_hist, chunk, prec)
+    qb = block_query(q, Hkv, qblock, prec)
+    if q_prev is None:
+        first = np.zeros_like(qb[:, :, :1])
+    else:
+        first = block_query(q_prev, Hkv, qblock, prec)
+        if first.shape[2] != 1:
+            raise ValueError("q_prev must hold exactly one query block")
+    qbc = np.concatenate([first, qb[:, :, :-1]], axis=2)
+    ci, gi, cgap, ggap = route(qbc, gs, cs, top_chunks, top_groups, prec, n_sink // chunk)
+    return dict(group_sum=gs, chunk_sum=cs, qb=qbc, chunk_idx=ci, group_idx=gi,
+                chunk_gap=cgap, group_gap=ggap)
+
+
 # --------------------------------------------------------------------------- attention
 def _layer(q, k_hist, v_hist, k_seg, v_seg, group_idx):
     q, kh, vh, ks, vs = (_f64(t) for t in (q, k_hist, v_hist, k_seg, v_seg))

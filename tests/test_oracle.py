@@ -392,6 +392,61 @@ def test_within_block_side_channel_is_present(oracle):
     assert not np.allclose(oz[0, 1, :63], o0[0, 1, :63])   # earlier queries of another head moved
 
 
+def test_causal_routing_closes_the_within_block_side_channel(oracle):
+    """Strictly causal variant (block n routed with block n-1's query): the perturbation that moves
+    earlier outputs under the standard routing leaves every earlier output of the block unchanged;
+    it reaches only the next block's routing, whose queries all come after it."""
+    w = HI.WORKLOADS["tiny_f32"]
+    x = HI.make_inputs(w, 0)
+    qp = HI.make_inputs(w.with_(hist_len=64, seg_len=64), 1)["q"]          # previous segment's last block
+    base = oracle.route_causal_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups, q_prev=qp)
+    z = {k: v.clone() for k, v in x.items() if k != "needles"}
+    cs = oracle.chunk_summaries(x["k_hist"])[0, 0]
+    std = oracle.route_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups)
+    other = next(i for i in range(w.nch) if i not in std["chunk_idx"][0, 0, 0])
+    z["q"][0, 0, 63] += torch.as_tensor(cs[other] * 400.0, dtype=z["q"].dtype)
+    rz = oracle.route_causal_from_inputs(z["q"], z["k_hist"], 1, w.top_chunks, w.top_groups, q_prev=qp)
+    assert np.array_equal(rz["group_idx"][:, :, 0], base["group_idx"][:, :, 0])
+    assert other in rz["chunk_idx"][0, 0, 1]                  # the next block's routing moved
+    o0, _ = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], base["group_idx"])
+    oz, _ = oracle.attn_fwd(z["q"], z["k_hist"], z["v_hist"], z["k_seg"], z["v_seg"], rz["group_idx"])
+    assert np.array_equal(oz[:, :, :63], o0[:, :, :63])       # nothing before the change moved
+
+
+def test_causal_routing_is_strictly_causal_at_every_position(oracle):
+    """Changing every query at or after position t (all heads) leaves all outputs before t equal."""
+    w = HI.WORKLOADS["tiny_f32"]
+    x = HI.make_inputs(w, 2)
+    r0 = oracle.route_causal_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups)
+    o0, _ = oracle.attn_fwd(x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r0["group_idx"])
+    g = torch.Generator().manual_seed(3)
+    for t in (1, 63, 64, 100, 200):
+        q = x["q"].clone()
+        q[:, :, t:] = torch.randn(q[:, :, t:].shape, generator=g) * 3
+        r = oracle.route_causal_from_inputs(q, x["k_hist"], 1, w.top_chunks, w.top_groups)
+        o, _ = oracle.attn_fwd(q, x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
+        assert np.array_equal(o[:, :, :t], o0[:, :, :t])
+
+
+def test_causal_routing_is_the_previous_blocks_routing(oracle):
+    """Block n >= 1 gets the standard routing of block n-1; block 0 that of q_prev, or with no
+    q_prev a zero query, whose all-equal scores take the lowest routable indices."""
+    w = HI.WORKLOADS["tiny_f32"].with_(n_sink=128)
+    x = HI.make_inputs(w, 4)
+    qp = HI.make_inputs(w.with_(hist_len=64, seg_len=64), 5)["q"]
+    std = oracle.route_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups, n_sink=128)
+    c = oracle.route_causal_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups, q_prev=qp,
+                                        n_sink=128)
+    assert np.array_equal(c["group_idx"][:, :, 1:], std["group_idx"][:, :, :-1])
+    assert np.array_equal(c["chunk_idx"][:, :, 1:], std["chunk_idx"][:, :, :-1])
+    q0 = torch.cat([qp, x["q"][:, :, 64:]], dim=2)              # a segment whose block 0 is q_prev
+    std0 = oracle.route_from_inputs(q0, x["k_hist"], 1, w.top_chunks, w.top_groups, n_sink=128)
+    assert np.array_equal(c["group_idx"][:, :, 0], std0["group_idx"][:, :, 0])
+    z = oracle.route_causal_from_inputs(x["q"], x["k_hist"], 1, w.top_chunks, w.top_groups, n_sink=128)
+    assert list(z["chunk_idx"][0, 0, 0]) == [2, 3, 4, 5]
+    assert list(z["group_idx"][0, 0, 0]) == list(range(16, 24))
+
+
 def test_row_and_key_subsets_match_full(oracle):
     w = HI.WORKLOADS["tiny_f32"]
     x = HI.make_inputs(w, 4)
