@@ -207,11 +207,14 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3) -> float:
-    """Mean device time (ms) of one whole layer step of workload w, L2 flushed before each step."""
+def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3, causal=False) -> float:
+    """Mean device time (ms) of one whole layer step of workload w, L2 flushed before each step
+    (causal: with the strictly causal routing, the previous segment's last block as q_prev)."""
     x = {k: v.to(dev) for k, v in HI.make_inputs(w, seed).items() if k != "needles"}
+    if causal:
+        x["q_prev"] = HI.prev_block_q(w, seed).to(dev)
     cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
-    step = H.LayerStep(cfg, dev)
+    step = H.LayerStep(cfg, dev, causal_routing=causal)
     calls = step.calls(x, stream.cuda_stream)
     for _ in range(warmup):
         for _, c in calls:
@@ -227,6 +230,34 @@ def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3) -> float:
     if H.read_status(step.ws) != 0:
         raise RuntimeError(f"device status word set while timing {w.name}")
     return sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+
+
+def _leakage_probe(H, w, seed, dev) -> dict:
+    """The pages' probe of the within-block side channel: change a later query of a block and see
+    whether earlier outputs move.  The last query of block 0 (head 0) is pushed towards a chunk block
+    0 did not select; reported is the largest change of any output before it, under the standard and
+    under the strictly causal routing."""
+    x = {k: v.to(dev) for k, v in HI.make_inputs(w, seed).items() if k != "needles"}
+    x["q_prev"] = HI.prev_block_q(w, seed).to(dev)
+    cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    out = {}
+    for name, causal in (("standard", False), ("strictly_causal", True)):
+        s0 = H.LayerStep(cfg, dev, causal_routing=causal)
+        s0.forward(x)
+        torch.cuda.synchronize(dev)
+        if name == "standard":
+            chosen = set(s0.chunk_idx[0, 0, 0].tolist())
+            other = next(i for i in range(w.nch) if i not in chosen)
+            z = dict(x)
+            z["q"] = x["q"].clone()
+            z["q"][0, 0, w.qblock - 1] += (400.0 * s0.chunk_sum[0, 0, other]).to(z["q"].dtype)
+        s1 = H.LayerStep(cfg, dev, causal_routing=causal)
+        s1.forward(z)
+        torch.cuda.synchronize(dev)
+        d = (s0.o[:, :, :w.qblock - 1].float() - s1.o[:, :, :w.qblock - 1].float()).abs().max().item()
+        out[f"{name}_max_abs_change_before"] = d
+    out["perturbed"] = f"query {w.qblock - 1} of head 0 (last of block 0), pushed towards an unselected chunk"
+    return out
 
 
 def _time_tiered(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=2) -> dict:
@@ -366,6 +397,13 @@ def main():
             budgets[f"top_chunks_{pw.top_chunks}_top_groups_{pw.top_groups}"] = {
                 "ms_per_step": ms, "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
 
+    # strictly causal routing (block n routed with block n-1's query): same kernels, other routing
+    causal = None
+    if w.name == "ctx16k" and not args.no_positions:
+        ms = all_max(_time_layer(H, w, args.seed + rank, dev, stream, flush_l2, causal=True), world, dev)
+        causal = {"ms_per_step": ms, "tokens_per_s": w.B * w.seg_len * world / (ms * 1e-3),
+                  "leakage_probe": _leakage_probe(H, w, args.seed + rank, dev)}
+
     # tiered-history variant of the 16K layer at batch 4: history K/V in pinned host memory, the
     # summaries in device memory, the routed groups gathered per batch element on a side stream
     tiered = None
@@ -447,6 +485,8 @@ def main():
             line["segment_positions"] = positions
         if budgets:
             line["routing_budget_sweep"] = budgets
+        if causal:
+            line["strictly_causal_routing"] = causal
         if tiered:
             line["tiered_history"] = tiered
         print(json.dumps(line), flush=True)

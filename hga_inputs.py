@@ -146,6 +146,12 @@ def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu") 
     return out
 
 
+def prev_block_q(w: Workload, seed: int) -> torch.Tensor:
+    """The previous segment's last query block [B, Hq, qblock, D] for strictly causal routing: one
+    query block drawn like ``make_inputs`` queries, with its own seed (seed + 100)."""
+    return make_inputs(w.with_(hist_len=w.chunk, seg_len=w.qblock, n_sink=0, needles=0), seed + 100)["q"]
+
+
 def sample_ids(n_total: int, n: int, seed: int) -> torch.Tensor:
     """``n`` distinct ids in [0, n_total), sorted, from a seeded generator (for sampled checks)."""
     g = torch.Generator().manual_seed(int(seed) + 7919)

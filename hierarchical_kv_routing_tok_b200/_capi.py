@@ -26,7 +26,8 @@ HGA_F32 = 0
 HGA_BF16 = 1
 
 #: every entry point declared in include/hga.h
-EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd",
+EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
+           "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
            "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
            "hga_read_status", "hga_strerror", "hga_version")
@@ -67,6 +68,7 @@ def load() -> ctypes.CDLL:
         "hga_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
         "hga_build_summaries": [C, P, P, P, P, P],
         "hga_route": [C, P, P, P, P, P, P, P],
+        "hga_route_causal": [C, P, P, P, P, P, P, P, P],
         "hga_attn_fwd": [C, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_preprocess": [C, P, P, P, P],
@@ -121,6 +123,12 @@ def build_summaries(cfg, k_hist, group_sum, chunk_sum, workspace, stream=0) -> N
 
 def route(cfg, q, group_sum, chunk_sum, chunk_idx, group_idx, workspace, stream=0) -> None:
     _call("hga_route", ctypes.byref(cfg), q, group_sum, chunk_sum, chunk_idx, group_idx, workspace, stream)
+
+
+def route_causal(cfg, q, q_prev, group_sum, chunk_sum, chunk_idx, group_idx, workspace, stream=0) -> None:
+    """Strictly causal routing: block n routed with block n-1's query (block 0: q_prev, or 0 = none)."""
+    _call("hga_route_causal", ctypes.byref(cfg), q, q_prev, group_sum, chunk_sum, chunk_idx, group_idx, workspace,
+          stream)
 
 
 def attn_fwd(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, workspace, stream=0) -> None:

@@ -73,7 +73,11 @@ def build_summaries(cfg, k_hist, group_sum=None, chunk_sum=None, workspace=None)
     return group_sum, chunk_sum
 
 
-def route(cfg, q, group_sum, chunk_sum, chunk_idx=None, group_idx=None, workspace=None):
+def route(cfg, q, group_sum, chunk_sum, chunk_idx=None, group_idx=None, workspace=None, causal: bool = False,
+          q_prev=None):
+    """Two-level routing of every query block.  causal=True: the strictly causal variant -- block n
+    is routed with block n-1's query, block 0 with q_prev [B, Hq, 64, D] (the previous segment's
+    last query block) or, when q_prev is None, a zero query."""
     B, Hq, Hkv, S, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.D
     nblk = S // cfg.qblock
     _need(q, "q", (B, Hq, S, D), _tdtype(cfg))
@@ -86,8 +90,18 @@ def route(cfg, q, group_sum, chunk_sum, chunk_idx=None, group_idx=None, workspac
     _need(chunk_sum, "chunk_sum", (B, Hkv, cfg.hist_len // cfg.chunk, D), torch.float32)
     _need(chunk_idx, "chunk_idx", (B, Hkv, nblk, cfg.top_chunks), torch.int32)
     _need(group_idx, "group_idx", (B, Hkv, nblk, cfg.top_groups), torch.int32)
-    C.route(cfg, q.data_ptr(), group_sum.data_ptr(), chunk_sum.data_ptr(), chunk_idx.data_ptr(),
-            group_idx.data_ptr(), workspace.data_ptr() if workspace is not None else None, _stream(q))
+    ws = workspace.data_ptr() if workspace is not None else None
+    if causal:
+        if q_prev is not None:
+            _need(q_prev, "q_prev", (B, Hq, cfg.qblock, D), _tdtype(cfg))
+        C.route_causal(cfg, q.data_ptr(), q_prev.data_ptr() if q_prev is not None else None,
+                       group_sum.data_ptr(), chunk_sum.data_ptr(), chunk_idx.data_ptr(), group_idx.data_ptr(), ws,
+                       _stream(q))
+    elif q_prev is not None:
+        raise ValueError("q_prev is only used by the causal routing")
+    else:
+        C.route(cfg, q.data_ptr(), group_sum.data_ptr(), chunk_sum.data_ptr(), chunk_idx.data_ptr(),
+                group_idx.data_ptr(), ws, _stream(q))
     return chunk_idx, group_idx
 
 
@@ -176,8 +190,9 @@ class LayerStep:
     """One full pass of the hot path (summaries, routing, forward, backward) over preallocated
     buffers, for a fixed configuration.  Used by the benchmark and the smoke check."""
 
-    def __init__(self, cfg, device="cuda"):
+    def __init__(self, cfg, device="cuda", causal_routing: bool = False):
         self.cfg = cfg
+        self.causal_routing = causal_routing
         dev = torch.device(device)
         B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
         dt = _tdtype(cfg)
@@ -203,7 +218,8 @@ class LayerStep:
         o, lse, dq, dk, dv = (t.data_ptr() for t in (self.o, self.lse, self.dq, self.dk, self.dv))
         return [
             ("summaries", lambda: C.build_summaries(cfg, p["k_hist"], gs, cs, ws, st)),
-            ("route", lambda: C.route(cfg, p["q"], gs, cs, ci, gi, ws, st)),
+            ("route", (lambda: C.route_causal(cfg, p["q"], p.get("q_prev"), gs, cs, ci, gi, ws, st))
+             if self.causal_routing else (lambda: C.route(cfg, p["q"], gs, cs, ci, gi, ws, st))),
             ("attn_fwd", lambda: C.attn_fwd(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi, o,
                                             lse, ws, st)),
             ("bwd_preprocess", lambda: C.attn_bwd_preprocess(cfg, o, p["d_o"], ws, st)),

@@ -12,9 +12,9 @@
 namespace hga {
 cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum,
                              int64_t n_chunks_total, cudaStream_t stream);
-cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
-                         int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S, int nch,
-                         int nsc, int kc, int kg, cudaStream_t stream);
+cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
+                         const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
+                         int64_t S, int nch, int nsc, int kc, int kg, cudaStream_t stream);
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
@@ -244,10 +244,24 @@ int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, co
   if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
   if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   (void)workspace;
-  return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, group_sum, chunk_sum, chunk_idx, group_idx, cfg->B,
-                                     cfg->Hq, cfg->Hkv, cfg->seg_len, (int)(cfg->hist_len / cfg->chunk),
-                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
-                                     static_cast<cudaStream_t>(stream)));
+  return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, nullptr, false, group_sum, chunk_sum, chunk_idx,
+                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
+                                     (int)(cfg->hist_len / cfg->chunk), (int)(cfg->n_sink_tokens / cfg->chunk),
+                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
+}
+
+int hga_route_causal(const hga_config_t* cfg, const void* q, const void* q_prev, const float* group_sum,
+                     const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
+  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
+  if (q_prev && !aligned16(q_prev)) return HGA_ERR_ALIGN;
+  (void)workspace;
+  return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, q_prev, true, group_sum, chunk_sum, chunk_idx,
+                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
+                                     (int)(cfg->hist_len / cfg->chunk), (int)(cfg->n_sink_tokens / cfg->chunk),
+                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
 }
 
 int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,

@@ -192,9 +192,9 @@ __device__ __forceinline__ void score_rows(const float* qb, const float* __restr
 
 template <typename T>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
-    const T* __restrict__ q, const float* __restrict__ group_sum, const float* __restrict__ chunk_sum,
-    int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq, int Hkv, int64_t S, int nch,
-    int nsc, int kc, int kg) {
+    const T* __restrict__ q, const T* __restrict__ q_prev, int causal, const float* __restrict__ group_sum,
+    const float* __restrict__ chunk_sum, int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq,
+    int Hkv, int64_t S, int nch, int nsc, int kc, int kg) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int N = Vec16<T>::N;
   constexpr int LPR = kD / N;
@@ -214,7 +214,23 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   int* gpos = csel + ((kc + 3) & ~3);                             // [kg]
   uint32_t* keys = reinterpret_cast<uint32_t*>(gpos + ((kg + 3) & ~3));   // [max(nch, 8kc) rounded to 4]
 
-  // ---- block query: mean over G heads x 64 positions
+  // ---- block query: mean over G heads x 64 positions of the routing block -- block n itself, or
+  // for strictly causal routing block n-1 (block 0: the previous segment's last block q_prev
+  // [B, Hq, 64, D], or a zero query when there is none)
+  const T* qsrc = q;
+  int64_t s_src = S, t_src = (int64_t)n * kQBlock;
+  bool zero_query = false;
+  if (causal) {
+    if (n > 0) {
+      t_src -= kQBlock;
+    } else if (q_prev) {
+      qsrc = q_prev;
+      s_src = kQBlock;
+      t_src = 0;
+    } else {
+      zero_query = true;
+    }
+  }
   {
     const int tid = threadIdx.x;
     const int col = (tid % LPR) * N, r0 = tid / LPR;
@@ -228,10 +244,10 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
 #pragma unroll
       for (int u = 0; u < UQ; ++u) {
         const int r = r1 + u * RP;
-        if (r < R) {
+        if (r < R && !zero_query) {
           const int h = kh * G + r / kQBlock;
-          const int64_t t = (int64_t)n * kQBlock + r % kQBlock;
-          raw[u] = *reinterpret_cast<const uint4*>(q + (((int64_t)b * Hq + h) * S + t) * kD + col);
+          const int64_t t = t_src + r % kQBlock;
+          raw[u] = *reinterpret_cast<const uint4*>(qsrc + (((int64_t)b * Hq + h) * s_src + t) * kD + col);
         } else {
           raw[u] = make_uint4(0, 0, 0, 0);
         }
@@ -294,9 +310,9 @@ size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
   return words * 4;
 }
 
-cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const float* chunk_sum,
-                         int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv, int64_t S,
-                         int nch, int nsc, int kc, int kg, cudaStream_t stream) {
+cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
+                         const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
+                         int64_t S, int nch, int nsc, int kc, int kg, cudaStream_t stream) {
   const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
   if (units == 0) return cudaSuccess;
   const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
@@ -305,13 +321,14 @@ cudaError_t launch_route(bool bf16, const void* q, const float* group_sum, const
     e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     route_kernel<__nv_bfloat16><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc,
-        kc, kg);
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(q_prev), causal ? 1 : 0, group_sum,
+        chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
   } else {
     e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     route_kernel<float><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const float*>(q), group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
+        static_cast<const float*>(q), static_cast<const float*>(q_prev), causal ? 1 : 0, group_sum, chunk_sum,
+        chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
   }
   return cudaGetLastError();
 }

@@ -131,6 +131,18 @@ HGA_API int hga_route(const hga_config_t* cfg, const void* q, const float* group
               const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx,
               void* workspace, void* stream);
 
+/* Strictly causal routing: as hga_route, except that block n is routed with the
+ * block query of block n-1 (block 0 with that of q_prev, the previous segment's
+ * last query block [B, Hq, qblock, D], same dtype; q_prev = NULL routes block 0
+ * with a zero query, so ties give it the lowest routable indices).  The routing of
+ * block n then depends on no token at or after the start of block n, which closes
+ * the within-block side channel ("Technical Summary" section 5, "Causal Leakage":
+ * a strictly causal variant is named there as future work).  The attention calls
+ * are unchanged. */
+HGA_API int hga_route_causal(const hga_config_t* cfg, const void* q, const void* q_prev,
+                             const float* group_sum, const float* chunk_sum, int32_t* chunk_idx,
+                             int32_t* group_idx, void* workspace, void* stream);
+
 /* Forward (Technical Summary 2.1 "Exact-Token Attention"; review Figure 2):
  * query (b, h, t) of block n = t/64 attends to the exact history tokens
  * 8j..8j+7 of every j in group_idx[b, h/G, n, :] and to the segment tokens

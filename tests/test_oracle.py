@@ -509,6 +509,21 @@ def test_parity_seeds_have_routing_margins(oracle, name):
         assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
 
 
+@pytest.mark.parametrize("name", ["small_bf16", "sink_bf16", "ctx16k"])
+def test_causal_parity_inputs_have_routing_margins(oracle, name):
+    """Block 0 of the causal routing in the GPU tests is routed with a separately drawn previous
+    block; its selection boundaries have the same margins as the other parity inputs."""
+    w = HI.WORKLOADS.get(name) or HI.EDGE_WORKLOADS[name]
+    x = HI.make_inputs(w, 0)
+    qp = HI.prev_block_q(w, 0)
+    kw = dict(q_prev=qp, n_sink=w.n_sink)
+    r32 = oracle.route_causal_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32, **kw)
+    r64 = oracle.route_causal_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=64, **kw)
+    assert np.array_equal(r32["chunk_idx"], r64["chunk_idx"])
+    assert np.array_equal(r32["group_idx"], r64["group_idx"])
+    assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
+
+
 def test_needles_recovered_at_131k(oracle):
     """131072-token workload: every planted needle group is routed to its target block."""
     w = HI.WORKLOADS["ctx131k"]
