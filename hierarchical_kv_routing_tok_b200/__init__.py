@@ -11,6 +11,8 @@ from . import _capi
 from ._capi import HGAConfig, HGAError, load
 from .api import (LayerStep, TieredLayerStep, attn_bwd, attn_fwd, build_summaries, hga_attention, make_config,
                   new_workspace, read_status, route)
+from .segment import HGAHistory, segment_attention
 
-__all__ = ["HGAConfig", "HGAError", "LayerStep", "TieredLayerStep", "attn_bwd", "attn_fwd", "build_summaries",
-           "hga_attention", "load", "make_config", "new_workspace", "read_status", "route", "_capi"]
+__all__ = ["HGAConfig", "HGAError", "HGAHistory", "LayerStep", "TieredLayerStep", "attn_bwd", "attn_fwd",
+           "build_summaries", "hga_attention", "load", "make_config", "new_workspace", "read_status", "route",
+           "segment_attention", "_capi"]

@@ -26,7 +26,7 @@ HGA_F32 = 0
 HGA_BF16 = 1
 
 #: every entry point declared in include/hga.h
-EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
+EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_append_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
            "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
            "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
@@ -39,7 +39,8 @@ class HGAConfig(ctypes.Structure):
                 ("hist_len", ctypes.c_int64), ("seg_len", ctypes.c_int64),
                 ("chunk", ctypes.c_int32), ("group", ctypes.c_int32), ("qblock", ctypes.c_int32),
                 ("top_chunks", ctypes.c_int32), ("top_groups", ctypes.c_int32),
-                ("n_sink_tokens", ctypes.c_int32), ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+                ("n_sink_tokens", ctypes.c_int32), ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("hist_capacity", ctypes.c_int64)]
 
     def __repr__(self):
         return "HGAConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -67,6 +68,7 @@ def load() -> ctypes.CDLL:
     sig = {
         "hga_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
         "hga_build_summaries": [C, P, P, P, P, P],
+        "hga_append_summaries": [C, P, P, P, ctypes.c_int64, P, P],
         "hga_route": [C, P, P, P, P, P, P, P],
         "hga_route_causal": [C, P, P, P, P, P, P, P, P],
         "hga_attn_fwd": [C, P, P, P, P, P, P, P, P, P, P],
@@ -106,9 +108,9 @@ def _call(name: str, *args) -> None:
 
 def make_config(B: int, Hq: int, Hkv: int, hist_len: int, seg_len: int, top_chunks: int, top_groups: int,
                 dtype: int = HGA_BF16, D: int = 128, softmax_scale: float = 0.0, chunk: int = 64,
-                group: int = 8, qblock: int = 64, n_sink_tokens: int = 0) -> HGAConfig:
+                group: int = 8, qblock: int = 64, n_sink_tokens: int = 0, hist_capacity: int = 0) -> HGAConfig:
     return HGAConfig(B, Hq, Hkv, D, hist_len, seg_len, chunk, group, qblock, top_chunks, top_groups,
-                     n_sink_tokens, dtype, softmax_scale)
+                     n_sink_tokens, dtype, softmax_scale, hist_capacity)
 
 
 def workspace_size(cfg: HGAConfig) -> int:
@@ -119,6 +121,11 @@ def workspace_size(cfg: HGAConfig) -> int:
 
 def build_summaries(cfg, k_hist, group_sum, chunk_sum, workspace, stream=0) -> None:
     _call("hga_build_summaries", ctypes.byref(cfg), k_hist, group_sum, chunk_sum, workspace, stream)
+
+
+def append_summaries(cfg, k_hist, group_sum, chunk_sum, first_token, workspace, stream=0) -> None:
+    _call("hga_append_summaries", ctypes.byref(cfg), k_hist, group_sum, chunk_sum, int(first_token), workspace,
+          stream)
 
 
 def route(cfg, q, group_sum, chunk_sum, chunk_idx, group_idx, workspace, stream=0) -> None:

@@ -100,6 +100,7 @@ struct Dims {
   int Hq, Hkv, G, kg, nblk;
   int nsg;              // sink groups at the start of every block's history key list
   int64_t H, S;
+  int64_t Hs;           // history rows per (batch, KV head) in k_hist / v_hist (>= H)
   float scale;
   int* status;          // workspace status word (HGA_ERR_ARG recorded for an out-of-range group index)
 };
@@ -142,8 +143,8 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const T* __restrict__ q, 
   const int kh = h / dm.G;
   const int64_t bkh = (int64_t)b * dm.Hkv + kh;
   const T* qrow = q + ((int64_t)bh * dm.S + (int64_t)n * BM) * kD;
-  const T* kh_base = k_hist + bkh * dm.H * kD;
-  const T* vh_base = v_hist + bkh * dm.H * kD;
+  const T* kh_base = k_hist + bkh * dm.Hs * kD;
+  const T* vh_base = v_hist + bkh * dm.Hs * kD;
   const T* ks_base = k_seg + bkh * dm.S * kD;
   const T* vs_base = v_seg + bkh * dm.S * kD;
   const int32_t* gi = group_idx + (bkh * dm.nblk + n) * dm.kg;
@@ -271,8 +272,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(const T* __restrict__ 
   const int kh = h / dm.G;
   const int64_t bkh = (int64_t)b * dm.Hkv + kh;
   const int64_t row0 = (int64_t)bh * dm.S + (int64_t)n * BM;
-  const T* kh_base = k_hist + bkh * dm.H * kD;
-  const T* vh_base = v_hist + bkh * dm.H * kD;
+  const T* kh_base = k_hist + bkh * dm.Hs * kD;
+  const T* vh_base = v_hist + bkh * dm.Hs * kD;
   const T* ks_base = k_seg + bkh * dm.S * kD;
   const T* vs_base = v_seg + bkh * dm.S * kD;
   const int32_t* gi = group_idx + (bkh * dm.nblk + n) * dm.kg;
@@ -447,15 +448,16 @@ cudaError_t bwd_dq(const void* q, const void* kh, const void* vh, const void* ks
 
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
-                                 int64_t H, int64_t S, int kg, int nsg, float scale, int* status, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, scale, status};
+                                 int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale, int* status,
+                                 cudaStream_t st) {
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale, status};
   return bf16 ? simt::fwd<__nv_bfloat16>(q, kh, vh, ks, vs, gi, o, lse, B, dm, st)
               : simt::fwd<float>(q, kh, vh, ks, vs, gi, o, lse, B, dm, st);
 }
 
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st) {
-  simt::Dims dm{Hq, 1, Hq, 0, (int)(S / kQBlock), 0, 0, S, 0.f, nullptr};
+  simt::Dims dm{Hq, 1, Hq, 0, (int)(S / kQBlock), 0, 0, S, 0, 0.f, nullptr};
   return bf16 ? simt::bwd_delta<__nv_bfloat16>(o, d_o, delta, B, dm, st)
               : simt::bwd_delta<float>(o, d_o, delta, B, dm, st);
 }
@@ -463,16 +465,16 @@ cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, flo
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
                                  const void* d_o, const float* delta, void* dk, void* dv, int B, int Hq, int Hkv,
                                  int64_t H, int64_t S, int kg, float scale, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), 0, H, S, scale, nullptr};
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), 0, H, S, H, scale, nullptr};
   return bf16 ? simt::bwd_dkdv<__nv_bfloat16>(q, ks, vs, lse, d_o, delta, dk, dv, B, dm, st)
               : simt::bwd_dkdv<float>(q, ks, vs, lse, d_o, delta, dk, dv, B, dm, st);
 }
 
 cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                const void* vs, const int32_t* gi, const float* lse, const void* d_o,
-                               const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
-                               int nsg, float scale, int* status, cudaStream_t st) {
-  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, scale, status};
+                               const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S,
+                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st) {
+  simt::Dims dm{Hq, Hkv, Hq / Hkv, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale, status};
   return bf16 ? simt::bwd_dq<__nv_bfloat16>(q, kh, vh, ks, vs, gi, lse, d_o, delta, dq, B, dm, st)
               : simt::bwd_dq<float>(q, kh, vh, ks, vs, gi, lse, d_o, delta, dq, B, dm, st);
 }

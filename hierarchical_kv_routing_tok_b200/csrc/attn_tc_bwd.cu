@@ -53,6 +53,7 @@ struct Params {
   int B, Hq, Hkv, G, kg, nblk;
   int nsg;        // sink groups at the start of every block's history key list
   int64_t H, S;
+  int64_t Hs;     // history rows per (batch, KV head) in k_hist / v_hist (>= H)
   float c2;       // scale * log2(e)
   float scale;
   const int32_t* group_idx;
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
           const int slot = j * 16 + lane;
           int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
           if (g < 0) g = 0;
-          const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
+          const int32_t row = (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup);
           tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
           tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
           tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(ks));
@@ -695,18 +696,22 @@ __global__ void __launch_bounds__(640, 1)
 // ------------------------------------------------------------------ host side
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, int nsg, float scale, int* status,
-                             cudaStream_t st) {
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale,
+                             int* status, cudaStream_t st) {
   namespace K = tcbwd::dq;
   CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
+  // with no history the history maps are never used: map the segment instead (maps need rows > 0)
+  const void* kh_m = Hs ? kh : ks;
+  const void* vh_m = Hs ? vh : vs;
+  const uint64_t hrows = (uint64_t)B * Hkv * (Hs ? Hs : S);
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mdo, d_o, (uint64_t)B * Hq * S, 64) ||
-      !make_map_bf16_rows(&mkh, kh, (uint64_t)B * Hkv * H, 8) ||
-      !make_map_bf16_rows(&mvh, vh, (uint64_t)B * Hkv * H, 8) ||
+      !make_map_bf16_rows(&mkh, kh_m, hrows, 8) ||
+      !make_map_bf16_rows(&mvh, vh_m, hrows, 8) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, K::BN) ||
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, scale * tcbwd::kLog2e, scale, gi, lse, delta,
+  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale * tcbwd::kLog2e, scale, gi, lse, delta,
               static_cast<__nv_bfloat16*>(dq), status};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / 2);
   const size_t smem = K::Smem::kBytes + 1024;

@@ -39,6 +39,7 @@ struct Params {
   int B, Hq, Hkv, G, hpc, kg, nblk;
   int nsg;        // sink groups at the start of every block's history key list
   int64_t H, S;
+  int64_t Hs;     // history rows per (batch, KV head) in k_hist / v_hist (>= H)
   float scale_log2;
   const int32_t* group_idx;
   __nv_bfloat16* o;
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
           const int slot = j * 16 + lane;
           int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
           if (g < 0) g = 0;
-          const int32_t row = (int32_t)((int64_t)bkh * p.H + (int64_t)g * kGroup);
+          const int32_t row = (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup);
           const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
           tma_load_2d(dst + lane * 2048, m, 0, row, full);
           tma_load_2d(dst + lane * 2048 + 1024, m, 64, row, full);
@@ -411,15 +412,19 @@ bool attn_fwd_tc_supported(int Hq, int Hkv) {
 
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int kg, int nsg, float scale, int* status, cudaStream_t st) {
+                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st) {
   CUtensorMap mq, mkh, mvh, mks, mvs;
-  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mkh, kh, (uint64_t)B * Hkv * H, 8) ||
-      !make_map_bf16_rows(&mvh, vh, (uint64_t)B * Hkv * H, 8) ||
+  // with no history the history maps are never used: map the segment instead (maps need rows > 0)
+  const void* kh_m = Hs ? kh : ks;
+  const void* vh_m = Hs ? vh : vs;
+  const uint64_t hrows = (uint64_t)B * Hkv * (Hs ? Hs : S);
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mkh, kh_m, hrows, 8) ||
+      !make_map_bf16_rows(&mvh, vh_m, hrows, 8) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, tcfwd::BN) ||
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, tcfwd::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), nsg, H, S,
+  tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), nsg, H, S, Hs,
                   scale * 1.4426950408889634f, gi, static_cast<__nv_bfloat16*>(o), lse, status};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
   cudaError_t e;

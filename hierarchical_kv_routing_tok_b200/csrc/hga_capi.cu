@@ -10,23 +10,24 @@
 #include "common.cuh"
 
 namespace hga {
-cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum,
-                             int64_t n_chunks_total, cudaStream_t stream);
+cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum, int64_t BHkv,
+                             int64_t Hs, int64_t c0, int64_t c1, cudaStream_t stream);
 cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
-                         int64_t S, int nch, int nsc, int kc, int kg, cudaStream_t stream);
+                         int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream);
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
-                                 int64_t H, int64_t S, int kg, int nsg, float scale, int* status, cudaStream_t st);
+                                 int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale, int* status,
+                                 cudaStream_t st);
 bool attn_fwd_tc_supported(int Hq, int Hkv);
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int kg, int nsg, float scale, int* status, cudaStream_t st);
+                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int kg, int nsg, float scale, int* status,
-                             cudaStream_t st);
+                             int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale,
+                             int* status, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
                                const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
                                int* status, cudaStream_t st);
@@ -37,8 +38,8 @@ cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const
                                  int64_t H, int64_t S, int kg, float scale, cudaStream_t st);
 cudaError_t launch_bwd_dq_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                const void* vs, const int32_t* gi, const float* lse, const void* d_o,
-                               const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int kg,
-                               int nsg, float scale, int* status, cudaStream_t st);
+                               const float* delta, void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S,
+                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st);
 size_t tier_plan_smem_bytes(int ngr);
 cudaError_t launch_tier_plan(const int32_t* group_idx, int BHkv, int nblk, int kg, int nsg, int ngr, int cap,
                              int32_t* used_groups, int32_t* n_used, int32_t* compact_idx, int* status,
@@ -61,22 +62,32 @@ int check_config(const hga_config_t* c) {
   if (c->dtype != HGA_F32 && c->dtype != HGA_BF16) return HGA_ERR_ARG;
   if (c->D != hga::kD || c->chunk != hga::kChunk || c->group != hga::kGroup || c->qblock != hga::kQBlock)
     return HGA_ERR_UNSUPPORTED;
-  if (c->hist_len < c->chunk || c->hist_len % c->chunk != 0) return HGA_ERR_ARG;
+  if (c->hist_len < 0 || c->hist_len % c->chunk != 0) return HGA_ERR_ARG;
+  if (c->hist_capacity != 0 && (c->hist_capacity < c->hist_len || c->hist_capacity % c->chunk != 0))
+    return HGA_ERR_ARG;
   if (c->seg_len < c->qblock || c->seg_len % c->qblock != 0) return HGA_ERR_ARG;
   const int64_t nch = c->hist_len / c->chunk;
   if (nch > kMaxChunks) return HGA_ERR_UNSUPPORTED;
-  // the sink window: whole chunks at the start of the history, at least one chunk left to route
-  if (c->n_sink_tokens < 0 || c->n_sink_tokens % c->chunk != 0 || c->n_sink_tokens >= c->hist_len)
-    return HGA_ERR_ARG;
-  const int64_t nsc = c->n_sink_tokens / c->chunk;
-  if (c->top_chunks < 1 || c->top_chunks > nch - nsc) return HGA_ERR_ARG;
-  if (c->top_groups < 1 || (int64_t)c->top_groups > (int64_t)c->top_chunks * (c->chunk / c->group))
-    return HGA_ERR_ARG;
+  if (nch == 0) {
+    // no history yet (the first segment of a sequence): local attention only, nothing to route
+    if (c->top_chunks != 0 || c->top_groups != 0 || c->n_sink_tokens != 0) return HGA_ERR_ARG;
+  } else {
+    // the sink window: whole chunks at the start of the history, at least one chunk left to route
+    if (c->n_sink_tokens < 0 || c->n_sink_tokens % c->chunk != 0 || c->n_sink_tokens >= c->hist_len)
+      return HGA_ERR_ARG;
+    const int64_t nsc = c->n_sink_tokens / c->chunk;
+    if (c->top_chunks < 1 || c->top_chunks > nch - nsc) return HGA_ERR_ARG;
+    if (c->top_groups < 1 || (int64_t)c->top_groups > (int64_t)c->top_chunks * (c->chunk / c->group))
+      return HGA_ERR_ARG;
+  }
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return HGA_ERR_ARG;
   // grid dimensions are 32-bit
   if ((int64_t)c->B * c->Hq * (c->seg_len / c->qblock) > INT32_MAX) return HGA_ERR_UNSUPPORTED;
   if ((int64_t)c->B * c->Hkv * nch > (int64_t)INT32_MAX) return HGA_ERR_UNSUPPORTED;   // one CTA per chunk
-  if (hga::route_smem_bytes(c->dtype == HGA_BF16, (int)nch, c->top_chunks, c->top_groups) > kMaxRouteSmem)
+  // history rows are addressed with 32-bit tensor-map coordinates
+  const int64_t hs = c->hist_capacity ? c->hist_capacity : c->hist_len;
+  if ((int64_t)c->B * c->Hkv * hs > (int64_t)INT32_MAX) return HGA_ERR_UNSUPPORTED;
+  if (nch && hga::route_smem_bytes(c->dtype == HGA_BF16, (int)nch, c->top_chunks, c->top_groups) > kMaxRouteSmem)
     return HGA_ERR_UNSUPPORTED;
   return HGA_OK;
 }
@@ -89,6 +100,9 @@ int check_ptrs(std::initializer_list<const void*> ps) {
   return HGA_OK;
 }
 
+// Rows per (batch, KV head) of the history and summary buffers (the history's capacity).
+int64_t hist_rows(const hga_config_t* c) { return c->hist_capacity ? c->hist_capacity : c->hist_len; }
+
 // Groups of the sink window, attended by every query ahead of the routed groups.
 int sink_groups(const hga_config_t* c) { return (int)(c->n_sink_tokens / c->group); }
 
@@ -99,6 +113,14 @@ int check_idx(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (reinterpret_cast<uintptr_t>(p) & 3u) return HGA_ERR_ALIGN;
   return HGA_OK;
+}
+
+// History K/V and routed group indices of the attention calls; with no history (hist_len == 0)
+// none of them is read and they may be NULL.
+int check_history(const hga_config_t* c, const void* k_hist, const void* v_hist, const int32_t* group_idx) {
+  if (c->hist_len == 0) return HGA_OK;
+  int rc = check_ptrs({k_hist, v_hist});
+  return rc ? rc : check_idx({group_idx});
 }
 
 float eff_scale(const hga_config_t* c) {
@@ -191,8 +213,8 @@ int hga_internal_attn_bwd_ws(const hga_config_t* cfg, const void* q, const void*
                              size_t ws_bytes, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
-  if ((rc = check_idx({group_idx}))) return rc;
+  if ((rc = check_ptrs({q, k_seg, v_seg, o, lse, d_o, dq, dk_seg, dv_seg}))) return rc;
+  if ((rc = check_history(cfg, k_hist, v_hist, group_idx))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
@@ -232,9 +254,21 @@ int hga_build_summaries(const hga_config_t* cfg, const void* k_hist, float* grou
   if (rc) return rc;
   if ((rc = check_ptrs({k_hist, group_sum, chunk_sum}))) return rc;
   (void)workspace;
-  const int64_t n_chunks = (int64_t)cfg->B * cfg->Hkv * (cfg->hist_len / cfg->chunk);
-  return from_cuda(hga::launch_summaries(cfg->dtype == HGA_BF16, k_hist, group_sum, chunk_sum, n_chunks,
+  return from_cuda(hga::launch_summaries(cfg->dtype == HGA_BF16, k_hist, group_sum, chunk_sum,
+                                         (int64_t)cfg->B * cfg->Hkv, hist_rows(cfg), 0, cfg->hist_len / cfg->chunk,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+int hga_append_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum, float* chunk_sum,
+                         int64_t first_token, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({k_hist, group_sum, chunk_sum}))) return rc;
+  if (first_token < 0 || first_token > cfg->hist_len || first_token % cfg->chunk != 0) return HGA_ERR_ARG;
+  (void)workspace;
+  return from_cuda(hga::launch_summaries(cfg->dtype == HGA_BF16, k_hist, group_sum, chunk_sum,
+                                         (int64_t)cfg->B * cfg->Hkv, hist_rows(cfg), first_token / cfg->chunk,
+                                         cfg->hist_len / cfg->chunk, static_cast<cudaStream_t>(stream)));
 }
 
 int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, const float* chunk_sum,
@@ -242,12 +276,14 @@ int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, co
   int rc = check_config(cfg);
   if (rc) return rc;
   if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
-  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   (void)workspace;
+  if (cfg->hist_len == 0) return HGA_OK;        // nothing to route
+  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, nullptr, false, group_sum, chunk_sum, chunk_idx,
                                      group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
-                                     (int)(cfg->hist_len / cfg->chunk), (int)(cfg->n_sink_tokens / cfg->chunk),
-                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
+                                     (int)(cfg->hist_len / cfg->chunk), (int)(hist_rows(cfg) / cfg->chunk),
+                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int hga_route_causal(const hga_config_t* cfg, const void* q, const void* q_prev, const float* group_sum,
@@ -255,32 +291,35 @@ int hga_route_causal(const hga_config_t* cfg, const void* q, const void* q_prev,
   int rc = check_config(cfg);
   if (rc) return rc;
   if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
-  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   if (q_prev && !aligned16(q_prev)) return HGA_ERR_ALIGN;
   (void)workspace;
+  if (cfg->hist_len == 0) return HGA_OK;        // nothing to route
+  if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, q_prev, true, group_sum, chunk_sum, chunk_idx,
                                      group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
-                                     (int)(cfg->hist_len / cfg->chunk), (int)(cfg->n_sink_tokens / cfg->chunk),
-                                     cfg->top_chunks, cfg->top_groups, static_cast<cudaStream_t>(stream)));
+                                     (int)(cfg->hist_len / cfg->chunk), (int)(hist_rows(cfg) / cfg->chunk),
+                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
                  const void* v_seg, const int32_t* group_idx, void* o, float* lse, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, o, lse}))) return rc;
-  if ((rc = check_idx({group_idx}))) return rc;
+  if ((rc = check_ptrs({q, k_seg, v_seg, o, lse}))) return rc;
+  if ((rc = check_history(cfg, k_hist, v_hist, group_idx))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   const bool bf16 = cfg->dtype == HGA_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (use_tc(cfg))
     return from_cuda(hga::launch_attn_fwd_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B, cfg->Hq,
-                                             cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups, sink_groups(cfg),
-                                             eff_scale(cfg), status_of(workspace), st));
-  return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
-                                             cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
+                                             cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg), cfg->top_groups,
                                              sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
+  return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
+                                             cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg),
+                                             cfg->top_groups, sink_groups(cfg), eff_scale(cfg), status_of(workspace),
+                                             st));
 }
 
 int hga_attn_bwd_preprocess(const hga_config_t* cfg, const void* o, const void* d_o, void* workspace,
@@ -306,19 +345,19 @@ int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, 
                     void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_hist, v_hist, k_seg, v_seg, lse, d_o, dq}))) return rc;
-  if ((rc = check_idx({group_idx}))) return rc;
+  if ((rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dq}))) return rc;
+  if ((rc = check_history(cfg, k_hist, v_hist, group_idx))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (use_tc(cfg))
     return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, delta_of(workspace),
-                                           dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, cfg->top_groups,
-                                           sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
+                                           dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg),
+                                           cfg->top_groups, sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
   return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
                                            d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
-                                           cfg->seg_len, cfg->top_groups, sink_groups(cfg), eff_scale(cfg),
-                                           status_of(workspace), st));
+                                           cfg->seg_len, hist_rows(cfg), cfg->top_groups, sink_groups(cfg),
+                                           eff_scale(cfg), status_of(workspace), st));
 }
 
 int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
@@ -336,6 +375,7 @@ int hga_tier_cache_config(const hga_config_t* cfg, hga_config_t* cache_cfg) {
   if (!cache_cfg) return HGA_ERR_ARG;
   *cache_cfg = *cfg;
   cache_cfg->hist_len = tier_cap_groups(cfg) * cfg->group;
+  cache_cfg->hist_capacity = 0;
   cache_cfg->top_chunks = (cfg->top_groups + (cfg->chunk / cfg->group) - 1) / (cfg->chunk / cfg->group);
   return check_config(cache_cfg);
 }
@@ -362,12 +402,12 @@ int hga_tier_gather(const hga_config_t* cfg, const void* k_hist, const void* v_h
   if ((rc = check_ptrs({k_hist, v_hist, k_cache, v_cache}))) return rc;
   if ((rc = check_idx({used_groups, n_used}))) return rc;
   const size_t esz = cfg->dtype == HGA_BF16 ? 2 : 4;
-  const size_t hist_bytes = (size_t)cfg->B * cfg->Hkv * cfg->hist_len * cfg->D * esz;
+  const size_t hist_bytes = (size_t)cfg->B * cfg->Hkv * hist_rows(cfg) * cfg->D * esz;
   const void* kh = device_view(k_hist, hist_bytes);
   const void* vh = device_view(v_hist, hist_bytes);
   if (!kh || !vh) return HGA_ERR_ARG;        // pageable host memory cannot be read by the device
   return from_cuda(hga::launch_tier_gather(cfg->dtype == HGA_BF16, kh, vh, used_groups, n_used, cfg->B * cfg->Hkv,
-                                           cfg->hist_len, (int)tier_cap_groups(cfg), k_cache, v_cache,
+                                           hist_rows(cfg), (int)tier_cap_groups(cfg), k_cache, v_cache,
                                            static_cast<cudaStream_t>(stream)));
 }
 

@@ -194,7 +194,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     const T* __restrict__ q, const T* __restrict__ q_prev, int causal, const float* __restrict__ group_sum,
     const float* __restrict__ chunk_sum, int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq,
-    int Hkv, int64_t S, int nch, int nsc, int kc, int kg) {
+    int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int N = Vec16<T>::N;
   constexpr int LPR = kD / N;
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
 
   // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
   // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
-  const float* cs = chunk_sum + (int64_t)bkh * nch * kD;
+  const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
   const int nc1 = nch - nsc;
   score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
   if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   }
 
   // ---- level 2: the 8 groups of every selected chunk
-  const float* gs = group_sum + (int64_t)bkh * nch * (kChunk / kGroup) * kD;
+  const float* gs = group_sum + (int64_t)bkh * nch_stride * (kChunk / kGroup) * kD;
   const int ncand = kc * (kChunk / kGroup);
   score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
   if (threadIdx.x < 4 && ncand + (int)threadIdx.x < ((ncand + 3) & ~3)) keys[ncand + threadIdx.x] = 0u;
@@ -312,7 +312,7 @@ size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
 
 cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
-                         int64_t S, int nch, int nsc, int kc, int kg, cudaStream_t stream) {
+                         int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream) {
   const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
   if (units == 0) return cudaSuccess;
   const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
@@ -322,13 +322,13 @@ cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool caus
     if (e != cudaSuccess) return e;
     route_kernel<__nv_bfloat16><<<(unsigned)units, kRouteThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(q_prev), causal ? 1 : 0, group_sum,
-        chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
+        chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
   } else {
     e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     route_kernel<float><<<(unsigned)units, kRouteThreads, smem, stream>>>(
         static_cast<const float*>(q), static_cast<const float*>(q_prev), causal ? 1 : 0, group_sum, chunk_sum,
-        chunk_idx, group_idx, Hq, Hkv, S, nch, nsc, kc, kg);
+        chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
   }
   return cudaGetLastError();
 }

@@ -14,22 +14,25 @@ namespace hga {
 // One CTA per 64-key chunk; warp w reduces group w (8 rows) with all of its 16-byte loads in flight
 // at once, writes the group mean, and the chunk mean is the mean of the eight group means (shared
 // memory).  Every byte of k_hist is read exactly once.
+// Chunks [c0, c0 + nc) of every (batch, KV head): history rows bkh * Hs + ..., summary rows
+// bkh * Hs / 8 + ... and bkh * Hs / 64 + ... (Hs = rows per (batch, KV head) of the buffers).
 template <typename T>
 __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k_hist,
                                                         float* __restrict__ group_sum,
-                                                        float* __restrict__ chunk_sum,
-                                                        int64_t n_chunks_total) {
+                                                        float* __restrict__ chunk_sum, int64_t Hs,
+                                                        int64_t c0, int64_t nc) {
   constexpr int N = Vec16<T>::N;              // elements per 16-byte load
   constexpr int LPR = kD / N;                 // lanes per row (16 bf16, 32 f32)
   constexpr int RPL = 32 / LPR;               // rows per warp-wide load (2 or 1)
   constexpr int LOADS = kGroup / RPL;         // loads per lane
   __shared__ float gmean[kChunk / kGroup][kD];
   const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
-  const int64_t chunk = blockIdx.x;
-  if (chunk >= n_chunks_total) return;
+  const int64_t bkh = blockIdx.x / nc;
+  const int64_t c = c0 + blockIdx.x % nc;
+  const int64_t chunk = bkh * (Hs / kChunk) + c;        // chunk row in the chunk-summary buffer
   const int col = (lane % LPR) * N;
   const int rsub = lane / LPR;
-  const T* base = k_hist + (chunk * kChunk + (int64_t)g * kGroup + rsub) * kD + col;
+  const T* base = k_hist + (bkh * Hs + c * kChunk + (int64_t)g * kGroup + rsub) * kD + col;
   float v[LOADS][N];
 #pragma unroll
   for (int i = 0; i < LOADS; ++i) Vec16<T>::load(base + (int64_t)i * RPL * kD, v[i]);
@@ -59,15 +62,17 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k_
   }
 }
 
-cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum,
-                             int64_t n_chunks_total, cudaStream_t stream) {
-  if (n_chunks_total == 0) return cudaSuccess;
+cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum, int64_t BHkv,
+                             int64_t Hs, int64_t c0, int64_t c1, cudaStream_t stream) {
+  const int64_t nc = c1 - c0;
+  if (BHkv == 0 || nc <= 0) return cudaSuccess;
+  const unsigned grid = (unsigned)(BHkv * nc);
   if (bf16)
-    summaries_kernel<__nv_bfloat16><<<(unsigned)n_chunks_total, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(k_hist), group_sum, chunk_sum, n_chunks_total);
+    summaries_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k_hist), group_sum,
+                                                              chunk_sum, Hs, c0, nc);
   else
-    summaries_kernel<float><<<(unsigned)n_chunks_total, 256, 0, stream>>>(
-        static_cast<const float*>(k_hist), group_sum, chunk_sum, n_chunks_total);
+    summaries_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(k_hist), group_sum, chunk_sum, Hs,
+                                                      c0, nc);
   return cudaGetLastError();
 }
 

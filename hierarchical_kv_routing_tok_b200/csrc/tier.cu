@@ -130,7 +130,7 @@ cudaError_t launch_tier_plan(const int32_t* group_idx, int BHkv, int nblk, int k
 template <int NV>     // 16-byte vectors per lane per tensor (8 rows x row_bytes / 16 / 32)
 __global__ void __launch_bounds__(256) tier_gather_kernel(const uint4* __restrict__ kh, const uint4* __restrict__ vh,
                                                           const int32_t* __restrict__ used_groups,
-                                                          const int32_t* __restrict__ n_used, int64_t H, int cap,
+                                                          const int32_t* __restrict__ n_used, int64_t Hs, int cap,
                                                           uint4* __restrict__ kc, uint4* __restrict__ vc) {
   const int lane = threadIdx.x & 31;
   const int64_t bkh = blockIdx.x;
@@ -138,8 +138,8 @@ __global__ void __launch_bounds__(256) tier_gather_kernel(const uint4* __restric
   if (slot >= cap || slot >= n_used[bkh]) return;
   const int64_t g = used_groups[bkh * cap + slot];
   constexpr int kVecPerGroup = 32 * NV;
-  const uint4* ks = kh + (bkh * H + g * kGroup) * (kVecPerGroup / kGroup);
-  const uint4* vs = vh + (bkh * H + g * kGroup) * (kVecPerGroup / kGroup);
+  const uint4* ks = kh + (bkh * Hs + g * kGroup) * (kVecPerGroup / kGroup);
+  const uint4* vs = vh + (bkh * Hs + g * kGroup) * (kVecPerGroup / kGroup);
   uint4* kd = kc + (bkh * cap + slot) * (int64_t)kVecPerGroup;
   uint4* vd = vc + (bkh * cap + slot) * (int64_t)kVecPerGroup;
   uint4 a[NV], b[NV];
@@ -156,17 +156,17 @@ __global__ void __launch_bounds__(256) tier_gather_kernel(const uint4* __restric
 }
 
 cudaError_t launch_tier_gather(bool bf16, const void* kh, const void* vh, const int32_t* used_groups,
-                               const int32_t* n_used, int BHkv, int64_t H, int cap, void* kc, void* vc,
+                               const int32_t* n_used, int BHkv, int64_t Hs, int cap, void* kc, void* vc,
                                cudaStream_t st) {
   if (BHkv == 0 || cap == 0) return cudaSuccess;
   const dim3 grid((unsigned)BHkv, (unsigned)((cap + 7) / 8));
   const auto* k4 = static_cast<const uint4*>(kh);
   const auto* v4 = static_cast<const uint4*>(vh);
   if (bf16)   // 8 rows x 256 bytes = 128 vectors per group: 4 per lane
-    tier_gather_kernel<4><<<grid, 256, 0, st>>>(k4, v4, used_groups, n_used, H, cap, static_cast<uint4*>(kc),
+    tier_gather_kernel<4><<<grid, 256, 0, st>>>(k4, v4, used_groups, n_used, Hs, cap, static_cast<uint4*>(kc),
                                                 static_cast<uint4*>(vc));
   else        // 8 rows x 512 bytes: 8 per lane
-    tier_gather_kernel<8><<<grid, 256, 0, st>>>(k4, v4, used_groups, n_used, H, cap, static_cast<uint4*>(kc),
+    tier_gather_kernel<8><<<grid, 256, 0, st>>>(k4, v4, used_groups, n_used, Hs, cap, static_cast<uint4*>(kc),
                                                 static_cast<uint4*>(vc));
   return cudaGetLastError();
 }

@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define HGA_VERSION 1
+#define HGA_VERSION 2
 
 /* Symbols of the shared library (built with hidden default visibility). */
 #if defined(__GNUC__)
@@ -87,8 +87,17 @@ enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 };
 
 /* Problem description.  chunk = 64, group = 8, qblock = 64 and D = 128 are
  * the only built values (pith.science free-parameter ledger: chunk 64,
- * group 8).  hist_len must be a positive multiple of chunk (only closed
- * chunks exist), seg_len a positive multiple of qblock.
+ * group 8).  hist_len must be a multiple of chunk (only closed chunks exist),
+ * seg_len a positive multiple of qblock.  hist_len = 0 (the first segment of a
+ * sequence, no history yet) requires top_chunks = top_groups = n_sink_tokens
+ * = 0: routing does nothing and attention covers the causal segment prefix
+ * only; k_hist, v_hist and group_idx are then not read and may be NULL.
+ * hist_capacity: rows per (batch, KV head) of the history buffers k_hist /
+ * v_hist [B, Hkv, hist_capacity, D] and of the summary buffers [B, Hkv,
+ * hist_capacity / group, D] and [B, Hkv, hist_capacity / chunk, D], of which
+ * the first hist_len tokens are the history (0 = hist_len; otherwise a
+ * multiple of chunk, >= hist_len): a history that grows segment by segment
+ * lives in one allocation.
  * n_sink_tokens: 0 <= n_sink_tokens < hist_len, a multiple of chunk; the
  * first n_sink_tokens history tokens are attended by every query and their
  * chunks are not routable, so 1 <= top_chunks <= (hist_len - n_sink_tokens) /
@@ -103,6 +112,7 @@ typedef struct hga_config {
   int32_t n_sink_tokens;
   int32_t dtype;
   float softmax_scale;
+  int64_t hist_capacity;
 } hga_config_t;
 
 /* Bytes of workspace the calls below need for this configuration. */
@@ -116,6 +126,15 @@ HGA_API int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out);
  *   chunk_sum  [B, Hkv, H/64, D]     float32           (out) */
 HGA_API int hga_build_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum,
                         float* chunk_sum, void* workspace, void* stream);
+
+/* As hga_build_summaries for the chunks of history tokens [first_token,
+ * hist_len) only (first_token a multiple of chunk): at a segment boundary the
+ * closed segment's keys are appended to the history and only their summaries
+ * are computed; every summary depends on its own keys only, so the result
+ * equals a full rebuild bit for bit. */
+HGA_API int hga_append_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum,
+                                 float* chunk_sum, int64_t first_token, void* workspace,
+                                 void* stream);
 
 /* Two-level routing (Technical Summary 2.1): for each (b, kv head kh, block
  * n) the block query qb = mean of q over the block's 64 positions and the
