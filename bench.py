@@ -59,7 +59,6 @@ def work_model(w) -> dict:
         "route": ("hbm", B * Hq * S * D * esz + B * Hkv * (nch + ngr) * D * 4
                   + B * Hkv * nblk * (w.top_chunks + w.top_groups) * 4),
         "attn_fwd": ("tensor", 4 * D * (routed_pairs + local_pairs)),
-        "bwd_preprocess": ("hbm", 2 * B * Hq * S * D * esz + B * Hq * S * 4),
         "bwd_dkdv": ("tensor", 8 * D * local_pairs),
         "bwd_dq": ("tensor", 6 * D * (routed_pairs + local_pairs)),
     }

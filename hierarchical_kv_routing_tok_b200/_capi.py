@@ -75,7 +75,7 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_preprocess": [C, P, P, P, P],
         "hga_attn_bwd_dkdv": [C, P, P, P, P, P, P, P, P, P],
-        "hga_attn_bwd_dq": [C, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_attn_bwd_dq": [C, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_noalloc": [C, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_tier_cache_config": [C, C],
         "hga_tier_plan": [C, P, P, P, P, P, P],
@@ -157,8 +157,9 @@ def attn_bwd_dkdv(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, str
     _call("hga_attn_bwd_dkdv", ctypes.byref(cfg), q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, stream)
 
 
-def attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream=0) -> None:
-    _call("hga_attn_bwd_dq", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq,
+def attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, workspace, stream=0) -> None:
+    """dq; also leaves delta = rowsum(d_o * o) in the workspace for attn_bwd_dkdv."""
+    _call("hga_attn_bwd_dq", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq,
           workspace, stream)
 
 

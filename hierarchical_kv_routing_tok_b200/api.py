@@ -222,11 +222,11 @@ class LayerStep:
              if self.causal_routing else (lambda: C.route(cfg, p["q"], gs, cs, ci, gi, ws, st))),
             ("attn_fwd", lambda: C.attn_fwd(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi, o,
                                             lse, ws, st)),
-            ("bwd_preprocess", lambda: C.attn_bwd_preprocess(cfg, o, p["d_o"], ws, st)),
+            # dq first: it also forms delta = rowsum(d_o * o), which dkdv reads
+            ("bwd_dq", lambda: C.attn_bwd_dq(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi,
+                                             o, lse, p["d_o"], dq, ws, st)),
             ("bwd_dkdv", lambda: C.attn_bwd_dkdv(cfg, p["q"], p["k_seg"], p["v_seg"], lse, p["d_o"], dk, dv, ws,
                                                  st)),
-            ("bwd_dq", lambda: C.attn_bwd_dq(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi,
-                                             lse, p["d_o"], dq, ws, st)),
         ]
 
     def forward(self, x: dict) -> None:

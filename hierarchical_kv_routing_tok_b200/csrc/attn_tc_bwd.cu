@@ -58,7 +58,8 @@ struct Params {
   float scale;
   const int32_t* group_idx;
   const float* lse;
-  const float* delta;
+  const __nv_bfloat16* o;   // forward output: delta = rowsum(dO o O) is formed here
+  float* delta;             // delta of this kernel's rows, written for the dK/dV kernel
   __nv_bfloat16* dq;
   int* status;
 };
@@ -281,11 +282,53 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     const int64_t t_pos = (int64_t)n * kQBlock + (r & 63);
     const int64_t row = ((int64_t)b * p.Hq + head) * p.S + t_pos;
     const float lse2 = p.lse[row] * kLog2e;
-    const float dl = p.delta[row];
+    // delta = sum_d dO o O of this row (FlashAttention-form backward).  Warpgroup w takes columns
+    // 32w .. 32w+31: O from global memory (loads issued before the wait for the Q/dO tile), dO from
+    // the 128B-swizzled tile the producer loaded for dP (row r: 8-row atom r/8, 16-byte chunk c of
+    // a 64-column half at position c ^ (r mod 8)).  The four partial sums meet in TMEM columns
+    // 384..387 (the dQ accumulator, not yet written) and every thread adds them in order; the
+    // first warpgroup stores delta for the dK/dV kernel.
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int c0 = 32 * w;
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
+    uint4 ov[4];
+    {
+      const uint4* orow = reinterpret_cast<const uint4*>(p.o + row * kD + c0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ov[c] = orow[c];
+    }
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qdo_full, 0, abort_flag, p.status));
+    float part = 0.f;
+    if (ok) {
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int chunk = 4 * w + c;                         // 16-byte chunk of the 128-column row
+        const uint32_t off = (uint32_t)(chunk >> 3) * kQHalf + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
+                             ((uint32_t)((chunk & 7) ^ (r & 7)) << 4);
+        const uint4 dv4 = *reinterpret_cast<const uint4*>(smem + L::kDO + off);
+        const uint32_t a[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w}, d4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc0 = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(d4[e] << 16), acc0);
+          acc1 = fmaf(__uint_as_float(a[e] & 0xffff0000u), __uint_as_float(d4[e] & 0xffff0000u), acc1);
+        }
+      }
+      part = acc0 + acc1;
+    }
+    tmem_st1(tmem + lane_off + 384 + w, __float_as_uint(part));
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar_sync(1, 32 * kEWWarps);                        // all element-wise warps, every path
+    tc_fence_after();
+    float dl;
+    {
+      uint32_t pv[4];
+      tmem_ld4(tmem + lane_off + 384, pv);
+      tmem_wait_ld();
+      dl = ((__uint_as_float(pv[0]) + __uint_as_float(pv[1])) + __uint_as_float(pv[2])) + __uint_as_float(pv[3]);
+    }
+    if (ok && w == 0) p.delta[row] = dl;
+    for (int j = 0; ok && j < T; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(sd_full, j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
@@ -695,9 +738,9 @@ __global__ void __launch_bounds__(640, 1)
 
 // ------------------------------------------------------------------ host side
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
-                             const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale,
-                             int* status, cudaStream_t st) {
+                             const int32_t* gi, const float* lse, const void* o, const void* d_o, float* delta,
+                             void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg,
+                             float scale, int* status, cudaStream_t st) {
   namespace K = tcbwd::dq;
   CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
   // with no history the history maps are never used: map the segment instead (maps need rows > 0)
@@ -711,8 +754,8 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale * tcbwd::kLog2e, scale, gi, lse, delta,
-              static_cast<__nv_bfloat16*>(dq), status};
+  K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale * tcbwd::kLog2e, scale, gi, lse,
+              static_cast<const __nv_bfloat16*>(o), delta, static_cast<__nv_bfloat16*>(dq), status};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / 2);
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -25,9 +25,9 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
                                int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
-                             const int32_t* gi, const float* lse, const void* d_o, const float* delta, void* dq,
-                             int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale,
-                             int* status, cudaStream_t st);
+                             const int32_t* gi, const float* lse, const void* o, const void* d_o, float* delta,
+                             void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg,
+                             float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
                                const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
                                int* status, cudaStream_t st);
@@ -217,9 +217,10 @@ int hga_internal_attn_bwd_ws(const hga_config_t* cfg, const void* q, const void*
   if ((rc = check_history(cfg, k_hist, v_hist, group_idx))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
-  if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
-  if ((rc = bwd_dkdv_ws(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, ws_bytes, stream))) return rc;
-  return hga_attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, dq, workspace, stream);
+  // dQ first: it also forms delta = rowsum(dO o O) into the workspace, which dK/dV then reads
+  if ((rc = hga_attn_bwd_dq(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o, dq, workspace, stream)))
+    return rc;
+  return bwd_dkdv_ws(cfg, q, k_seg, v_seg, lse, d_o, dk_seg, dv_seg, workspace, ws_bytes, stream);
 }
 
 extern "C" {
@@ -341,19 +342,21 @@ int hga_attn_bwd_dkdv(const hga_config_t* cfg, const void* q, const void* k_seg,
 }
 
 int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, const void* v_hist, const void* k_seg,
-                    const void* v_seg, const int32_t* group_idx, const float* lse, const void* d_o, void* dq,
-                    void* workspace, void* stream) {
+                    const void* v_seg, const int32_t* group_idx, const void* o, const float* lse, const void* d_o,
+                    void* dq, void* workspace, void* stream) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if ((rc = check_ptrs({q, k_seg, v_seg, lse, d_o, dq}))) return rc;
+  if ((rc = check_ptrs({q, k_seg, v_seg, o, lse, d_o, dq}))) return rc;
   if ((rc = check_history(cfg, k_hist, v_hist, group_idx))) return rc;
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (use_tc(cfg))
-    return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, d_o, delta_of(workspace),
-                                           dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg),
-                                           cfg->top_groups, sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
+  if (use_tc(cfg))   // the tensor-core kernel forms delta of its own rows as it starts
+    return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, o, d_o,
+                                           delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
+                                           cfg->seg_len, hist_rows(cfg), cfg->top_groups, sink_groups(cfg),
+                                           eff_scale(cfg), status_of(workspace), st));
+  if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
   return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
                                            d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
                                            cfg->seg_len, hist_rows(cfg), cfg->top_groups, sink_groups(cfg),

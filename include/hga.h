@@ -188,12 +188,15 @@ HGA_API int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_h
                  const void* d_o, void* dq, void* dk_seg, void* dv_seg, void* workspace,
                  void* stream);
 
-/* The three steps of hga_attn_bwd as separate calls, in this order, on one
- * stream and one workspace (the same computation; each launches one kernel):
+/* The steps of hga_attn_bwd as separate calls, on one stream and one workspace
+ * (the same computation):
  *   preprocess: delta[b,h,t] = sum_d d_o * o  -> workspace scratch
  *               (the FlashAttention-form backward the pages cite);
- *   dkdv:       dk_seg, dv_seg from the local causal pairs (needs delta);
- *   dq:         dq over routed and local keys (needs delta).
+ *   dq:         dq over routed and local keys; it also forms delta itself and
+ *               leaves it in the workspace (so dq then dkdv needs no
+ *               preprocess -- that is the order hga_attn_bwd uses);
+ *   dkdv:       dk_seg, dv_seg from the local causal pairs (needs delta: from
+ *               preprocess or from an earlier dq on the same workspace).
  * Arguments as for hga_attn_bwd. */
 HGA_API int hga_attn_bwd_preprocess(const hga_config_t* cfg, const void* o, const void* d_o,
                                     void* workspace, void* stream);
@@ -202,8 +205,8 @@ HGA_API int hga_attn_bwd_dkdv(const hga_config_t* cfg, const void* q, const void
                               void* dk_seg, void* dv_seg, void* workspace, void* stream);
 HGA_API int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist,
                             const void* v_hist, const void* k_seg, const void* v_seg,
-                            const int32_t* group_idx, const float* lse, const void* d_o,
-                            void* dq, void* workspace, void* stream);
+                            const int32_t* group_idx, const void* o, const float* lse,
+                            const void* d_o, void* dq, void* workspace, void* stream);
 
 /* Backward without any allocation: the same computation and kernels as
  * hga_attn_bwd, for callers that cannot allocate device memory -- e.g. a host
