@@ -70,20 +70,45 @@ struct Smem {
   static constexpr uint32_t kK = kDO + kQTile;
   static constexpr uint32_t kV = kK + KS * kKVTile;
   static constexpr uint32_t kBar = kV + VS * kKVTile;
-  // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], sd_full, dp_free, ds_full, final, mma_done
-  static constexpr int kNumBars = 1 + 2 * KS + VS + 5;
+  // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], sd_full, dp_free, ds_full, dq_ready, mma_done,
+  // qdo_empty, delta_bar
+  static constexpr int kNumBars = 1 + 2 * KS + VS + 7;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
 static_assert(Smem::kBytes + 1024 <= 227 * 1024, "dq shared memory exceeds the per-CTA limit");
 
-// One CTA per (batch, KV head, query block, pair of query heads): a single M=128 tile whose rows
-// 0-63 are the block's queries of head h0 and rows 64-127 those of head h0+1.  Key tiles of 128:
-// the routed groups of the block (16 groups per tile) then the causal segment prefix.
-// TMEM: S in two buffers (columns 0 and 128), dP (256), dQ (384).  Per tile j the MMA thread
-// issues dP(j+1) and S(j+1) as soon as the element-wise warps have loaded S(j), dP(j) into
-// registers, and dQ(j) += dS(j) K(j) when they have written dS(j) (bf16, packed into S(j)'s
-// columns).
+// Work unit u (heavy first): (batch, KV head, query block, pair of query heads), unit 0 being the
+// last query block.  A persistent CTA c of G takes the units c, 2G-1-c, 2G+c, 4G-1-c, ... (a snake
+// over the list, which spreads the long units evenly).
+struct Unit {
+  int b, bkh, n, h0, T;
+};
+__device__ __forceinline__ int unit_of_cta(int k, int c, int G) {
+  const int round = k >> 1;
+  return (k & 1) ? (2 * round + 2) * G - 1 - c : 2 * round * G + c;
+}
+__device__ __forceinline__ Unit decode_unit(int u, const Params& p, int n_rt) {
+  const int hp = p.G / 2;
+  Unit x;
+  const int hpi = u % hp;
+  u /= hp;
+  x.bkh = u % (p.B * p.Hkv);
+  x.n = p.nblk - 1 - u / (p.B * p.Hkv);
+  x.b = x.bkh / p.Hkv;
+  x.h0 = (x.bkh % p.Hkv) * p.G + 2 * hpi;
+  x.T = n_rt + ((x.n + 1) * kQBlock + BN - 1) / BN;              // history tiles + causal-prefix tiles
+  return x;
+}
+
+// Persistent: one CTA per SM walks its units; per unit a single M=128 tile whose rows 0-63 are the
+// block's queries of head h0 and rows 64-127 those of head h0+1, over key tiles of 128 (the sink
+// and routed groups of the block, 16 groups per tile, then the causal segment prefix).
+// TMEM: S in two buffers (columns 0 and 128), dP (256), dQ (384).  Per tile j the MMA warp issues
+// dP(j+1) and S(j+1) as soon as the element-wise warps have loaded S(j), dP(j) into registers, and
+// dQ(j) += dS(j) K(j) when they have written dS(j) (bf16, packed into S(j)'s columns).  A running
+// tile count J carries the K/V ring and the per-tile barrier phases across units; the next unit's
+// Q/dO are loaded (warp 2) as soon as the last S, dP MMAs of the current unit have read them.
 __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
@@ -96,31 +121,24 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   const uint32_t bar0 = sbase + L::kBar;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const uint32_t qdo_full = BAR(0);
-  auto kv_full = [&](int s) { return BAR(1 + s); };          // K(j) and V(j) of tile j, slot j mod KS
+  auto kv_full = [&](int s) { return BAR(1 + s); };          // K(J) and V(J) of tile J, slot J mod KS
   auto k_empty = [&](int s) { return BAR(1 + KS + s); };
   auto v_empty = [&](int s) { return BAR(1 + 2 * KS + s); };
   const uint32_t sd_full = BAR(1 + 2 * KS + VS);
   const uint32_t dp_free = BAR(2 + 2 * KS + VS);
   const uint32_t ds_full = BAR(3 + 2 * KS + VS);
-  const uint32_t final_bar = BAR(4 + 2 * KS + VS);
+  const uint32_t dq_ready = BAR(4 + 2 * KS + VS);
   const uint32_t mma_done = BAR(5 + 2 * KS + VS);
+  const uint32_t qdo_empty = BAR(6 + 2 * KS + VS);          // the unit's Q/dO fully read
+  const uint32_t delta_bar = BAR(7 + 2 * KS + VS);          // delta partial sums in TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- unit decode: query block (heavy = late first), batch x KV head, head pair
-  const int hp = p.G / 2;
-  int c = blockIdx.x;
-  const int hpi = c % hp;
-  c /= hp;
-  const int bkh = c % (p.B * p.Hkv);
-  const int n = p.nblk - 1 - c / (p.B * p.Hkv);
-  const int b = bkh / p.Hkv, kh = bkh % p.Hkv;
-  const int h0 = kh * p.G + 2 * hpi;
   const int n_hist = 8 * (p.nsg + p.kg);                         // sink + routed history keys
   const int n_rt = (n_hist + BN - 1) / BN;                        // history tiles
-  const int T = n_rt + ((n + 1) * kQBlock + BN - 1) / BN;        // + causal-prefix tiles
-  const int32_t* gi = p.group_idx + ((int64_t)bkh * p.nblk + n) * p.kg;
+  const int n_units = p.B * p.Hkv * p.nblk * (p.G / 2);
+  const int G = gridDim.x, cta = blockIdx.x;
   const int64_t ngr = p.H / kGroup;
 
   if (threadIdx.x == 0) {
@@ -133,8 +151,10 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     mbar_init(sd_full, 1);
     mbar_init(dp_free, kEWWarps);
     mbar_init(ds_full, kEWWarps);
-    mbar_init(final_bar, 1);
+    mbar_init(dq_ready, 1);
     mbar_init(mma_done, 1);
+    mbar_init(qdo_empty, 1 + kEWWarps);     // the MMA warp's commit + every element-wise warp
+    mbar_init(delta_bar, kEWWarps);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -148,230 +168,288 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ======================= TMA producer: Q, dO once; then K(j), V(j) per tile into their rings
-    if (lane == 0) {
-      mbar_arrive_expect_tx(qdo_full, 2 * kQTile);
-      for (int jh = 0; jh < 2; ++jh) {
-        const int64_t row = ((int64_t)b * p.Hq + h0 + jh) * p.S + (int64_t)n * kQBlock;
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t off = h * kQHalf + jh * (kQHalf / 2);
-          tma_load_2d(sbase + L::kQ + off, &tm_q, 64 * h, (int32_t)row, qdo_full);
-          tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
-        }
-      }
-    }
+    // ======================= TMA producer of K(J), V(J) into their rings, across all units
     int issued[KS] = {0, 0, 0};
-    for (int j = 0; j < T; ++j) {
-      const int ks = j % KS, vs = j % VS;
-      int ok = 1;
-      if (lane == 0) {
-        ok = mbar_wait(k_empty(ks), ((j / KS) & 1) ^ 1, abort_flag, p.status) &&
-             mbar_wait(v_empty(vs), ((j / VS) & 1) ^ 1, abort_flag, p.status);
-        if (ok) mbar_arrive_expect_tx(kv_full(ks), 2 * kKVTile);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      const uint32_t kd = sbase + L::kK + ks * kKVTile, vd = sbase + L::kV + vs * kKVTile;
-      if (j < n_rt) {
-        // 16 routed groups, one per lane: two 8-row x 64-column boxes each of K and V
-        if (lane < 16) {
-          const int slot = j * 16 + lane;
-          int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
-          if (g < 0) g = 0;
-          const int32_t row = (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup);
-          tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
-          tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
-          tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(ks));
-          tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(ks));
+    int J = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of_cta(k, cta, G);
+      if (u >= n_units) break;
+      const Unit x = decode_unit(u, p, n_rt);
+      const int32_t* gi = p.group_idx + ((int64_t)x.bkh * p.nblk + x.n) * p.kg;
+      for (int j = 0; j < x.T; ++j, ++J) {
+        const int ks = J % KS, vs = J % VS;
+        int okk = 1;
+        if (lane == 0) {
+          okk = mbar_wait(k_empty(ks), ((J / KS) & 1) ^ 1, abort_flag, p.status) &&
+                mbar_wait(v_empty(vs), ((J / VS) & 1) ^ 1, abort_flag, p.status);
+          if (okk) mbar_arrive_expect_tx(kv_full(ks), 2 * kKVTile);
         }
-      } else if (lane == 0) {
-        const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)(j - n_rt) * BN);
-        tma_load_2d(kd, &tm_ks, 0, row, kv_full(ks));
-        tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(ks));
-        tma_load_2d(vd, &tm_vs, 0, row, kv_full(ks));
-        tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(ks));
+        ok = __shfl_sync(0xffffffffu, okk, 0) != 0;
+        if (!ok) break;
+        const uint32_t kd = sbase + L::kK + ks * kKVTile, vd = sbase + L::kV + vs * kKVTile;
+        if (j < n_rt) {
+          // 16 routed groups, one per lane: two 8-row x 64-column boxes each of K and V
+          if (lane < 16) {
+            const int slot = j * 16 + lane;
+            int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
+            if (g < 0) g = 0;
+            const int32_t row = (int32_t)((int64_t)x.bkh * p.Hs + (int64_t)g * kGroup);
+            tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
+            tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
+            tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(ks));
+            tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(ks));
+          }
+        } else if (lane == 0) {
+          const int32_t row = (int32_t)((int64_t)x.bkh * p.S + (int64_t)(j - n_rt) * BN);
+          tma_load_2d(kd, &tm_ks, 0, row, kv_full(ks));
+          tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(ks));
+          tma_load_2d(vd, &tm_vs, 0, row, kv_full(ks));
+          tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(ks));
+        }
+        __syncwarp();
+        ++issued[ks];
       }
-      __syncwarp();
-      ++issued[ks];
     }
-    if (lane == 0) {
-      drain_wait(qdo_full, 0, p.status);
+    if (lane == 0)
       for (int s = 0; s < KS; ++s)
         if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
+    __syncwarp();
+  } else if (warp == 2) {
+    // ======================= TMA producer of each unit's Q and dO (once the previous unit's
+    // last S, dP MMAs and delta reads are done with them)
+    int loads = 0;
+    if (lane == 0) {
+      for (int k = 0;; ++k) {
+        const int u = unit_of_cta(k, cta, G);
+        if (u >= n_units) break;
+        if (k > 0 && !mbar_wait(qdo_empty, (k - 1) & 1, abort_flag, p.status)) break;
+        const Unit x = decode_unit(u, p, n_rt);
+        mbar_arrive_expect_tx(qdo_full, 2 * kQTile);
+        for (int jh = 0; jh < 2; ++jh) {
+          const int64_t row = ((int64_t)x.b * p.Hq + x.h0 + jh) * p.S + (int64_t)x.n * kQBlock;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t off = h * kQHalf + jh * (kQHalf / 2);
+            tma_load_2d(sbase + L::kQ + off, &tm_q, 64 * h, (int32_t)row, qdo_full);
+            tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
+          }
+        }
+        ++loads;
+      }
+      if (loads) drain_wait(qdo_full, (loads - 1) & 1, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer: the whole warp runs the loop (warp-uniform descriptors
-    // and waits) and one elected lane issues each tcgen05 instruction.  Q and dO are fixed for
-    // the CTA, so their descriptor arrays are built once; K / V stage descriptors come from
-    // prebuilt bases.
-    {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
-      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
-      uint64_t qa[8], da[8];
-      kmajor_descs(qa, sbase + L::kQ, kQHalf, 1024);
-      kmajor_descs(da, sbase + L::kDO, kQHalf, 1024);
-      // routed tiles: group g at g * 2048 bytes, 64-column halves 1024 apart; local tiles: halves
-      // kKVHalf apart, 8-row groups 1024 apart.  Stage st is st * kKVTile bytes after stage 0.
-      const uint64_t k_rt = smem_desc_sw128(sbase + L::kK, 16, 2048), k_lc = smem_desc_sw128(sbase + L::kK, 16, 1024);
-      const uint64_t v_rt = smem_desc_sw128(sbase + L::kV, 16, 2048), v_lc = smem_desc_sw128(sbase + L::kV, 16, 1024);
-      const uint64_t kmn_rt = smem_desc_sw128(sbase + L::kK, 1024, 2048);
-      const uint64_t kmn_lc = smem_desc_sw128(sbase + L::kK, kKVHalf, 1024);
-      auto issue_s = [&](int j) {   // S(j) = Q K(j)^T into S buffer j mod 2
-        const bool rt = j < n_rt;
-        const uint64_t soff = (uint64_t)((j % KS) * (kKVTile >> 4));
-        uint64_t bb[8];
-        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + (j & 1) * 128, qa[ks], bb[ks], idesc_s, ks > 0);
-      };
-      auto issue_dp = [&](int j) {  // dP(j) = dO V(j)^T
-        const bool rt = j < n_rt;
-        const uint64_t soff = (uint64_t)((j % VS) * (kKVTile >> 4));
+    // and waits) and one elected lane issues each tcgen05 instruction.  Q and dO sit at fixed
+    // addresses, so their descriptor arrays are built once; K / V stage descriptors come from
+    // prebuilt bases.  Global tile J: K stage J mod KS, V stage J mod VS, S buffer J mod 2.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, kD, true);
+    uint64_t qa[8], da[8];
+    kmajor_descs(qa, sbase + L::kQ, kQHalf, 1024);
+    kmajor_descs(da, sbase + L::kDO, kQHalf, 1024);
+    // routed tiles: group g at g * 2048 bytes, 64-column halves 1024 apart; local tiles: halves
+    // kKVHalf apart, 8-row groups 1024 apart.  Stage st is st * kKVTile bytes after stage 0.
+    const uint64_t k_rt = smem_desc_sw128(sbase + L::kK, 16, 2048), k_lc = smem_desc_sw128(sbase + L::kK, 16, 1024);
+    const uint64_t v_rt = smem_desc_sw128(sbase + L::kV, 16, 2048), v_lc = smem_desc_sw128(sbase + L::kV, 16, 1024);
+    const uint64_t kmn_rt = smem_desc_sw128(sbase + L::kK, 1024, 2048);
+    const uint64_t kmn_lc = smem_desc_sw128(sbase + L::kK, kKVHalf, 1024);
+    // S(J) = Q K(J)^T into S buffer J mod 2 and dP(J) = dO V(J)^T; `rt`: a routed-history tile
+    auto issue_sdp = [&](int J, bool rt) {
+      tc_fence_after();
+      {
+        const uint64_t soff = (uint64_t)((J % VS) * (kKVTile >> 4));
         uint64_t bb[8];
         kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + 256, da[ks], bb[ks], idesc_s, ks > 0);
-      };
-      auto issue_dq = [&](int j) {  // dQ += dS(j) K(j); dS of keys 32w..32w+31 sits in columns 32w..32w+15
-        const bool rt = j < n_rt;
-        const uint64_t soff = (uint64_t)((j % KS) * (kKVTile >> 4));
-        uint64_t bb[8];
-        mnmajor_from_base<8>(bb, (rt ? kmn_rt : kmn_lc) + soff, rt ? (2 * 2048u) >> 4 : (2 * 1024u) >> 4);
-        const uint32_t sb = tmem + (j & 1) * 128;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ts_w(tmem + 384, sb + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq, (j > 0 || ks > 0));
-      };
-      // Per tile j: once the element-wise warps hold S(j), dP(j) in registers, dP(j+1) and S(j+1)
-      // (the other S buffer, whose dS(j-1) dQ(j-1) has already read); once they have written
-      // dS(j), dQ(j) += dS(j) K(j).
-      auto issue_sdp = [&](int j) {   // K(j), V(j) have landed
-        tc_fence_after();
-        issue_dp(j);
-        issue_s(j);
-        mma_commit_w(sd_full);
-        mma_commit_w(v_empty(j % VS));
-      };
-      bool ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status);
-      if (ok) issue_sdp(0);
-      for (int j = 0; ok && j < T; ++j) {
-        // the next tile's K/V usually landed long ago: check that before the wait on the
-        // element-wise warps, so nothing but that wait sits between it and the next MMAs
-        if (j + 1 < T) ok = mbar_wait_w(kv_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
-        if (ok) ok = mbar_wait_w(dp_free, j & 1, abort_flag, p.status);
-        if (!ok) break;
-        if (j + 1 < T) issue_sdp(j + 1);
-        ok = mbar_wait_w(ds_full, j & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dq(j);
-        mma_commit_w(k_empty(j % KS));
       }
-      if (ok) mma_commit_w(final_bar);
-      mma_commit_w(mma_done);
-      drain_wait(mma_done, 0, p.status);
+      {
+        const uint64_t soff = (uint64_t)((J % KS) * (kKVTile >> 4));
+        uint64_t bb[8];
+        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + (J & 1) * 128, qa[ks], bb[ks], idesc_s, ks > 0);
+      }
+      mma_commit_w(sd_full);
+      mma_commit_w(v_empty(J % VS));
+    };
+    // dQ (+)= dS(J) K(J); dS of keys 32w..32w+31 sits in columns 32w..32w+15 of S buffer J mod 2
+    auto issue_dq = [&](int J, bool rt, bool first) {
+      const uint64_t soff = (uint64_t)((J % KS) * (kKVTile >> 4));
+      uint64_t bb[8];
+      mnmajor_from_base<8>(bb, (rt ? kmn_rt : kmn_lc) + soff, rt ? (2 * 2048u) >> 4 : (2 * 1024u) >> 4);
+      const uint32_t sb = tmem + (J & 1) * 128;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts_w(tmem + 384, sb + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq, !(first && ks == 0));
+    };
+    // Per tile: once the element-wise warps hold S, dP in registers, the next tile's dP and S (the
+    // next tile may be the next unit's first, once its Q/dO have landed); once they have written
+    // dS, dQ += dS K.  The unit's Q/dO are released after its last S/dP MMAs, dQ after its last
+    // dS K MMAs.
+    bool ok = true;
+    int J = 0;
+    Unit x{};
+    int u = unit_of_cta(0, cta, G);
+    if (u < n_units) {
+      x = decode_unit(u, p, n_rt);
+      ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status);
+      if (ok) {
+        issue_sdp(0, 0 < n_rt);
+        if (x.T == 1) mma_commit_w(qdo_empty);
+      }
     }
+    for (int k = 0; ok && u < n_units; ++k) {
+      const int un = unit_of_cta(k + 1, cta, G);
+      const bool has_next = un < n_units;
+      const Unit xn = has_next ? decode_unit(un, p, n_rt) : x;
+      for (int j = 0; j < x.T; ++j, ++J) {
+        // the next tile's K/V usually landed long ago: check that (and, across units, the next
+        // unit's Q/dO) before the wait on the element-wise warps
+        const bool last = j + 1 == x.T;
+        const bool next = !last || has_next;
+        if (last && has_next) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status);
+        if (ok && next) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status);
+        if (ok) ok = mbar_wait_w(dp_free, J & 1, abort_flag, p.status);
+        if (!ok) break;
+        if (next) {
+          const int jn = last ? 0 : j + 1;
+          const int Tn = last ? xn.T : x.T;
+          issue_sdp(J + 1, jn < n_rt);
+          if (jn + 1 == Tn) mma_commit_w(qdo_empty);
+        }
+        ok = mbar_wait_w(ds_full, J & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dq(J, j < n_rt, j == 0);
+        mma_commit_w(k_empty(J % KS));
+      }
+      if (!ok) break;
+      mma_commit_w(dq_ready);
+      u = un;
+      x = xn;
+    }
+    mma_commit_w(mma_done);
+    drain_wait(mma_done, 0, p.status);
   } else if (warp >= 4) {
     // ======================= element-wise: dS = P o (dP - delta), P = exp2(S c2 - lse log2 e).
     // Thread = TMEM lane = row of the M tile; warpgroup w owns key columns 32w .. 32w+31.
     const int w = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int head = h0 + (r >> 6);
-    const int64_t t_pos = (int64_t)n * kQBlock + (r & 63);
-    const int64_t row = ((int64_t)b * p.Hq + head) * p.S + t_pos;
-    const float lse2 = p.lse[row] * kLog2e;
-    // delta = sum_d dO o O of this row (FlashAttention-form backward).  Warpgroup w takes columns
-    // 32w .. 32w+31: O from global memory (loads issued before the wait for the Q/dO tile), dO from
-    // the 128B-swizzled tile the producer loaded for dP (row r: 8-row atom r/8, 16-byte chunk c of
-    // a 64-column half at position c ^ (r mod 8)).  The four partial sums meet in TMEM columns
-    // 384..387 (the dQ accumulator, not yet written) and every thread adds them in order; the
-    // first warpgroup stores delta for the dK/dV kernel.
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int c0 = 32 * w;
-    uint4 ov[4];
-    {
-      const uint4* orow = reinterpret_cast<const uint4*>(p.o + row * kD + c0);
+    bool ok = true;
+    int J = 0;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of_cta(k, cta, G);
+      if (u >= n_units) break;
+      const Unit x = decode_unit(u, p, n_rt);
+      const int head = x.h0 + (r >> 6);
+      const int64_t t_pos = (int64_t)x.n * kQBlock + (r & 63);
+      const int64_t row = ((int64_t)x.b * p.Hq + head) * p.S + t_pos;
+      const float lse2 = p.lse[row] * kLog2e;
+      // delta = sum_d dO o O of this row (FlashAttention-form backward).  Warpgroup w takes columns
+      // 32w .. 32w+31: O from global memory (loads issued before the wait for the Q/dO tile), dO
+      // from the 128B-swizzled tile loaded for dP (row r: 8-row atom r/8, 16-byte chunk c of a
+      // 64-column half at position c ^ (r mod 8)).  The four partial sums meet in TMEM column
+      // 384 + 32w (the first column of this warpgroup's dQ, already read out for the previous
+      // unit and not rewritten before this unit's first dS K MMA) and every thread adds them in
+      // order; the first warpgroup stores delta for the dK/dV kernel.
+      uint4 ov[4];
+      {
+        const uint4* orow = reinterpret_cast<const uint4*>(p.o + row * kD + c0);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) ov[c] = orow[c];
-    }
-    bool ok = __all_sync(0xffffffffu, mbar_wait(qdo_full, 0, abort_flag, p.status));
-    float part = 0.f;
-    if (ok) {
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int chunk = 4 * w + c;                         // 16-byte chunk of the 128-column row
-        const uint32_t off = (uint32_t)(chunk >> 3) * kQHalf + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
-                             ((uint32_t)((chunk & 7) ^ (r & 7)) << 4);
-        const uint4 dv4 = *reinterpret_cast<const uint4*>(smem + L::kDO + off);
-        const uint32_t a[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w}, d4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc0 = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(d4[e] << 16), acc0);
-          acc1 = fmaf(__uint_as_float(a[e] & 0xffff0000u), __uint_as_float(d4[e] & 0xffff0000u), acc1);
-        }
+        for (int c = 0; c < 4; ++c) ov[c] = orow[c];
       }
-      part = acc0 + acc1;
-    }
-    tmem_st1(tmem + lane_off + 384 + w, __float_as_uint(part));
-    tmem_wait_st();
-    tc_fence_before();
-    named_bar_sync(1, 32 * kEWWarps);                        // all element-wise warps, every path
-    tc_fence_after();
-    float dl;
-    {
-      uint32_t pv[4];
-      tmem_ld4(tmem + lane_off + 384, pv);
-      tmem_wait_ld();
-      dl = ((__uint_as_float(pv[0]) + __uint_as_float(pv[1])) + __uint_as_float(pv[2])) + __uint_as_float(pv[3]);
-    }
-    if (ok && w == 0) p.delta[row] = dl;
-    for (int j = 0; ok && j < T; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(sd_full, j & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(qdo_full, k & 1, abort_flag, p.status));
       if (!ok) break;
-      tc_fence_after();
-      const uint32_t tS = tmem + lane_off + (j & 1) * 128 + c0;
-      // one TMEM round trip: both loads in flight, one wait; then dP is free for dP(j+1)
-      uint32_t sv[32], dv[32], pk[16];
-      tmem_ld32(tS, sv);
-      tmem_ld32(tmem + lane_off + 256 + c0, dv);
-      tmem_wait_ld();
-      tc_fence_before();
+      float part;
+      {
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * w + c;                       // 16-byte chunk of the 128-column row
+          const uint32_t off = (uint32_t)(chunk >> 3) * kQHalf + (uint32_t)(r >> 3) * 1024u +
+                               (uint32_t)(r & 7) * 128u + ((uint32_t)((chunk & 7) ^ (r & 7)) << 4);
+          const uint4 dv4 = *reinterpret_cast<const uint4*>(smem + L::kDO + off);
+          const uint32_t a[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w}, d4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc0 = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(d4[e] << 16), acc0);
+            acc1 = fmaf(__uint_as_float(a[e] & 0xffff0000u), __uint_as_float(d4[e] & 0xffff0000u), acc1);
+          }
+        }
+        part = acc0 + acc1;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(dp_free);
-      int nvalid;   // valid key columns of this tile for this row
-      if (j < n_rt) {
-        nvalid = min(BN, n_hist - j * BN);
-      } else {
-        const int64_t u0 = (int64_t)(j - n_rt) * BN;
-        nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
-      }
-      if (nvalid >= c0 + 32) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2));
-          const float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2));
-          pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = (c0 + e < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
-          const float p1 = (c0 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
-          pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
-        }
-      }
-      // packed bf16 dS stays inside this warpgroup's own (already read) column range
-      tmem_st16(tS, pk);
+      if (lane == 0) mbar_arrive(qdo_empty);                 // this warp is done with dO
+      tmem_st1(tmem + lane_off + 384 + c0, __float_as_uint(part));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(final_bar, 0, abort_flag, p.status));
-    if (ok) {
+      if (lane == 0) mbar_arrive(delta_bar);
+      ok = __all_sync(0xffffffffu, mbar_wait(delta_bar, k & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      float dl;
+      {
+        uint32_t pv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
+                       : "=r"(pv[i])
+                       : "r"(tmem + lane_off + 384 + 32 * i));
+        tmem_wait_ld();
+        dl = ((__uint_as_float(pv[0]) + __uint_as_float(pv[1])) + __uint_as_float(pv[2])) + __uint_as_float(pv[3]);
+      }
+      if (w == 0) p.delta[row] = dl;
+      for (int j = 0; j < x.T; ++j, ++J) {
+        ok = __all_sync(0xffffffffu, mbar_wait(sd_full, J & 1, abort_flag, p.status));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_off + (J & 1) * 128 + c0;
+        // one TMEM round trip: both loads in flight, one wait; then dP is free for the next dP
+        uint32_t sv[32], dv[32], pk[16];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tmem + lane_off + 256 + c0, dv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dp_free);
+        int nvalid;   // valid key columns of this tile for this row
+        if (j < n_rt) {
+          nvalid = min(BN, n_hist - j * BN);
+        } else {
+          const int64_t u0 = (int64_t)(j - n_rt) * BN;
+          nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
+        }
+        if (nvalid >= c0 + 32) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2));
+            const float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2));
+            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = (c0 + e < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
+            const float p1 = (c0 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
+            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
+          }
+        }
+        // packed bf16 dS stays inside this warpgroup's own (already read) column range
+        tmem_st16(tS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
+      }
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_ready, k & 1, abort_flag, p.status));
+      if (!ok) break;
       tc_fence_after();
       uint32_t v[32], pk[16];
       tmem_ld32(tmem + lane_off + 384 + c0, v);
@@ -382,6 +460,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       uint4* d4 = reinterpret_cast<uint4*>(p.dq + row * kD + c0);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      tc_fence_before();
     }
   }
   tc_fence_before();
@@ -756,7 +835,12 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
   const int G = Hq / Hkv;
   K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale * tcbwd::kLog2e, scale, gi, lse,
               static_cast<const __nv_bfloat16*>(o), delta, static_cast<__nv_bfloat16*>(dq), status};
-  const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / 2);
+  // persistent: one CTA per SM (or per unit, when there are fewer units than SMs)
+  const int64_t units = (int64_t)B * Hkv * p.nblk * (G / 2);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int64_t grid = units < sms ? units : sms;
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
