@@ -30,6 +30,7 @@
 namespace hga {
 
 bool make_map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows);
+bool make_map_bf16_groups(CUtensorMap* m, const void* base, uint64_t rows);
 
 namespace tcbwd {
 
@@ -48,6 +49,7 @@ constexpr uint32_t kKVHalf = BN * 128;      // 16 KB (local layout)
 constexpr int KS = 3;                       // K stages (a K tile lives until its dQ MMAs are done)
 constexpr int VS = 2;                       // V stages (a V tile lives until its dP MMAs are done)
 constexpr int kEWWarps = 16;                // four element-wise warpgroups
+constexpr int kIdxRegs = 8;                 // history slots per producer lane read ahead (256 a unit)
 
 struct Params {
   int B, Hq, Hkv, G, kg, nblk;
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
     for (int s = 0; s < KS; ++s) {
-      mbar_init(kv_full(s), 1);
+      mbar_init(kv_full(s), 2);             // the K and the V producer
       mbar_init(k_empty(s), 1);
     }
     for (int s = 0; s < VS; ++s) mbar_init(v_empty(s), 1);
@@ -167,50 +169,76 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ======================= TMA producer of K(J), V(J) into their rings, across all units
+  if (warp == 0 || warp == 3) {
+    // ======================= TMA producers of K(J) (warp 0) and V(J) (warp 3), each into its own
+    // ring, across all units; both arrive on kv_full of the tile.  A routed history group (8 rows)
+    // is one 3-D box: its two 64-column halves land 1 KB apart in the group layout.  A unit's
+    // group indices are read one unit ahead, all in one round trip (lane l holds slots l, l + 32,
+    // ...), so the index reads never stand between a free slot and its loads.
+    const bool is_v = warp == 3;
+    const CUtensorMap* hist_map = is_v ? &tm_vh : &tm_kh;
+    const CUtensorMap* seg_map = is_v ? &tm_vs : &tm_ks;
     int issued[KS] = {0, 0, 0};
     int J = 0;
     bool ok = true;
+    int32_t cur[kIdxRegs], nxt[kIdxRegs];
+    auto read_idx = [&](int k, int32_t(&r)[kIdxRegs]) {
+      const int u = unit_of_cta(k, cta, G);
+      if (u >= n_units) return;
+      const Unit x = decode_unit(u, p, n_rt);
+      const int32_t* gi = p.group_idx + ((int64_t)x.bkh * p.nblk + x.n) * p.kg;
+#pragma unroll
+      for (int i = 0; i < kIdxRegs; ++i) {
+        const int slot = 32 * i + lane;
+        r[i] = slot < 16 * n_rt ? routed_group(gi, slot, p.nsg, p.kg, ngr, p.status) : 0;
+      }
+    };
+    read_idx(0, nxt);
     for (int k = 0; ok; ++k) {
       const int u = unit_of_cta(k, cta, G);
       if (u >= n_units) break;
       const Unit x = decode_unit(u, p, n_rt);
       const int32_t* gi = p.group_idx + ((int64_t)x.bkh * p.nblk + x.n) * p.kg;
+#pragma unroll
+      for (int i = 0; i < kIdxRegs; ++i) cur[i] = nxt[i];
+      read_idx(k + 1, nxt);
       for (int j = 0; j < x.T; ++j, ++J) {
         const int ks = J % KS, vs = J % VS;
         int okk = 1;
         if (lane == 0) {
-          okk = mbar_wait(k_empty(ks), ((J / KS) & 1) ^ 1, abort_flag, p.status) &&
-                mbar_wait(v_empty(vs), ((J / VS) & 1) ^ 1, abort_flag, p.status);
-          if (okk) mbar_arrive_expect_tx(kv_full(ks), 2 * kKVTile);
+          okk = is_v ? mbar_wait(v_empty(vs), ((J / VS) & 1) ^ 1, abort_flag, p.status)
+                     : mbar_wait(k_empty(ks), ((J / KS) & 1) ^ 1, abort_flag, p.status);
+          if (okk) mbar_arrive_expect_tx(kv_full(ks), kKVTile);
         }
         ok = __shfl_sync(0xffffffffu, okk, 0) != 0;
         if (!ok) break;
-        const uint32_t kd = sbase + L::kK + ks * kKVTile, vd = sbase + L::kV + vs * kKVTile;
+        const uint32_t dst = is_v ? sbase + L::kV + vs * kKVTile : sbase + L::kK + ks * kKVTile;
         if (j < n_rt) {
-          // 16 routed groups, one per lane: two 8-row x 64-column boxes each of K and V
-          if (lane < 16) {
-            const int slot = j * 16 + lane;
-            int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
-            if (g < 0) g = 0;
-            const int32_t row = (int32_t)((int64_t)x.bkh * p.Hs + (int64_t)g * kGroup);
-            tma_load_2d(kd + lane * 2048, &tm_kh, 0, row, kv_full(ks));
-            tma_load_2d(kd + lane * 2048 + 1024, &tm_kh, 64, row, kv_full(ks));
-            tma_load_2d(vd + lane * 2048, &tm_vh, 0, row, kv_full(ks));
-            tma_load_2d(vd + lane * 2048 + 1024, &tm_vh, 64, row, kv_full(ks));
+          // 16 routed groups, one per lane
+          int32_t g;
+          if (j < 2 * kIdxRegs) {
+            int32_t sel = 0;
+#pragma unroll
+            for (int i = 0; i < kIdxRegs; ++i)
+              if (i == (j >> 1)) sel = cur[i];
+            g = __shfl_sync(0xffffffffu, sel, (16 * j + lane) & 31);
+          } else {
+            g = lane < 16 ? routed_group(gi, j * 16 + lane, p.nsg, p.kg, ngr, p.status) : 0;
           }
+          if (g < 0) g = 0;
+          if (lane < 16)
+            tma_load_3d(dst + lane * 2048, hist_map, 0, (int32_t)((int64_t)x.bkh * p.Hs + (int64_t)g * kGroup), 0,
+                        kv_full(ks));
         } else if (lane == 0) {
           const int32_t row = (int32_t)((int64_t)x.bkh * p.S + (int64_t)(j - n_rt) * BN);
-          tma_load_2d(kd, &tm_ks, 0, row, kv_full(ks));
-          tma_load_2d(kd + kKVHalf, &tm_ks, 64, row, kv_full(ks));
-          tma_load_2d(vd, &tm_vs, 0, row, kv_full(ks));
-          tma_load_2d(vd + kKVHalf, &tm_vs, 64, row, kv_full(ks));
+          tma_load_2d(dst, seg_map, 0, row, kv_full(ks));
+          tma_load_2d(dst + kKVHalf, seg_map, 64, row, kv_full(ks));
         }
         __syncwarp();
         ++issued[ks];
       }
     }
+    // every load this warp issued has landed (its tile's barrier completed) before the CTA exits
     if (lane == 0)
       for (int s = 0; s < KS; ++s)
         if (issued[s]) drain_wait(kv_full(s), (issued[s] - 1) & 1, p.status);
@@ -827,8 +855,7 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
   const void* vh_m = Hs ? vh : vs;
   const uint64_t hrows = (uint64_t)B * Hkv * (Hs ? Hs : S);
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mdo, d_o, (uint64_t)B * Hq * S, 64) ||
-      !make_map_bf16_rows(&mkh, kh_m, hrows, 8) ||
-      !make_map_bf16_rows(&mvh, vh_m, hrows, 8) ||
+      !make_map_bf16_groups(&mkh, kh_m, hrows) || !make_map_bf16_groups(&mvh, vh_m, hrows) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, K::BN) ||
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BN))
     return cudaErrorInvalidValue;

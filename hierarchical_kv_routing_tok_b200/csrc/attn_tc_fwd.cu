@@ -47,6 +47,7 @@ struct Params {
   int* status;
 };
 
+constexpr int kIdxRegs = 8;                // history slots per producer lane read up front (256)
 constexpr int KS = 3;                      // K stages (K runs ahead of V)
 constexpr int VS = 2;                      // V stages
 
@@ -155,6 +156,14 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       tma_prefetch_desc(&tm_vh);
       tma_prefetch_desc(&tm_vs);
     }
+    // the block's history group indices, all read in one round trip before the first load (lane
+    // l holds slots l, l + 32, ...; longer lists read the rest per tile)
+    int32_t gidx[kIdxRegs];
+#pragma unroll
+    for (int i = 0; i < kIdxRegs; ++i) {
+      const int slot = 32 * i + lane;
+      gidx[i] = slot < 16 * n_rt ? routed_group(gi, slot, p.nsg, p.kg, ngr, p.status) : 0;
+    }
     int issued[KS] = {0, 0, 0};
     for (int j = 0; j < T; ++j) {
       const int s = j % NS;
@@ -169,15 +178,22 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       if (j < n_rt) {
-        if (lane < 16) {
-          const int slot = j * 16 + lane;
-          int32_t g = routed_group(gi, slot, p.nsg, p.kg, ngr, p.status);
-          if (g < 0) g = 0;
-          const int32_t row = (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup);
-          const CUtensorMap* m = kv ? &tm_vh : &tm_kh;
-          tma_load_2d(dst + lane * 2048, m, 0, row, full);
-          tma_load_2d(dst + lane * 2048 + 1024, m, 64, row, full);
+        // 16 routed groups, one per lane, each group's 8 rows one 3-D box (its two 64-column halves
+        // land 1 KB apart)
+        int32_t g;
+        if (j < 2 * kIdxRegs) {
+          int32_t sel = 0;
+#pragma unroll
+          for (int i = 0; i < kIdxRegs; ++i)
+            if (i == (j >> 1)) sel = gidx[i];
+          g = __shfl_sync(0xffffffffu, sel, (16 * j + lane) & 31);
+        } else {
+          g = lane < 16 ? routed_group(gi, j * 16 + lane, p.nsg, p.kg, ngr, p.status) : 0;
         }
+        if (g < 0) g = 0;
+        if (lane < 16)
+          tma_load_3d(dst + lane * 2048, kv ? &tm_vh : &tm_kh, 0, (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup),
+                      0, full);
       } else if (lane == 0) {
         const int jl = j - n_rt;
         const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)jl * BN);
@@ -376,6 +392,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
 }  // namespace tcfwd
 
 // ------------------------------------------------------------------ host side
+bool make_map_bf16_groups(CUtensorMap* m, const void* base, uint64_t rows);
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -405,6 +422,21 @@ bool make_map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 map over a [rows, 128] row-major tensor seen as {64 dims, rows, 2 halves} (the halves 128
+// bytes apart in global memory): a box {64, 8, 2} is one 8-row group, landing in shared memory as
+// two 1 KB 128B-swizzled atoms, first the dims 0-63 of its 8 rows, then the dims 64-127.
+bool make_map_bf16_groups(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, 2};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)kGroup, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool attn_fwd_tc_supported(int Hq, int Hkv) {
   const int G = Hq / Hkv;
   return G % 2 == 0;
@@ -418,8 +450,8 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
   const void* kh_m = Hs ? kh : ks;
   const void* vh_m = Hs ? vh : vs;
   const uint64_t hrows = (uint64_t)B * Hkv * (Hs ? Hs : S);
-  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mkh, kh_m, hrows, 8) ||
-      !make_map_bf16_rows(&mvh, vh_m, hrows, 8) ||
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_groups(&mkh, kh_m, hrows) ||
+      !make_map_bf16_groups(&mvh, vh_m, hrows) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, tcfwd::BN) ||
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, tcfwd::BN))
     return cudaErrorInvalidValue;
