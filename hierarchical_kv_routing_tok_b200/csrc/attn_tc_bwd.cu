@@ -72,9 +72,9 @@ struct Smem {
   static constexpr uint32_t kK = kDO + kQTile;
   static constexpr uint32_t kV = kK + KS * kKVTile;
   static constexpr uint32_t kBar = kV + VS * kKVTile;
-  // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], sd_full, dp_free, ds_full, dq_ready, mma_done,
-  // qdo_empty, delta_bar
-  static constexpr int kNumBars = 1 + 2 * KS + VS + 7;
+  // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], s_full[2], dp_full, dp_free, ds_full[2],
+  // dq_ready, mma_done, qdo_empty, delta_bar
+  static constexpr int kNumBars = 1 + 2 * KS + VS + 11;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
@@ -126,13 +126,16 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   auto kv_full = [&](int s) { return BAR(1 + s); };          // K(J) and V(J) of tile J, slot J mod KS
   auto k_empty = [&](int s) { return BAR(1 + KS + s); };
   auto v_empty = [&](int s) { return BAR(1 + 2 * KS + s); };
-  const uint32_t sd_full = BAR(1 + 2 * KS + VS);
-  const uint32_t dp_free = BAR(2 + 2 * KS + VS);
-  const uint32_t ds_full = BAR(3 + 2 * KS + VS);
-  const uint32_t dq_ready = BAR(4 + 2 * KS + VS);
-  const uint32_t mma_done = BAR(5 + 2 * KS + VS);
-  const uint32_t qdo_empty = BAR(6 + 2 * KS + VS);          // the unit's Q/dO fully read
-  const uint32_t delta_bar = BAR(7 + 2 * KS + VS);          // delta partial sums in TMEM
+  // S, dS of tile J live in S buffer J mod 2: their barriers are per buffer (phase J / 2), so that
+  // S(J+1), issued before the element-wise warps are done with tile J, never runs a phase ahead
+  auto s_full = [&](int b) { return BAR(1 + 2 * KS + VS + b); };
+  const uint32_t dp_full = BAR(3 + 2 * KS + VS);
+  const uint32_t dp_free = BAR(4 + 2 * KS + VS);
+  auto ds_full = [&](int b) { return BAR(5 + 2 * KS + VS + b); };
+  const uint32_t dq_ready = BAR(7 + 2 * KS + VS);
+  const uint32_t mma_done = BAR(8 + 2 * KS + VS);
+  const uint32_t qdo_empty = BAR(9 + 2 * KS + VS);          // the unit's Q/dO fully read
+  const uint32_t delta_bar = BAR(10 + 2 * KS + VS);         // delta partial sums in TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,9 +153,12 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       mbar_init(k_empty(s), 1);
     }
     for (int s = 0; s < VS; ++s) mbar_init(v_empty(s), 1);
-    mbar_init(sd_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(ds_full(b), kEWWarps);
+    }
+    mbar_init(dp_full, 1);
     mbar_init(dp_free, kEWWarps);
-    mbar_init(ds_full, kEWWarps);
     mbar_init(dq_ready, 1);
     mbar_init(mma_done, 1);
     mbar_init(qdo_empty, 1 + kEWWarps);     // the MMA warp's commit + every element-wise warp
@@ -283,24 +289,24 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     const uint64_t v_rt = smem_desc_sw128(sbase + L::kV, 16, 2048), v_lc = smem_desc_sw128(sbase + L::kV, 16, 1024);
     const uint64_t kmn_rt = smem_desc_sw128(sbase + L::kK, 1024, 2048);
     const uint64_t kmn_lc = smem_desc_sw128(sbase + L::kK, kKVHalf, 1024);
-    // S(J) = Q K(J)^T into S buffer J mod 2 and dP(J) = dO V(J)^T; `rt`: a routed-history tile
-    auto issue_sdp = [&](int J, bool rt) {
+    // S(J) = Q K(J)^T into S buffer J mod 2; dP(J) = dO V(J)^T; `rt`: a routed-history tile
+    auto issue_s = [&](int J, bool rt) {
       tc_fence_after();
-      {
-        const uint64_t soff = (uint64_t)((J % VS) * (kKVTile >> 4));
-        uint64_t bb[8];
-        kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
+      const uint64_t soff = (uint64_t)((J % KS) * (kKVTile >> 4));
+      uint64_t bb[8];
+      kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + 256, da[ks], bb[ks], idesc_s, ks > 0);
-      }
-      {
-        const uint64_t soff = (uint64_t)((J % KS) * (kKVTile >> 4));
-        uint64_t bb[8];
-        kmajor_from_base(bb, (rt ? k_rt : k_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
+      for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + (J & 1) * 128, qa[ks], bb[ks], idesc_s, ks > 0);
+      mma_commit_w(s_full(J & 1));
+    };
+    auto issue_dp = [&](int J, bool rt) {
+      tc_fence_after();
+      const uint64_t soff = (uint64_t)((J % VS) * (kKVTile >> 4));
+      uint64_t bb[8];
+      kmajor_from_base(bb, (rt ? v_rt : v_lc) + soff, rt ? (1024u >> 4) : (kKVHalf >> 4));
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + (J & 1) * 128, qa[ks], bb[ks], idesc_s, ks > 0);
-      }
-      mma_commit_w(sd_full);
+      for (int ks = 0; ks < 8; ++ks) mma_ss_w(tmem + 256, da[ks], bb[ks], idesc_s, ks > 0);
+      mma_commit_w(dp_full);
       mma_commit_w(v_empty(J % VS));
     };
     // dQ (+)= dS(J) K(J); dS of keys 32w..32w+31 sits in columns 32w..32w+15 of S buffer J mod 2
@@ -313,10 +319,11 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       for (int ks = 0; ks < 8; ++ks)
         mma_ts_w(tmem + 384, sb + (ks >> 1) * 32 + (ks & 1) * 8, bb[ks], idesc_dq, !(first && ks == 0));
     };
-    // Per tile: once the element-wise warps hold S, dP in registers, the next tile's dP and S (the
-    // next tile may be the next unit's first, once its Q/dO have landed); once they have written
-    // dS, dQ += dS K.  The unit's Q/dO are released after its last S/dP MMAs, dQ after its last
-    // dS K MMAs.
+    // Per tile J: S(J+1) as soon as its K tile has landed (the other S buffer, whose dS(J-1) the
+    // last dQ MMA has read); dP(J+1) once the element-wise warps hold dP(J); dQ += dS(J) K(J) once
+    // they have written dS(J).  The next tile may be the next unit's first, once its Q/dO have
+    // landed.  The unit's Q/dO are released after its last dP MMAs (issued after its last S MMAs),
+    // dQ after its last dS K MMAs.
     bool ok = true;
     int J = 0;
     Unit x{};
@@ -325,7 +332,8 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       x = decode_unit(u, p, n_rt);
       ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status);
       if (ok) {
-        issue_sdp(0, 0 < n_rt);
+        issue_s(0, 0 < n_rt);
+        issue_dp(0, 0 < n_rt);
         if (x.T == 1) mma_commit_w(qdo_empty);
       }
     }
@@ -334,21 +342,23 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       const bool has_next = un < n_units;
       const Unit xn = has_next ? decode_unit(un, p, n_rt) : x;
       for (int j = 0; j < x.T; ++j, ++J) {
-        // the next tile's K/V usually landed long ago: check that (and, across units, the next
-        // unit's Q/dO) before the wait on the element-wise warps
         const bool last = j + 1 == x.T;
         const bool next = !last || has_next;
-        if (last && has_next) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status);
-        if (ok && next) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status);
-        if (ok) ok = mbar_wait_w(dp_free, J & 1, abort_flag, p.status);
+        const int jn = last ? 0 : j + 1;          // the next tile's index in its unit
+        const int Tn = last ? xn.T : x.T;
+        if (next) {
+          if (last) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status);
+          if (ok) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status);
+          if (!ok) break;
+          issue_s(J + 1, jn < n_rt);
+        }
+        ok = mbar_wait_w(dp_free, J & 1, abort_flag, p.status);
         if (!ok) break;
         if (next) {
-          const int jn = last ? 0 : j + 1;
-          const int Tn = last ? xn.T : x.T;
-          issue_sdp(J + 1, jn < n_rt);
+          issue_dp(J + 1, jn < n_rt);
           if (jn + 1 == Tn) mma_commit_w(qdo_empty);
         }
-        ok = mbar_wait_w(ds_full, J & 1, abort_flag, p.status);
+        ok = mbar_wait_w(ds_full(J & 1), (J >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         issue_dq(J, j < n_rt, j == 0);
@@ -435,18 +445,12 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       }
       if (w == 0) p.delta[row] = dl;
       for (int j = 0; j < x.T; ++j, ++J) {
-        ok = __all_sync(0xffffffffu, mbar_wait(sd_full, J & 1, abort_flag, p.status));
+        // P of this warpgroup's 32 keys from S (masked keys -> 0) while dP is still in the tensor
+        // pipe; then dP, which frees the dP columns for the next tile's dP
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(J & 1), (J >> 1) & 1, abort_flag, p.status));
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + (J & 1) * 128 + c0;
-        // one TMEM round trip: both loads in flight, one wait; then dP is free for the next dP
-        uint32_t sv[32], dv[32], pk[16];
-        tmem_ld32(tS, sv);
-        tmem_ld32(tmem + lane_off + 256 + c0, dv);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dp_free);
         int nvalid;   // valid key columns of this tile for this row
         if (j < n_rt) {
           nvalid = min(BN, n_hist - j * BN);
@@ -454,27 +458,38 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
           const int64_t u0 = (int64_t)(j - n_rt) * BN;
           nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
         }
-        if (nvalid >= c0 + 32) {
+        float pr[32];
+        {
+          uint32_t sv[32];
+          tmem_ld32(tS, sv);
+          tmem_wait_ld();
+          auto pexp = [&](int e) { return ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)); };
+          if (nvalid >= c0 + 32) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2));
-            const float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2));
-            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
-          }
-        } else {
+            for (int e = 0; e < 32; ++e) pr[e] = pexp(e);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = (c0 + e < nvalid) ? ex2(fmaf(__uint_as_float(sv[e]), p.c2, -lse2)) : 0.f;
-            const float p1 = (c0 + e + 1 < nvalid) ? ex2(fmaf(__uint_as_float(sv[e + 1]), p.c2, -lse2)) : 0.f;
-            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dv[e]) - dl), p1 * (__uint_as_float(dv[e + 1]) - dl));
+            for (int e = 0; e < 32; ++e) pr[e] = (c0 + e < nvalid) ? pexp(e) : 0.f;
           }
         }
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, J & 1, abort_flag, p.status));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t dv[32], pk[16];
+        tmem_ld32(tmem + lane_off + 256 + c0, dv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dp_free);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          pk[e >> 1] = pack_bf16(pr[e] * (__uint_as_float(dv[e]) - dl), pr[e + 1] * (__uint_as_float(dv[e + 1]) - dl));
         // packed bf16 dS stays inside this warpgroup's own (already read) column range
         tmem_st16(tS, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_full);
+        if (lane == 0) mbar_arrive(ds_full(J & 1));
       }
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_ready, k & 1, abort_flag, p.status));
       if (!ok) break;
