@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
 
   if (warp == 0 || warp == 3) {
     // ======================= TMA producers of K(J) (warp 0) and V(J) (warp 3), each into its own
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         r[i] = slot < 16 * n_rt ? routed_group(gi, slot, p.nsg, p.kg, ngr, p.status) : 0;
       }
     };
+    pdl_wait();                 // the group indices come from the router (completed before the kernel before)
     read_idx(0, nxt);
     for (int k = 0; ok; ++k) {
       const int u = unit_of_cta(k, cta, G);
@@ -379,6 +381,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int c0 = 32 * w;
+    pdl_wait();                 // O and lse come from the forward kernel, the kernel before
     bool ok = true;
     int J = 0;
     for (int k = 0; ok; ++k) {
@@ -627,6 +630,7 @@ __global__ void __launch_bounds__(640, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
 
   if (warp == 0) {
     // ======================= TMA producer
@@ -637,6 +641,8 @@ __global__ void __launch_bounds__(640, 1)
       tma_load_2d(sbase + L::kK + kKHalf, &tm_ks, 64, krow, kv_full);
       tma_load_2d(sbase + L::kV, &tm_vs, 0, krow, kv_full);
       tma_load_2d(sbase + L::kV + kKHalf, &tm_vs, 64, krow, kv_full);
+      // lse and delta (loaded with each Q/dO step) come from the forward and dQ kernels
+      pdl_wait();
       int issued[NS] = {0, 0, 0, 0};
       for (int j = 0; j < NJ; ++j) {
         const int s = j % NS;
@@ -886,7 +892,9 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  K::dq_tc_kernel<<<(unsigned)grid, 128 + 32 * K::kEWWarps, smem, st>>>(mq, mdo, mkh, mvh, mks, mvs, p);
+  e = launch_dependent(K::dq_tc_kernel, dim3((unsigned)grid), dim3(128 + 32 * K::kEWWarps), smem, st, 1, mq, mdo, mkh,
+                       mvh, mks, mvs, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -921,19 +929,7 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3((unsigned)grid);
-  lc.blockDim = dim3(640);
-  lc.dynamicSmemBytes = smem;
-  lc.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
-  e = cudaLaunchKernelEx(&lc, K::dkdv_tc_kernel, mq, mdo, mks, mvs, p);
+  e = launch_dependent(K::dkdv_tc_kernel, dim3((unsigned)grid), dim3(640), smem, st, (unsigned)cs, mq, mdo, mks, mvs, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

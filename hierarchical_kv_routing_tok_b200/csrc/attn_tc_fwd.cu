@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
 
   if (warp == 0 || warp == 2) {
     // ======================= TMA producers: warp 0 loads Q and the K tiles, warp 2 the V tiles,
@@ -156,8 +157,10 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       tma_prefetch_desc(&tm_vh);
       tma_prefetch_desc(&tm_vs);
     }
-    // the block's history group indices, all read in one round trip before the first load (lane
-    // l holds slots l, l + 32, ...; longer lists read the rest per tile)
+    // the block's history group indices (written by the router, the kernel before: waited for
+    // here, after the Q loads), all read in one round trip before the first load (lane l holds
+    // slots l, l + 32, ...; longer lists read the rest per tile)
+    pdl_wait();
     int32_t gidx[kIdxRegs];
 #pragma unroll
     for (int i = 0; i < kIdxRegs; ++i) {
@@ -464,12 +467,16 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
     const size_t smem = tcfwd::Smem<2>::kBytes + 1024;
     e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    tcfwd::fwd_tc_kernel<2><<<(unsigned)grid, 384, smem, st>>>(mq, mkh, mvh, mks, mvs, p);
+    e = launch_dependent(tcfwd::fwd_tc_kernel<2>, dim3((unsigned)grid), dim3(384), smem, st, 1, mq, mkh, mvh, mks, mvs,
+                         p);
+    if (e != cudaSuccess) return e;
   } else {
     const size_t smem = tcfwd::Smem<1>::kBytes + 1024;
     e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    tcfwd::fwd_tc_kernel<1><<<(unsigned)grid, 256, smem, st>>>(mq, mkh, mvh, mks, mvs, p);
+    e = launch_dependent(tcfwd::fwd_tc_kernel<1>, dim3((unsigned)grid), dim3(256), smem, st, 1, mq, mkh, mvh, mks, mvs,
+                         p);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

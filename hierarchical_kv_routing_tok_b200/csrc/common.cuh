@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace hga {
 
 constexpr int kD = 128;       // head dimension built
@@ -56,6 +58,43 @@ template <> struct Vec16<__nv_bfloat16> {
     }
   }
 };
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization (see
+// launch_dependent) may start while the kernel before it in the stream is still running: its CTAs
+// take SMs as that kernel's CTAs leave them, once every CTA of that kernel has called pdl_trigger().
+// Each of its threads must call pdl_wait() before reading anything an earlier kernel wrote; the
+// wait returns once the kernel before has completed and its memory is visible (at once when the
+// kernel was launched normally).  A kernel whose every CTA waits completes only after its
+// predecessor, so the order of a whole chain of such launches is kept.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch `kernel` as a dependent of the previous kernel in `st` (programmatic stream
+// serialization), optionally in clusters of `cluster` CTAs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                    unsigned cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  unsigned na = 0;
+  at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = cluster;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Record a device-side failure code in the workspace status word (first one wins).
 __device__ __forceinline__ void set_status(int* status, int code) {

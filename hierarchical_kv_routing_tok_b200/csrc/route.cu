@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     const float* __restrict__ chunk_sum, int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq,
     int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  if (threadIdx.x == 0) pdl_trigger();
   constexpr int N = Vec16<T>::N;
   constexpr int LPR = kD / N;
   constexpr int RP = kRouteThreads / LPR;       // rows reduced in parallel
@@ -271,6 +272,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     __syncthreads();
   }
 
+  // the block query needs only q: the summaries are read once the kernel before has completed
+  pdl_wait();
+
   // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
   // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
   const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
@@ -320,15 +324,18 @@ cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool caus
   if (bf16) {
     e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_kernel<__nv_bfloat16><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(q_prev), causal ? 1 : 0, group_sum,
-        chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
+    e = launch_dependent(route_kernel<__nv_bfloat16>, dim3((unsigned)units), dim3(kRouteThreads), smem, stream, 1,
+                         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(q_prev),
+                         causal ? 1 : 0, group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc,
+                         kc, kg);
+    if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_kernel<float><<<(unsigned)units, kRouteThreads, smem, stream>>>(
-        static_cast<const float*>(q), static_cast<const float*>(q_prev), causal ? 1 : 0, group_sum, chunk_sum,
-        chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
+    e = launch_dependent(route_kernel<float>, dim3((unsigned)units), dim3(kRouteThreads), smem, stream, 1,
+                         static_cast<const float*>(q), static_cast<const float*>(q_prev), causal ? 1 : 0, group_sum,
+                         chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

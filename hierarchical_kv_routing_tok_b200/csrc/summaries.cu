@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k_
   constexpr int RPL = 32 / LPR;               // rows per warp-wide load (2 or 1)
   constexpr int LOADS = kGroup / RPL;         // loads per lane
   __shared__ float gmean[kChunk / kGroup][kD];
+  if (threadIdx.x == 0) pdl_trigger();          // the router may start its block-query means
   const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
   const int64_t bkh = blockIdx.x / nc;
   const int64_t c = c0 + blockIdx.x % nc;
