@@ -16,8 +16,8 @@
 //   M dimension: S^T = K Q^T and dP^T = V dO^T (64 queries per step, double-buffered in TMEM),
 //   then dV += P^T dO and dK += dS^T Q with P^T / dS^T read from TMEM.  The G query heads of the
 //   KV head accumulate into the same TMEM dK / dV, one head after another; in a cluster of two each
-//   CTA takes G/2 heads and the two float32 tiles are added through distributed shared memory (one
-//   bulk copy each way), so no partial sums go through HBM and the result is reproducible.
+//   CTA takes G/2 heads and each hands the float32 sums of the rows the other writes over through
+//   an L2-resident exchange area of the workspace, so the result is reproducible.
 // Warp roles as in the forward: warp 0 TMA, warp 1 TMEM owner + single-thread MMA issuer,
 // warps 4..19 four element-wise warpgroups (thread = TMEM lane = row; the warpgroups split a
 // tile's columns so that each thread handles 32 elements per step).  All mbarrier waits are bounded.
@@ -530,7 +530,6 @@ constexpr uint32_t kKHalf = BM * 128;       // 16 KB
 constexpr uint32_t kQTileB = BQ * 256;      // 16 KB
 constexpr uint32_t kQHalfB = BQ * 128;      // 8 KB
 constexpr uint32_t kStatBytes = 2 * BQ * 4; // lse[64], delta[64]
-constexpr uint32_t kAccRow = 2 * kD * 4;    // one key's float32 dV | dK row in the reduction buffer
 
 struct Params {
   int B, Hq, Hkv, G;
@@ -543,6 +542,7 @@ struct Params {
   const float* delta;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* xchg;          // cs == 2: per cluster, two [32 chunks of 4 columns x 2][64 rows] float32 areas
   int* status;
 };
 
@@ -553,24 +553,16 @@ struct Smem {
   static constexpr uint32_t kDO = kQ + NS * kQTileB;
   static constexpr uint32_t kStat = kDO + NS * kQTileB;
   static constexpr uint32_t kBar = kStat + NS * kStatBytes;
-  // kv_full, q_full[NS], q_empty[NS], sd_full[2], pd_full[2], done, mma_done, recv
-  static constexpr int kNumBars = 1 + 2 * NS + 4 + 3;
+  // kv_full, q_full[NS], q_empty[NS], sd_full[2], pd_full[2], done, mma_done
+  static constexpr int kNumBars = 1 + 2 * NS + 4 + 2;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
-  // After the main loop the K, V and Q/dO stage area holds this CTA's float32 dV | dK tile (kAcc)
-  // and, in a cluster of two, the peer's half of its tile for the rows this CTA writes (kRecv).
-  static constexpr uint32_t kAcc = 0;
-  static constexpr uint32_t kRecv = kAcc + BM * kAccRow;
-  static constexpr uint32_t kHalfBytes = (BM / 2) * kAccRow;
-  static_assert(kRecv + kHalfBytes <= kStat, "reduction buffers must not reach the stats or barriers");
 };
 
-// Byte offset of the float4 chunk c16 (0..63: dV columns 0..127, then dK) of key row r in the
-// reduction buffer.  The chunk index is XOR-swizzled by r mod 8 so that a warp writing one
-// chunk of 32 rows, and 16 threads reading consecutive chunks of one row, hit distinct banks.
-__device__ __forceinline__ uint32_t acc_off(int r, int c16) {
-  return (uint32_t)r * kAccRow + ((uint32_t)(c16 ^ (r & 7)) << 4);
-}
+// Exchange area of one direction of one cluster: 64 key rows x 256 float32 (dV | dK), stored as
+// [64 float4 chunks][64 rows] so that a warp's 32 rows of one chunk are 512 contiguous bytes.
+constexpr size_t kXchgFloats = 64 * 256;
+__device__ __forceinline__ size_t xchg_off(int chunk, int row) { return ((size_t)chunk * 64 + row) * 4; }
 
 __global__ void __launch_bounds__(640, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -589,7 +581,6 @@ __global__ void __launch_bounds__(640, 1)
   auto pd_full = [&](int b) { return BAR(3 + 2 * NS + b); };
   const uint32_t done = BAR(5 + 2 * NS);
   const uint32_t mma_done = BAR(6 + 2 * NS);
-  const uint32_t recv_bar = BAR(7 + 2 * NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -618,7 +609,6 @@ __global__ void __launch_bounds__(640, 1)
     }
     mbar_init(done, 1);
     mbar_init(mma_done, 1);
-    mbar_init(recv_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -631,6 +621,8 @@ __global__ void __launch_bounds__(640, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) pdl_trigger();
+  uint32_t va[32], vb[32];   // element-wise threads after the main loop: 64 accumulator columns
+  bool ew_ok = false;
 
   if (warp == 0) {
     // ======================= TMA producer
@@ -786,79 +778,80 @@ __global__ void __launch_bounds__(640, 1)
       tc_fence_before();
       mbar_arrive(pd_full(x));
     }
-    // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK.
-    // After `done` every MMA has completed, so the K, V and Q/dO stage area is free: this CTA's
-    // float32 tile (the sum over its hpc heads) goes there for the reduction and the store.
+    // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK;
+    // after `done` every MMA has completed and each thread takes its 64 columns of the float32 sums
+    // over this CTA's heads into registers.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
     if (ok) {
       tc_fence_after();
-      const bool is_dk = w4 >= 2;
-      const int ch = w4 & 1;
-      const uint32_t tacc = tmem + lane_off + (is_dk ? 384 : 256) + 64 * ch;
-      const float mul = is_dk ? p.scale : 1.f;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tacc + cc * 32, v);
-        tmem_wait_ld();
-        const int c16 = (is_dk ? 32 : 0) + 16 * ch + 8 * cc;
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          st_smem_f4(sbase + L::kAcc + acc_off(r, c16 + e / 4), __uint_as_float(v[e]) * mul,
-                     __uint_as_float(v[e + 1]) * mul, __uint_as_float(v[e + 2]) * mul,
-                     __uint_as_float(v[e + 3]) * mul);
-      }
-      fence_proxy_async_smem();   // the tile is read by a bulk copy below
+      const uint32_t tacc = tmem + lane_off + (w4 >= 2 ? 384 : 256) + 64 * (w4 & 1);
+      tmem_ld32(tacc, va);
+      tmem_ld32(tacc + 32, vb);
+      tmem_wait_ld();
     }
+    ew_ok = ok;
+  }
+  // ---- reduction over the query heads of this KV head and store.  In a cluster of two, CTA
+  // `crank` writes key rows [64 crank, 64 crank + 64): each thread holding a row of the other half
+  // stores its 64 float32 sums into the cluster's exchange area for the peer (L2-resident; a
+  // transfer through distributed shared memory measured several times slower), then a release /
+  // acquire cluster barrier, then each owner adds the row the peer left for it and stores bf16.  A
+  // sum of two terms does not depend on their order, so the result is reproducible.  Every thread
+  // takes part in the barriers on the error path too; a CTA that gave up leaves arbitrary rows and
+  // the status word says so.
+  const int nrows = BM / p.cs;
+  const int r0 = crank * nrows;
+  const int er = (warp & 3) * 32 + lane;                  // element-wise thread: key row (TMEM lane)
+  const int ew4 = (warp - 4) >> 2;
+  const int c16 = (ew4 >= 2 ? 32 : 0) + 16 * (ew4 & 1);   // first float4 chunk of its 64 columns
+  const bool mine = er >= r0 && er < r0 + nrows;
+  float* xc = p.xchg + (size_t)c * 2 * kXchgFloats;        // this cluster's two areas
+  if (p.cs == 2 && warp >= 4 && ew_ok && !mine) {
+    float* to = xc + (size_t)(crank ^ 1) * kXchgFloats;
+    const int rl = er - (crank ^ 1) * nrows;
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      __stcg(reinterpret_cast<float4*>(to + xchg_off(c16 + e / 4, rl)),
+             make_float4(__uint_as_float(va[e]), __uint_as_float(va[e + 1]), __uint_as_float(va[e + 2]),
+                         __uint_as_float(va[e + 3])));
+      __stcg(reinterpret_cast<float4*>(to + xchg_off(c16 + 8 + e / 4, rl)),
+             make_float4(__uint_as_float(vb[e]), __uint_as_float(vb[e + 1]), __uint_as_float(vb[e + 2]),
+                         __uint_as_float(vb[e + 3])));
+    }
+    __threadfence();
   }
   tc_fence_before();
-  __syncthreads();
+  if (p.cs == 2) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  // ---- reduction over the query heads of this KV head and store.  In a cluster of two, CTA
-  // `crank` writes key rows [64 crank, 64 crank + 64): after a cluster barrier (both CTAs have left
-  // their main loops, so the peer's stage area is free) each CTA pushes the peer's rows of its tile
-  // into the peer's kRecv with one bulk copy, then adds the received rows to its own.  A sum of two
-  // terms does not depend on their order, so the result is reproducible.  Every thread takes
-  // part on the error path too; a CTA that gave up leaves an arbitrary tile and the status word
-  // says so.
-  const int nrows = BM / p.cs;
-  const int r0 = crank * nrows;
-  if (p.cs == 2) {
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, L::kHalfBytes);
-    cluster_sync();
-    if (threadIdx.x == 0) {
-      const uint32_t peer = (uint32_t)(crank ^ 1);
-      bulk_copy_to_peer(dsmem_addr(sbase + L::kRecv, peer), sbase + L::kAcc + peer * L::kHalfBytes, L::kHalfBytes,
-                        dsmem_addr(recv_bar, peer));
-      bulk_commit_group();
-    }
-    drain_wait(recv_bar, 0, p.status);
-  }
-  {
-    const int r1 = (int)min((int64_t)(r0 + nrows), p.S - (int64_t)m * BM);
-    const int nitems = max(0, r1 - r0) * 32;  // per row: dV and dK, 16 chunks of 8 columns each
-    const int64_t key0 = (int64_t)bkh * p.S + (int64_t)m * BM;
-    for (int it = threadIdx.x; it < nitems; it += blockDim.x) {
-      const int pr = it & 15, is_dk = (it >> 4) & 1, rr = r0 + (it >> 5);
-      const int c16 = is_dk * 32 + 2 * pr;
-      float4 a = *reinterpret_cast<const float4*>(smem + L::kAcc + acc_off(rr, c16));
-      float4 a2 = *reinterpret_cast<const float4*>(smem + L::kAcc + acc_off(rr, c16 + 1));
-      if (p.cs == 2) {   // received rows keep the row's swizzle: (rr - r0) mod 8 == rr mod 8
-        const float4 x0 = *reinterpret_cast<const float4*>(smem + L::kRecv + acc_off(rr - r0, c16));
-        const float4 x1 = *reinterpret_cast<const float4*>(smem + L::kRecv + acc_off(rr - r0, c16 + 1));
-        a.x += x0.x; a.y += x0.y; a.z += x0.z; a.w += x0.w;
-        a2.x += x1.x; a2.y += x1.y; a2.z += x1.z; a2.w += x1.w;
+  if (warp >= 4 && ew_ok && mine && (int64_t)m * BM + er < p.S) {
+    const bool is_dk = ew4 >= 2;
+    const float mul = is_dk ? p.scale : 1.f;
+    const float* from = xc + (size_t)crank * kXchgFloats;
+    const int rl = er - r0;
+    __nv_bfloat16* dst = (is_dk ? p.dk : p.dv) + ((int64_t)bkh * p.S + (int64_t)m * BM + er) * kD + 64 * (ew4 & 1);
+    auto store32 = [&](const uint32_t(&v)[32], int cbase, int col0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * q + e]);
+        if (p.cs == 2) {
+          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(from + xchg_off(cbase + 2 * q, rl)));
+          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(from + xchg_off(cbase + 2 * q + 1, rl)));
+          f[0] += x0.x; f[1] += x0.y; f[2] += x0.z; f[3] += x0.w;
+          f[4] += x1.x; f[5] += x1.y; f[6] += x1.z; f[7] += x1.w;
+        }
+        *reinterpret_cast<uint4*>(dst + col0 + 8 * q) =
+            make_uint4(pack_bf16(f[0] * mul, f[1] * mul), pack_bf16(f[2] * mul, f[3] * mul),
+                       pack_bf16(f[4] * mul, f[5] * mul), pack_bf16(f[6] * mul, f[7] * mul));
       }
-      __nv_bfloat16* dst = (is_dk ? p.dk : p.dv) + (key0 + rr) * kD + 8 * pr;
-      *reinterpret_cast<uint4*>(dst) =
-          make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(a2.x, a2.y), pack_bf16(a2.z, a2.w));
-    }
+    };
+    store32(va, c16, 0);
+    store32(vb, c16 + 8, 32);
   }
-  // the outgoing copy must have finished reading this CTA's shared memory before the CTA exits
-  if (p.cs == 2 && threadIdx.x == 0) bulk_wait_read_all();
 }
 
 }  // namespace dkdv
@@ -910,9 +903,17 @@ int dkdv_cluster_size(int B, int Hkv, int G, int nkt) {
   return ((int64_t)B * Hkv * nkt >= sms) ? 1 : 2;
 }
 
+// Bytes of the exchange area the dK/dV kernel uses when it pairs CTAs (0 when it does not).
+size_t dkdv_xchg_bytes(int B, int Hq, int Hkv, int64_t S) {
+  const int nkt = (int)((S + tcbwd::dkdv::BM - 1) / tcbwd::dkdv::BM);
+  if (dkdv_cluster_size(B, Hkv, Hq / Hkv, nkt) != 2) return 0;
+  return (size_t)B * Hkv * nkt * 2 * tcbwd::dkdv::kXchgFloats * sizeof(float);
+}
+
+// xchg: the exchange area (dkdv_xchg_bytes), or nullptr, in which case no CTAs are paired.
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
-                               const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
-                               int* status, cudaStream_t st) {
+                               const float* delta, void* dk, void* dv, float* xchg, int B, int Hq, int Hkv, int64_t S,
+                               float scale, int* status, cudaStream_t st) {
   namespace K = tcbwd::dkdv;
   CUtensorMap mq, mdo, mks, mvs;
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, K::BQ) ||
@@ -921,10 +922,10 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BM))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
-  const int cs = dkdv_cluster_size(B, Hkv, G, (int)((S + K::BM - 1) / K::BM));
   const int nkt = (int)((S + K::BM - 1) / K::BM);
+  const int cs = xchg ? dkdv_cluster_size(B, Hkv, G, nkt) : 1;
   K::Params p{B, Hq, Hkv, G, cs, G / cs, (int)(S / kQBlock), nkt, S, scale * tcbwd::kLog2e, scale, lse, delta,
-              static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), status};
+              static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), xchg, status};
   const int64_t grid = (int64_t)B * Hkv * nkt * cs;
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

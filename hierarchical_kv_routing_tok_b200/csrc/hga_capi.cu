@@ -28,9 +28,10 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
                              const int32_t* gi, const float* lse, const void* o, const void* d_o, float* delta,
                              void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg,
                              float scale, int* status, cudaStream_t st);
+size_t dkdv_xchg_bytes(int B, int Hq, int Hkv, int64_t S);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
-                               const float* delta, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, float scale,
-                               int* status, cudaStream_t st);
+                               const float* delta, void* dk, void* dv, float* xchg, int B, int Hq, int Hkv, int64_t S,
+                               float scale, int* status, cudaStream_t st);
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
@@ -139,17 +140,29 @@ bool force_cuda_cores() {
 // The workspace starts with the status word.
 int* status_of(void* workspace) { return static_cast<int*>(workspace); }
 
-// Workspace layout: [status word | delta rows (float32)].
+// The tensor-core attention kernels handle bf16 with an even number of query heads per KV head.
+bool use_tc(const hga_config_t* c) {
+  return c->dtype == HGA_BF16 && hga::attn_fwd_tc_supported(c->Hq, c->Hkv) && !force_cuda_cores();
+}
+
+// Workspace layout: [status word | delta rows (float32) | dK/dV exchange area].  The exchange area
+// is used only by the tensor-core dK/dV kernel when it pairs CTAs (few (batch, KV head, key tile)
+// units for the GPU's SMs); a workspace that ends before it (the no-allocation entry point's fixed
+// scratch) runs that kernel unpaired.
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t delta_bytes(const hga_config_t* c) { return (size_t)c->B * c->Hq * c->seg_len * sizeof(float); }
 float* delta_of(void* workspace) {
   return reinterpret_cast<float*>(static_cast<char*>(workspace) + hga::kStatusBytes);
 }
-size_t full_workspace_bytes(const hga_config_t* c) { return hga::kStatusBytes + round256(delta_bytes(c)); }
-
-// The tensor-core attention kernels handle bf16 with an even number of query heads per KV head.
-bool use_tc(const hga_config_t* c) {
-  return c->dtype == HGA_BF16 && hga::attn_fwd_tc_supported(c->Hq, c->Hkv) && !force_cuda_cores();
+size_t base_workspace_bytes(const hga_config_t* c) { return hga::kStatusBytes + round256(delta_bytes(c)); }
+size_t xchg_bytes(const hga_config_t* c) {
+  return use_tc(c) ? hga::dkdv_xchg_bytes(c->B, c->Hq, c->Hkv, c->seg_len) : 0;
+}
+size_t full_workspace_bytes(const hga_config_t* c) { return base_workspace_bytes(c) + xchg_bytes(c); }
+float* xchg_of(void* workspace, const hga_config_t* c, size_t ws_bytes) {
+  const size_t x = xchg_bytes(c);
+  if (x == 0 || ws_bytes < base_workspace_bytes(c) + x) return nullptr;
+  return reinterpret_cast<float*>(static_cast<char*>(workspace) + base_workspace_bytes(c));
 }
 
 // dK/dV with a workspace of ws_bytes (status word and delta rows).
@@ -160,11 +173,11 @@ int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const
   if (!workspace) return HGA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HGA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (ws_bytes < full_workspace_bytes(cfg)) return HGA_ERR_WORKSPACE;
+  if (ws_bytes < base_workspace_bytes(cfg)) return HGA_ERR_WORKSPACE;
   if (use_tc(cfg))
-    return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg, cfg->B,
-                                             cfg->Hq, cfg->Hkv, cfg->seg_len, eff_scale(cfg), status_of(workspace),
-                                             st));
+    return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg,
+                                             xchg_of(workspace, cfg, ws_bytes), cfg->B, cfg->Hq, cfg->Hkv,
+                                             cfg->seg_len, eff_scale(cfg), status_of(workspace), st));
   return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
                                              dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
                                              cfg->top_groups, eff_scale(cfg), st));

@@ -65,16 +65,24 @@ def cfg(**kw):
     return C.make_config(**base)
 
 
-def _expected_ws(B, Hq, Hkv, S):
+def _expected_ws(B, Hq, Hkv, S, bf16=True, sms=148):
+    """Status word, delta rows, and (bf16 tensor-core path, fewer (batch, KV head, 128-key tile)
+    units than SMs: the dK/dV kernel pairs CTAs) one 2 x 64 KB exchange area per unit."""
     r256 = lambda x: (x + 255) // 256 * 256
     delta = B * Hq * S * 4
-    return 256 + r256(delta)
+    units = B * Hkv * ((S + 127) // 128)
+    paired = bf16 and (Hq // Hkv) % 2 == 0 and units < sms
+    return 256 + r256(delta) + (units * 2 * 64 * 256 * 4 if paired else 0)
 
 
 def test_workspace_size(lib):
     assert C.workspace_size(cfg()) == _expected_ws(1, 32, 8, 2048)
     assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) == _expected_ws(3, 4, 1, 64)
     assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) % 256 == 0
+    # float32, odd G and many units: no exchange area
+    assert C.workspace_size(cfg(dtype=C.HGA_F32)) == 256 + 1 * 32 * 2048 * 4
+    assert C.workspace_size(cfg(Hq=24)) == _expected_ws(1, 24, 8, 2048, sms=0)
+    assert C.workspace_size(cfg(B=4)) == _expected_ws(4, 32, 8, 2048, sms=0)
 
 
 @pytest.mark.parametrize("kw,code", [
