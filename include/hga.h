@@ -44,7 +44,11 @@
  *     filled once before its first use (cudaMemset).  Layout: a 256-byte
  *     sticky status word (must start at zero; read and cleared by
  *     hga_read_status()), then the backward's delta rows (B*Hq*S float32,
- *     written before they are read).  Kernels that wait on on-chip barriers give up after
+ *     written before they are read), then, only for the bf16 tensor-core path
+ *     when B*Hkv*ceil(S/128) is below the GPU's SM count, an exchange area of
+ *     128 KB per such (batch, KV head, 128-key tile) unit in which the dK/dV
+ *     kernel's CTA pairs hand each other float32 row sums (written before they
+ *     are read).  Kernels that wait on on-chip barriers give up after
  *     a bounded time and record HGA_ERR_TIMEOUT there instead of hanging; an
  *     attention kernel given a group index outside [0, H/8) reads that group
  *     as zeros (never out of bounds) and records HGA_ERR_ARG there; so does a
@@ -181,7 +185,7 @@ HGA_API int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_h
  *   pairs only, summed over the G query heads of each KV head.
  * No gradient is produced for k_hist / v_hist.  o and lse are the forward's
  * outputs.  dq [B,Hq,S,D], dk_seg, dv_seg [B,Hkv,S,D] in cfg->dtype (out).
- * Uses the workspace scratch described above (delta, dK/dV accumulators). */
+ * Uses the workspace scratch described above (delta, dK/dV exchange area). */
 HGA_API int hga_attn_bwd(const hga_config_t* cfg, const void* q, const void* k_hist,
                  const void* v_hist, const void* k_seg, const void* v_seg,
                  const int32_t* group_idx, const void* o, const float* lse,
@@ -216,7 +220,9 @@ HGA_API int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* 
  *
  * Scratch: instead of a caller workspace it uses one fixed device array of
  * 256 + 4 * HGA_NOALLOC_MAX_ROWS bytes (4 MiB + 256 B) that every GPU loading
- * the library holds until the process exits.  B * Hq * S must not exceed
+ * the library holds until the process exits.  It has no dK/dV exchange area,
+ * so the dK/dV kernel runs with unpaired CTAs here (same result up to float32
+ * summation order, slower when B*Hkv*ceil(S/128) is below the SM count).  B * Hq * S must not exceed
  * HGA_NOALLOC_MAX_ROWS, else HGA_ERR_TOO_LARGE is returned and nothing runs.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
