@@ -290,6 +290,44 @@ def _time_tiered(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=2) ->
             "resident_ms_per_step": resident_ms, "resident_tokens_per_s": tokens / (resident_ms * 1e-3)}
 
 
+def _time_forward_131k(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=3) -> dict:
+    """Evaluation-length forward, no backward: the summaries of the whole history built on the
+    device, routing, and the routed + causal forward.  Each kernel is bracketed by CUDA events (so
+    the kernels do not overlap through dependent launch here), L2 flushed before every step; also
+    reports how many planted needle groups the routing recovered."""
+    xc = HI.make_inputs(w, seed)
+    needles = xc.pop("needles")
+    x = {k: v.to(dev) for k, v in xc.items()}
+    cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    step = H.LayerStep(cfg, dev)
+    calls = step.calls(x, stream.cuda_stream)[:3]          # summaries, route, attn_fwd
+    for _ in range(warmup):
+        for _, c in calls:
+            c()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    for e in ev:
+        flush_l2()
+        e[0].record(stream)
+        for j, (_, c) in enumerate(calls):
+            c()
+            e[j + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    if H.read_status(step.ws) != 0:
+        raise RuntimeError(f"device status word set while timing {w.name}")
+    ms = all_max(sum(e[0].elapsed_time(e[-1]) for e in ev) / steps, world, dev)
+    per_us = {n: 1e3 * sum(e[j].elapsed_time(e[j + 1]) for e in ev) / steps for j, (n, _) in enumerate(calls)}
+    wm, pk = work_model(w), _peaks()
+    frac = {n: wm[n][1] / (per_us[n] * 1e-6) / ((pk["bf16"] * 1e12) if wm[n][0] == "tensor" else (pk["hbm"] * 1e9))
+            for n in per_us}
+    gi = step.group_idx.cpu()
+    hits = sum(int(j) in gi[0, kh, n].tolist() for kh, n, j in needles.tolist())
+    return {"workload": f"{w.name}: B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, history={w.hist_len}, segment={w.seg_len}, "
+                        f"top_chunks={w.top_chunks}, top_groups={w.top_groups}, {w.dtype}, forward only",
+            "ms_per_step": ms, "tokens_per_s": w.B * w.seg_len * world / (ms * 1e-3),
+            "per_kernel_us": per_us, "per_kernel_frac": frac,
+            "needles_recovered": f"{hits}/{len(needles)}"}
+
+
 def _config(w, args):
     return {"workload": f"{w.name}: routed HGA layer, B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, "
                         f"history={w.hist_len}, segment={w.seg_len}, chunk=64, group=8, qblock=64, "
@@ -312,6 +350,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tiered", action="store_true", help="skip the tiered-history (batch 4) measurement")
+    ap.add_argument("--no-131k", action="store_true", help="skip the 131K-context forward measurement")
     ap.add_argument("--no-positions", action="store_true",
                     help="skip timing the 16K layer at its earlier segment positions and other budgets")
     args = ap.parse_args()
@@ -420,6 +459,11 @@ def main():
     if w.name == "ctx16k" and not args.no_tiered:
         tiered = _time_tiered(H, HI.WORKLOADS["ctx16k_b4"], args.seed + rank, dev, stream, flush_l2, world)
 
+    # evaluation-length forward (131K context, routing over 129,024 history tokens, planted needles)
+    fwd131k = None
+    if w.name == "ctx16k" and not args.no_131k:
+        fwd131k = _time_forward_131k(H, HI.WORKLOADS["ctx131k"], args.seed + rank, dev, stream, flush_l2, world)
+
     # roofline of the dominant kernel
     wm = work_model(w)
     pk = _peaks()
@@ -526,6 +570,8 @@ def main():
             line["strictly_causal_routing"] = causal
         if tiered:
             line["tiered_history"] = tiered
+        if fwd131k:
+            line["forward_131k"] = fwd131k
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
