@@ -73,8 +73,8 @@ struct Smem {
   static constexpr uint32_t kV = kK + KS * kKVTile;
   static constexpr uint32_t kBar = kV + VS * kKVTile;
   // qdo_full, kv_full[KS], k_empty[KS], v_empty[VS], s_full[2], dp_full, dp_free, ds_full[2],
-  // dq_ready, mma_done, qdo_empty, delta_bar
-  static constexpr int kNumBars = 1 + 2 * KS + VS + 11;
+  // dq_ready, mma_done, qdo_empty, delta_bar, qdo_issued
+  static constexpr int kNumBars = 1 + 2 * KS + VS + 12;
   static constexpr uint32_t kMisc = kBar + 8 * kNumBars;
   static constexpr uint32_t kBytes = kMisc + 16;
 };
@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
   const uint32_t mma_done = BAR(8 + 2 * KS + VS);
   const uint32_t qdo_empty = BAR(9 + 2 * KS + VS);          // the unit's Q/dO fully read
   const uint32_t delta_bar = BAR(10 + 2 * KS + VS);         // delta partial sums in TMEM
+  const uint32_t qdo_issued = BAR(11 + 2 * KS + VS);        // a unit's Q/dO loads are issued
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     mbar_init(mma_done, 1);
     mbar_init(qdo_empty, 1 + kEWWarps);     // the MMA warp's commit + every element-wise warp
     mbar_init(delta_bar, kEWWarps);
+    mbar_init(qdo_issued, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -181,7 +183,9 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     // ring, across all units; both arrive on kv_full of the tile.  A routed history group (8 rows)
     // is one 3-D box: its two 64-column halves land 1 KB apart in the group layout.  A unit's
     // group indices are read one unit ahead, all in one round trip (lane l holds slots l, l + 32,
-    // ...), so the index reads never stand between a free slot and its loads.
+    // ...), so the index reads never stand between a free slot and its loads.  A unit's first
+    // tiles are issued only after its Q/dO loads: those are needed first, and otherwise wait in the
+    // TMA queue behind the dozens of group boxes the rings run ahead.
     const bool is_v = warp == 3;
     const CUtensorMap* hist_map = is_v ? &tm_vh : &tm_kh;
     const CUtensorMap* seg_map = is_v ? &tm_vs : &tm_ks;
@@ -210,6 +214,12 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
 #pragma unroll
       for (int i = 0; i < kIdxRegs; ++i) cur[i] = nxt[i];
       read_idx(k + 1, nxt);
+      if (k > 0) {
+        int okq = 1;
+        if (lane == 0) okq = mbar_wait(qdo_issued, k & 1, abort_flag, p.status);
+        ok = __shfl_sync(0xffffffffu, okq, 0) != 0;
+        if (!ok) break;
+      }
       for (int j = 0; j < x.T; ++j, ++J) {
         const int ks = J % KS, vs = J % VS;
         int okk = 1;
@@ -270,6 +280,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
             tma_load_2d(sbase + L::kDO + off, &tm_do, 64 * h, (int32_t)row, qdo_full);
           }
         }
+        mbar_arrive(qdo_issued);
         ++loads;
       }
       if (loads) drain_wait(qdo_full, (loads - 1) & 1, p.status);
@@ -324,8 +335,9 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     // Per tile J: S(J+1) as soon as its K tile has landed (the other S buffer, whose dS(J-1) the
     // last dQ MMA has read); dP(J+1) once the element-wise warps hold dP(J); dQ += dS(J) K(J) once
     // they have written dS(J).  The next tile may be the next unit's first, once its Q/dO have
-    // landed.  The unit's Q/dO are released after its last dP MMAs (issued after its last S MMAs),
-    // dQ after its last dS K MMAs.
+    // landed: at a unit's last tile dQ += dS K is issued first and dQ released, so that the
+    // element-wise warps' dQ epilogue and the next unit's delta do not wait for the next unit's
+    // loads.  The unit's Q/dO are released after its last dP MMAs (issued after its last S MMAs).
     bool ok = true;
     int J = 0;
     Unit x{};
@@ -348,6 +360,18 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         const bool next = !last || has_next;
         const int jn = last ? 0 : j + 1;          // the next tile's index in its unit
         const int Tn = last ? xn.T : x.T;
+        auto finish_tile = [&]() {                // dQ (+)= dS(J) K(J), then K(J) is free
+          ok = mbar_wait_w(ds_full(J & 1), (J >> 1) & 1, abort_flag, p.status);
+          if (!ok) return;
+          tc_fence_after();
+          issue_dq(J, j < n_rt, j == 0);
+          mma_commit_w(k_empty(J % KS));
+        };
+        if (last) {                               // the unit's dQ is complete after these MMAs
+          finish_tile();
+          if (!ok) break;
+          mma_commit_w(dq_ready);
+        }
         if (next) {
           if (last) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status);
           if (ok) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status);
@@ -360,14 +384,12 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
           issue_dp(J + 1, jn < n_rt);
           if (jn + 1 == Tn) mma_commit_w(qdo_empty);
         }
-        ok = mbar_wait_w(ds_full(J & 1), (J >> 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dq(J, j < n_rt, j == 0);
-        mma_commit_w(k_empty(J % KS));
+        if (!last) {
+          finish_tile();
+          if (!ok) break;
+        }
       }
       if (!ok) break;
-      mma_commit_w(dq_ready);
       u = un;
       x = xn;
     }
