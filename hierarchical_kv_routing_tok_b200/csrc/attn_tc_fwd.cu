@@ -7,10 +7,12 @@
 //
 // One CTA per (batch, KV head, 64-query block, pair of query-head pairs): its query tile is
 // hpc = 2 * NT query heads x 64 positions = NT M-tiles of 128 rows that share one routed key set,
-// so every gathered K/V byte feeds NT MMAs.  Key tiles hold 128 keys:
-//   routed tiles: 16 groups of 8 history rows, each group fetched by TMA as two 8x64 boxes
-//                 (one per 64-dim half) into its own 1 KB swizzle atoms ("group layout");
-//   local tiles:  128 consecutive segment rows, two 128x64 boxes ("tile layout").
+// so every gathered K/V byte feeds NT MMAs.  Key tiles hold 128 keys, the causal-local tiles first
+// (they need only the step's inputs, so they run while the router, the kernel before, finishes
+// and while the routed groups' indices are read and their K/V gathered), then the routed ones:
+//   local tiles:  128 consecutive segment rows, two 128x64 boxes ("tile layout");
+//   routed tiles: 16 groups of 8 history rows, each group fetched by TMA as one 3-D box whose two
+//                 64-dim halves land in its own two 1 KB swizzle atoms ("group layout").
 // Warp roles: warp 0 = TMA producer, warp 1 = TMEM owner + single-thread MMA issuer,
 // warps 4.. = one softmax warpgroup per M-tile (thread = TMEM lane = query row).
 // TMEM: S_i (128 fp32 columns, P_i packed bf16 aliased into its first 64) and O_i (128 columns).
@@ -157,18 +159,21 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       tma_prefetch_desc(&tm_vh);
       tma_prefetch_desc(&tm_vs);
     }
-    // the block's history group indices (written by the router, the kernel before: waited for
-    // here, after the Q loads), all read in one round trip before the first load (lane l holds
-    // slots l, l + 32, ...; longer lists read the rest per tile)
-    pdl_wait();
     int32_t gidx[kIdxRegs];
-#pragma unroll
-    for (int i = 0; i < kIdxRegs; ++i) {
-      const int slot = 32 * i + lane;
-      gidx[i] = slot < 16 * n_rt ? routed_group(gi, slot, p.nsg, p.kg, ngr, p.status) : 0;
-    }
     int issued[KS] = {0, 0, 0};
     for (int j = 0; j < T; ++j) {
+      const int jr = j - n_lt;                            // routed tile index (>= 0: routed)
+      if (jr == 0) {
+        // the block's history group indices, written by the router (the kernel before): waited
+        // for only here, after the local tiles, and all read in one round trip (lane l holds
+        // slots l, l + 32, ...; longer lists read the rest per tile)
+        pdl_wait();
+#pragma unroll
+        for (int i = 0; i < kIdxRegs; ++i) {
+          const int slot = 32 * i + lane;
+          gidx[i] = slot < 16 * n_rt ? routed_group(gi, slot, p.nsg, p.kg, ngr, p.status) : 0;
+        }
+      }
       const int s = j % NS;
       const uint32_t full = kv ? v_full(s) : k_full(s);
       const uint32_t empty = kv ? v_empty(s) : k_empty(s);
@@ -180,25 +185,25 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      if (j < n_rt) {
+      if (jr >= 0) {
         // 16 routed groups, one per lane, each group's 8 rows one 3-D box (its two 64-column halves
         // land 1 KB apart)
         int32_t g;
-        if (j < 2 * kIdxRegs) {
+        if (jr < 2 * kIdxRegs) {
           int32_t sel = 0;
 #pragma unroll
           for (int i = 0; i < kIdxRegs; ++i)
-            if (i == (j >> 1)) sel = gidx[i];
-          g = __shfl_sync(0xffffffffu, sel, (16 * j + lane) & 31);
+            if (i == (jr >> 1)) sel = gidx[i];
+          g = __shfl_sync(0xffffffffu, sel, (16 * jr + lane) & 31);
         } else {
-          g = lane < 16 ? routed_group(gi, j * 16 + lane, p.nsg, p.kg, ngr, p.status) : 0;
+          g = lane < 16 ? routed_group(gi, jr * 16 + lane, p.nsg, p.kg, ngr, p.status) : 0;
         }
         if (g < 0) g = 0;
         if (lane < 16)
           tma_load_3d(dst + lane * 2048, kv ? &tm_vh : &tm_kh, 0, (int32_t)((int64_t)bkh * p.Hs + (int64_t)g * kGroup),
                       0, full);
       } else if (lane == 0) {
-        const int jl = j - n_rt;
+        const int jl = j;
         const int32_t row = (int32_t)((int64_t)bkh * p.S + (int64_t)jl * BN);
         const CUtensorMap* m = kv ? &tm_vs : &tm_ks;
         tma_load_2d(dst, m, 0, row, full);
@@ -222,11 +227,11 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
 #pragma unroll
       for (int i = 0; i < NT; ++i) kmajor_descs(qd[i], sbase + L::kQ + i * kTileBytes, kHalfBytes, 1024);
       auto build_k = [&](int j) {
-        const bool routed = j < n_rt;
+        const bool routed = j >= n_lt;
         kmajor_descs(kd, sbase + L::kK + (j % KS) * kTileBytes, routed ? 1024u : kHalfBytes, routed ? 2048u : 1024u);
       };
       auto build_v = [&](int j) {
-        const bool routed = j < n_rt;
+        const bool routed = j >= n_lt;
         mnmajor_descs<8>(vd, sbase + L::kV + (j % VS) * kTileBytes, routed ? 1024u : kHalfBytes,
                          routed ? 2048u : 1024u);
       };
@@ -293,12 +298,12 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const bool routed = j < n_rt;
+      const bool routed = j >= n_lt;
       int nvalid;
       if (routed) {
-        nvalid = min(BN, n_hist - j * BN);
+        nvalid = min(BN, n_hist - (j - n_lt) * BN);
       } else {
-        const int64_t u0 = (int64_t)(j - n_rt) * BN;
+        const int64_t u0 = (int64_t)j * BN;
         nvalid = (int)max((int64_t)0, min((int64_t)BN, t_pos - u0 + 1));
       }
       // The whole 128-column row is loaded with one TMEM round trip and kept in registers.
