@@ -494,60 +494,73 @@ def main():
     # end to end through the public API with pinned host buffers: every step copies its inputs in
     # and its outputs out.  Steps are pipelined the way a stream of steps would run: two sets of
     # device buffers, the host->device copy of step i+1 and the device->host copy of step i-1 (two
-    # copy engines, two streams) overlap the compute of step i.
+    # copy engines, two streams) overlap the compute of step i.  The workload keeps the detached
+    # history's K/V resident in HBM (it is device state that successive segments append to, not a
+    # per-step input), so the headline copies the active segment's q, k_seg, v_seg, d_o per step;
+    # the same pipeline with the history K/V copied in every step as well is reported beside it.
     e2e = None
     if not args.no_e2e:
-        in_names = ["q", "k_hist", "v_hist", "k_seg", "v_seg", "d_o"]
-        host_in = {k: x_cpu[k].pin_memory() for k in in_names}
-        sets = []
-        for b in range(2):
-            xs = x if b == 0 else {k: torch.empty_like(v) for k, v in x.items()}
-            st_b = step if b == 0 else H.LayerStep(cfg, dev)
-            sets.append((xs, st_b, st_b.calls(xs, stream.cuda_stream)))
+        x_host = {k: x_cpu[k].pin_memory() for k in ("q", "k_hist", "v_hist", "k_seg", "v_seg", "d_o")}
         outs_of = lambda st_b: [st_b.o, st_b.dq, st_b.dk, st_b.dv]
         host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_of(step)]
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out)
         K2 = max(3, min(K, 10))
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-        def run_e2e(n):
-            ev = lambda: torch.cuda.Event()
-            copied, computed, drained = [None] * n, [None] * n, [None] * n
-            for i in range(n):
-                xs, st_b, cl = sets[i % 2]
-                with torch.cuda.stream(s_in):            # inputs of step i (set i % 2 free after step i-2)
-                    if i >= 2:
-                        s_in.wait_event(computed[i - 2])
-                    for k in in_names:
-                        xs[k].copy_(host_in[k], non_blocking=True)
-                    copied[i] = ev(); copied[i].record(s_in)
-                stream.wait_event(copied[i])             # compute of step i
-                if i >= 2:
-                    stream.wait_event(drained[i - 2])    # its output buffers were read out
-                for _, c in cl:
-                    c()
-                computed[i] = ev(); computed[i].record(stream)
-                with torch.cuda.stream(s_out):           # outputs of step i
-                    s_out.wait_event(computed[i])
-                    for d, h in zip(outs_of(st_b), host_out):
-                        h.copy_(d, non_blocking=True)
-                    drained[i] = ev(); drained[i].record(s_out)
-            stream.wait_event(drained[n - 1])
+        def time_e2e(in_names):
+            sets = []
+            for b in range(2):
+                xs = x if b == 0 else {k: (torch.empty_like(v) if k in in_names else v) for k, v in x.items()}
+                st_b = step if b == 0 else H.LayerStep(cfg, dev)
+                sets.append((xs, st_b, st_b.calls(xs, stream.cuda_stream)))
 
-        run_e2e(2)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run_e2e(K2)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        t_e2e = all_max(e0.elapsed_time(e1) / K2, world, dev) * 1e-3
+            def run_e2e(n):
+                ev = lambda: torch.cuda.Event()
+                copied, computed, drained = [None] * n, [None] * n, [None] * n
+                for i in range(n):
+                    xs, st_b, cl = sets[i % 2]
+                    with torch.cuda.stream(s_in):            # inputs of step i (set i % 2 free after step i-2)
+                        if i >= 2:
+                            s_in.wait_event(computed[i - 2])
+                        for k in in_names:
+                            xs[k].copy_(x_host[k], non_blocking=True)
+                        copied[i] = ev(); copied[i].record(s_in)
+                    stream.wait_event(copied[i])             # compute of step i
+                    if i >= 2:
+                        stream.wait_event(drained[i - 2])    # its output buffers were read out
+                    for _, c in cl:
+                        c()
+                    computed[i] = ev(); computed[i].record(stream)
+                    with torch.cuda.stream(s_out):           # outputs of step i
+                        s_out.wait_event(computed[i])
+                        for d, h in zip(outs_of(st_b), host_out):
+                            h.copy_(d, non_blocking=True)
+                        drained[i] = ev(); drained[i].record(s_out)
+                stream.wait_event(drained[n - 1])
+
+            run_e2e(2)
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run_e2e(K2)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            t = all_max(e0.elapsed_time(e1) / K2, world, dev) * 1e-3
+            h2d = sum(x_host[k].numel() * x_host[k].element_size() for k in in_names)
+            return t, h2d
+
+        t_e2e, h2d = time_e2e(["q", "k_seg", "v_seg", "d_o"])
+        t_all, h2d_all = time_e2e(["q", "k_hist", "v_hist", "k_seg", "v_seg", "d_o"])
         e2e = {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": t_e2e * 1e3,
-               "pipelining": "host->device copy of step i+1 and device->host copy of step i-1 overlap step i"}
+               "per_step_inputs": "q, k_seg, v_seg, d_o copied in, o, dq, dk, dv copied out every step; the "
+                                  "history K/V resident in HBM (device state the segments append to)",
+               "pipelining": "host->device copy of step i+1 and device->host copy of step i-1 overlap step i",
+               "history_copied_every_step": {"value": tokens / t_all, "unit": "tokens/s",
+                                             "h2d_bytes_per_step": h2d_all, "d2h_bytes_per_step": d2h,
+                                             "ms_per_step": t_all * 1e3}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
