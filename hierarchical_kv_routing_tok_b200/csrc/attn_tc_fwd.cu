@@ -71,7 +71,8 @@ template <int NT>
 __global__ void __launch_bounds__(128 + 128 * NT, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                   const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
-                  const __grid_constant__ CUtensorMap tm_vs, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_o,
+                  const Params p) {
   using L = Smem<NT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -370,9 +371,13 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // O / l as bf16 into this M-tile's (now unused) Q area, in the layout its Q tile was loaded
+      // in (two 64-dim halves, 128-byte swizzle), then each warp stores its 32 rows with TMA (one
+      // 32-row box per half): full 128-byte lines instead of one 16-byte piece per row per store
+      // instruction.  After o_final every MMA has completed, so nothing reads Q any more.
       tc_fence_after();
       const float inv = 1.f / l;
-      __nv_bfloat16* dst = p.o + (((int64_t)b * p.Hq + head) * p.S + t_pos) * kD;
+      const uint32_t qt = sbase + L::kQ + i * kTileBytes + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
@@ -382,10 +387,28 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
           pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+        // columns 32 cc .. 32 cc + 31: half cc / 2, 16-byte chunks 4 (cc % 2) .. + 3 of the row
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t chunk = (uint32_t)(4 * (cc & 1) + q4);
+          const uint32_t a = qt + (uint32_t)(cc >> 1) * kHalfBytes + ((chunk ^ (uint32_t)(r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]),
+                       "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3])
+                       : "memory");
+        }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        // rows 32 quarter .. + 31 of the M-tile: head 2 i + quarter / 2, positions 32 (quarter % 2) ..
+        const int64_t orow =
+            ((int64_t)b * p.Hq + h0 + 2 * i + (quarter >> 1)) * p.S + (int64_t)n * kQBlock + 32 * (quarter & 1);
+        for (int h = 0; h < 2; ++h)
+          tma_store_2d(&tm_o, 64 * h, (int32_t)orow, sbase + L::kQ + i * kTileBytes + h * kHalfBytes + quarter * 4096);
+        bulk_commit_group();
+        bulk_wait_read_all();   // the shared-memory source must be read before the CTA exits
+      }
+      __syncwarp();
       p.lse[((int64_t)b * p.Hq + head) * p.S + t_pos] = (m + __log2f(l)) * 0.6931471805599453f;
     }
   }
@@ -458,7 +481,9 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
   const void* kh_m = Hs ? kh : ks;
   const void* vh_m = Hs ? vh : vs;
   const uint64_t hrows = (uint64_t)B * Hkv * (Hs ? Hs : S);
-  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_groups(&mkh, kh_m, hrows) ||
+  CUtensorMap mo;   // O stores: one 32-row box per warp and 64-dim half
+  if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, 64) || !make_map_bf16_rows(&mo, o, (uint64_t)B * Hq * S, 32) ||
+      !make_map_bf16_groups(&mkh, kh_m, hrows) ||
       !make_map_bf16_groups(&mvh, vh_m, hrows) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, tcfwd::BN) ||
       !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, tcfwd::BN))
@@ -473,14 +498,14 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
     e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = launch_dependent(tcfwd::fwd_tc_kernel<2>, dim3((unsigned)grid), dim3(384), smem, st, 1, mq, mkh, mvh, mks, mvs,
-                         p);
+                         mo, p);
     if (e != cudaSuccess) return e;
   } else {
     const size_t smem = tcfwd::Smem<1>::kBytes + 1024;
     e = cudaFuncSetAttribute(tcfwd::fwd_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = launch_dependent(tcfwd::fwd_tc_kernel<1>, dim3((unsigned)grid), dim3(256), smem, st, 1, mq, mkh, mvh, mks, mvs,
-                         p);
+                         mo, p);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
