@@ -589,6 +589,7 @@ __device__ __forceinline__ size_t xchg_off(int chunk, int row) { return ((size_t
 __global__ void __launch_bounds__(640, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                    const Params p) {
   using L = Smem;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -849,12 +850,16 @@ __global__ void __launch_bounds__(640, 1)
     tmem_dealloc(tmem, 512);
   }
   if (warp >= 4 && ew_ok && mine && (int64_t)m * BM + er < p.S) {
+    // the row's 64 bf16 columns go into this warp's 4 KB slot of the (now unused) K/V stage area in
+    // the 128-byte swizzled layout of a {64 columns, 32 rows} box, and the warp stores its 32 rows
+    // with one TMA store (the rows past the segment end are whole warps, S being a multiple of 64)
     const bool is_dk = ew4 >= 2;
     const float mul = is_dk ? p.scale : 1.f;
     const float* from = xc + (size_t)crank * kXchgFloats;
     const int rl = er - r0;
-    __nv_bfloat16* dst = (is_dk ? p.dk : p.dv) + ((int64_t)bkh * p.S + (int64_t)m * BM + er) * kD + 64 * (ew4 & 1);
-    auto store32 = [&](const uint32_t(&v)[32], int cbase, int col0) {
+    const uint32_t slot = sbase + L::kK + (uint32_t)(warp - 4) * 4096u;
+    const uint32_t row_addr = slot + (uint32_t)lane * 128u;
+    auto stage32 = [&](const uint32_t(&v)[32], int cbase, int chunk0) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float f[8];
@@ -866,13 +871,24 @@ __global__ void __launch_bounds__(640, 1)
           f[0] += x0.x; f[1] += x0.y; f[2] += x0.z; f[3] += x0.w;
           f[4] += x1.x; f[5] += x1.y; f[6] += x1.z; f[7] += x1.w;
         }
-        *reinterpret_cast<uint4*>(dst + col0 + 8 * q) =
-            make_uint4(pack_bf16(f[0] * mul, f[1] * mul), pack_bf16(f[2] * mul, f[3] * mul),
-                       pack_bf16(f[4] * mul, f[5] * mul), pack_bf16(f[6] * mul, f[7] * mul));
+        const uint32_t chunk = (uint32_t)(chunk0 + q);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((chunk ^ (uint32_t)(lane & 7)) << 4)),
+                     "r"(pack_bf16(f[0] * mul, f[1] * mul)), "r"(pack_bf16(f[2] * mul, f[3] * mul)),
+                     "r"(pack_bf16(f[4] * mul, f[5] * mul)), "r"(pack_bf16(f[6] * mul, f[7] * mul))
+                     : "memory");
       }
     };
-    store32(va, c16, 0);
-    store32(vb, c16 + 8, 32);
+    stage32(va, c16, 0);
+    stage32(vb, c16 + 8, 4);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int32_t row0 = (int32_t)((int64_t)bkh * p.S + (int64_t)m * BM + (warp & 3) * 32);
+      tma_store_2d(is_dk ? &tm_dk : &tm_dv, 64 * (ew4 & 1), row0, slot);
+      bulk_commit_group();
+      bulk_wait_read_all();   // the shared-memory source must be read before the CTA exits
+    }
+    __syncwarp();
   }
 }
 
@@ -937,11 +953,12 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
                                const float* delta, void* dk, void* dv, float* xchg, int B, int Hq, int Hkv, int64_t S,
                                float scale, int* status, cudaStream_t st) {
   namespace K = tcbwd::dkdv;
-  CUtensorMap mq, mdo, mks, mvs;
+  CUtensorMap mq, mdo, mks, mvs, mdk, mdv;
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, K::BQ) ||
       !make_map_bf16_rows(&mdo, d_o, (uint64_t)B * Hq * S, K::BQ) ||
       !make_map_bf16_rows(&mks, ks, (uint64_t)B * Hkv * S, K::BM) ||
-      !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BM))
+      !make_map_bf16_rows(&mvs, vs, (uint64_t)B * Hkv * S, K::BM) ||
+      !make_map_bf16_rows(&mdk, dk, (uint64_t)B * Hkv * S, 32) || !make_map_bf16_rows(&mdv, dv, (uint64_t)B * Hkv * S, 32))
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
   const int nkt = (int)((S + K::BM - 1) / K::BM);
@@ -952,7 +969,8 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch_dependent(K::dkdv_tc_kernel, dim3((unsigned)grid), dim3(640), smem, st, (unsigned)cs, mq, mdo, mks, mvs, p);
+  e = launch_dependent(K::dkdv_tc_kernel, dim3((unsigned)grid), dim3(640), smem, st, (unsigned)cs, mq, mdo, mks, mvs, mdk,
+                       mdv, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
