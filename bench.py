@@ -214,16 +214,12 @@ def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3, causal=Fal
         x["q_prev"] = HI.prev_block_q(w, seed).to(dev)
     cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
     step = H.LayerStep(cfg, dev, causal_routing=causal)
-    calls = step.calls(x, stream.cuda_stream)
-    for _ in range(warmup):
-        for _, c in calls:
-            c()
+    graph = step.capture(x, warmup=warmup)            # replayed like the headline's step
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for e0, e1 in ev:
         flush_l2()
         e0.record(stream)
-        for _, c in calls:
-            c()
+        graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
     if H.read_status(step.ws) != 0:
@@ -397,14 +393,17 @@ def main():
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize(dev)
+    # the step captured once as a CUDA graph (the same kernels and dependent launches, without the
+    # per-call host work of the C ABI); the headline replays it
+    graph = step.capture(x)
+    torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        # the headline: K steps with events at the step boundaries only (an event between two
-        # kernels would cost its own time and keep the next kernel from starting early)
+        # the headline: K graph replays of the step, events at the step boundaries only (an event
+        # between two kernels would cost its own time and keep the next kernel from starting early)
         for i in range(K):
             flush_l2()
             ev_step[i][0].record(stream)
-            for _, c in calls:
-                c()
+            graph.replay()
             ev_step[i][1].record(stream)
         torch.cuda.synchronize(dev)
         # the per-kernel device times for the roofline: K more steps, an event after every kernel
@@ -510,15 +509,15 @@ def main():
         def time_e2e(in_names):
             sets = []
             for b in range(2):
-                xs = x if b == 0 else {k: (torch.empty_like(v) if k in in_names else v) for k, v in x.items()}
+                xs = x if b == 0 else {k: (v.clone() if k in in_names else v) for k, v in x.items()}
                 st_b = step if b == 0 else H.LayerStep(cfg, dev)
-                sets.append((xs, st_b, st_b.calls(xs, stream.cuda_stream)))
+                sets.append((xs, st_b, st_b.capture(xs)))
 
             def run_e2e(n):
                 ev = lambda: torch.cuda.Event()
                 copied, computed, drained = [None] * n, [None] * n, [None] * n
                 for i in range(n):
-                    xs, st_b, cl = sets[i % 2]
+                    xs, st_b, g_b = sets[i % 2]
                     with torch.cuda.stream(s_in):            # inputs of step i (set i % 2 free after step i-2)
                         if i >= 2:
                             s_in.wait_event(computed[i - 2])
@@ -528,8 +527,7 @@ def main():
                     stream.wait_event(copied[i])             # compute of step i
                     if i >= 2:
                         stream.wait_event(drained[i - 2])    # its output buffers were read out
-                    for _, c in cl:
-                        c()
+                    g_b.replay()
                     computed[i] = ev(); computed[i].record(stream)
                     with torch.cuda.stream(s_out):           # outputs of step i
                         s_out.wait_event(computed[i])
@@ -574,6 +572,9 @@ def main():
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
                 "config": _config(w, args), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": K * len(calls), "clocks": clk.summary(),
+                "step_launch": "one CUDA graph replay per step: the step's kernels and their dependent "
+                               "launches, captured once through the C ABI (the per-kernel pass launches "
+                               "them one by one)",
                 "kernels_per_step": names}
         if positions:
             line["segment_positions"] = positions

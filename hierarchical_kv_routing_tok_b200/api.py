@@ -241,6 +241,27 @@ class LayerStep:
         for _, call in self.calls(x):
             call()
 
+    def capture(self, x: dict, stream: "torch.cuda.Stream | None" = None, warmup: int = 2) -> "torch.cuda.CUDAGraph":
+        """The whole step on the buffers of ``x`` as a CUDA graph: ``graph.replay()`` runs the same
+        kernels (with their dependent launches) without the per-call host work of the C ABI (argument
+        checks, tensor maps, launches).  The step is first run ``warmup`` times on ``stream`` (a
+        side stream by default), then captured there; replay on any stream of the same device.
+        The buffers of ``x`` and of this step must stay alive and in place while the graph is used."""
+        dev = self.o.device
+        s = stream if stream is not None else torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        calls = self.calls(x, s.cuda_stream)
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                for _, call in calls:
+                    call()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _, call in calls:
+                call()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        return g
+
 
 class TieredLayerStep:
     """One layer step with the detached history K/V in pinned host memory (tiered storage,

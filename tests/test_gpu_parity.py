@@ -200,6 +200,30 @@ def test_repeat_runs_are_bitwise_identical(hga):
         assert torch.equal(a[k], b[k]), k
 
 
+@pytest.mark.parametrize("name", ["small_bf16", "tiny_f32"])
+def test_captured_step_replays_bitwise(hga, name):
+    """LayerStep.capture: a CUDA-graph replay of the whole step gives bitwise the outputs of the
+    step launched call by call, on new inputs copied into the captured buffers too."""
+    w = _wl(name)
+    x = {k: v.cuda() for k, v in HI.make_inputs(w, 0).items() if k != "needles"}
+    cfg = hga.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
+    step = hga.LayerStep(cfg)
+    outs = lambda: [t.clone() for t in (step.group_idx, step.o, step.lse, step.dq, step.dk, step.dv)]
+    g = step.capture(x)
+    for seed in (1, 2):
+        x2 = {k: v.cuda() for k, v in HI.make_inputs(w, seed).items() if k != "needles"}
+        for k in x:
+            x[k].copy_(x2[k])
+        g.replay()
+        torch.cuda.synchronize()
+        got = outs()
+        step(x)
+        torch.cuda.synchronize()
+        assert hga.read_status(step.ws) == 0
+        for a, b in zip(got, outs()):
+            assert torch.equal(a, b)
+
+
 def test_autograd_function_matches_oracle(hga, oracle):
     w = HI.WORKLOADS["small_bf16"]
     x = HI.make_inputs(w, 1)
