@@ -5,7 +5,8 @@ Workload (default ``ctx16k``): batch 1, 32 query / 8 KV heads, head dim 128, bf1
 accumulation; 14336 detached history tokens + 2048 active-segment tokens; chunk 64, group 8,
 query block 64; top-16 chunks then top-64 groups (512 routed tokens per block).  One step =
 the whole hot path on synthetic inputs already in HBM: key summaries, routing, forward,
-backward (6 kernel launches).  Metric: active-segment tokens per second, forward + backward.
+backward dQ, backward dK/dV (5 kernels, captured once as a CUDA graph and replayed per step).
+Metric: active-segment tokens per second, forward + backward.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
