@@ -256,7 +256,9 @@ class LayerStep:
                 for _, call in calls:
                     call()
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
+        # thread-local capture: CUDA calls of other host threads (a collective library's proxy
+        # thread, say) neither join nor invalidate it
+        with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
             for _, call in calls:
                 call()
         torch.cuda.current_stream(dev).wait_stream(s)
