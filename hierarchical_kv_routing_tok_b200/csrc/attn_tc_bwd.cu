@@ -525,9 +525,14 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
 #pragma unroll
       for (int e = 0; e < 32; e += 2)
         pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale);
-      uint4* d4 = reinterpret_cast<uint4*>(p.dq + row * kD + c0);
+      // the row's 32 columns (64 bytes, 64-byte aligned) as two 32-byte stores: whole sectors
+      __nv_bfloat16* dst = p.dq + row * kD + c0;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      for (int h = 0; h < 2; ++h)
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16 * h), "r"(pk[8 * h]),
+                     "r"(pk[8 * h + 1]), "r"(pk[8 * h + 2]), "r"(pk[8 * h + 3]), "r"(pk[8 * h + 4]), "r"(pk[8 * h + 5]),
+                     "r"(pk[8 * h + 6]), "r"(pk[8 * h + 7])
+                     : "memory");
       tc_fence_before();
     }
   }
