@@ -403,6 +403,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int c0 = 32 * w;
+    const bool dq_v8 = (reinterpret_cast<uintptr_t>(p.dq) & 31u) == 0;
     pdl_wait();                 // O and lse come from the forward kernel, the kernel before
     bool ok = true;
     int J = 0;
@@ -525,14 +526,22 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
 #pragma unroll
       for (int e = 0; e < 32; e += 2)
         pk[e >> 1] = pack_bf16(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale);
-      // the row's 32 columns (64 bytes, 64-byte aligned) as two 32-byte stores: whole sectors
+      // The row's 32 columns: 64 bytes at a 64-byte offset from dq.  With dq 32-byte aligned they
+      // go out as two 32-byte stores (whole sectors); the interface only promises 16-byte
+      // alignment, and then as four 16-byte stores.
       __nv_bfloat16* dst = p.dq + row * kD + c0;
+      if (dq_v8) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16 * h), "r"(pk[8 * h]),
-                     "r"(pk[8 * h + 1]), "r"(pk[8 * h + 2]), "r"(pk[8 * h + 3]), "r"(pk[8 * h + 4]), "r"(pk[8 * h + 5]),
-                     "r"(pk[8 * h + 6]), "r"(pk[8 * h + 7])
-                     : "memory");
+        for (int h = 0; h < 2; ++h)
+          asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16 * h), "r"(pk[8 * h]),
+                       "r"(pk[8 * h + 1]), "r"(pk[8 * h + 2]), "r"(pk[8 * h + 3]), "r"(pk[8 * h + 4]),
+                       "r"(pk[8 * h + 5]), "r"(pk[8 * h + 6]), "r"(pk[8 * h + 7])
+                       : "memory");
+      } else {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      }
       tc_fence_before();
     }
   }

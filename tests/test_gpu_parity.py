@@ -112,6 +112,35 @@ def test_attention_on_arbitrary_routing(hga, oracle):
     assert max(maxerr(g["o"], o), maxerr(g["dq"], dq), maxerr(g["dk"], dk), maxerr(g["dv"], dv)) <= 2e-2
 
 
+def test_bwd_outputs_only_16_byte_aligned(hga, oracle):
+    """The interface promises 16-byte alignment only: dQ, dK, dV placed 16 bytes past a 32-byte
+    boundary give the same bits as the aligned buffers (the dQ kernel stores 32-byte vectors only
+    into a 32-byte aligned dQ) and match the oracle."""
+    w = HI.WORKLOADS["small_bf16"]
+    x = HI.make_inputs(w, 2)
+    xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
+    cfg = hga.make_config(xd["q"], xd["k_hist"], w.top_chunks, w.top_groups)
+    step = hga.LayerStep(cfg)
+    step(xd)
+
+    def off16(like):
+        buf = torch.empty(like.numel() + 8, dtype=like.dtype, device=like.device)
+        t = buf[8:].view(like.shape)
+        assert t.data_ptr() % 32 == 16
+        return t
+
+    dq, dk, dv = off16(step.dq), off16(step.dk), off16(step.dv)
+    hga.attn_bwd(cfg, xd["q"], xd["k_hist"], xd["v_hist"], xd["k_seg"], xd["v_seg"], step.group_idx, step.o,
+                 step.lse, xd["d_o"], dq, dk, dv, step.ws)
+    torch.cuda.synchronize()
+    assert hga.read_status(step.ws) == 0
+    for got, ref in ((dq, step.dq), (dk, step.dk), (dv, step.dv)):
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    args = (x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], step.group_idx.cpu().numpy())
+    rdq, rdk, rdv = oracle.attn_bwd(*args, x["d_o"])
+    assert max(maxerr(dq.float().cpu(), rdq), maxerr(dk.float().cpu(), rdk), maxerr(dv.float().cpu(), rdv)) <= 2e-2
+
+
 # ----------------------------------------------------------------------------- ties
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_routing_ties_go_to_lower_index(hga, dtype):
