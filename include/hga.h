@@ -30,8 +30,9 @@
  * Conventions for every entry point
  *   - Memory: the caller allocates and owns every buffer, including the
  *     workspace.  All tensor pointers are DEVICE pointers, 16-byte aligned
- *     (int32 index arrays: 4-byte aligned),
- *     contiguous, head-major: q, o, d_o, dq: [B, Hq, S, D]; k/v history:
+ *     (int32 index arrays: 4-byte aligned; a 32-byte aligned dq lets the
+ *     bf16 backward store whole 32-byte sectors, which is faster, and gives
+ *     the same result), contiguous, head-major: q, o, d_o, dq: [B, Hq, S, D]; k/v history:
  *     [B, Hkv, H, D]; k/v segment, dk/dv segment: [B, Hkv, S, D].  Query head
  *     h uses KV head h / (Hq / Hkv).  Element type: float32 or bfloat16 as
  *     set by cfg->dtype (summaries, LSE are always float32; indices int32).
