@@ -186,6 +186,9 @@ EDGE_WORKLOADS = {
     "sink_gqa2_bf16": Workload("sink_gqa2_bf16", 1, 4, 2, 128, 1024, 448, 3, 20, "bf16", 1.0, n_sink=128),
     # eight query heads per KV head (two CTAs per query block), 5 query blocks, bf16
     "gqa8_bf16": Workload("gqa8_bf16", 1, 8, 1, 128, 512, 320, 4, 12, "bf16", 1.0),
+    # six query heads per KV head: three 2-head forward CTAs per query block, three head pairs per
+    # dQ unit list, three heads per paired dK/dV CTA; 7 query blocks, ragged routed tiles, bf16
+    "gqa6_bf16": Workload("gqa6_bf16", 1, 12, 2, 128, 1024, 448, 3, 20, "bf16", 1.0),
     # many (batch, KV head) units of short segments: as many dK/dV key tiles as SMs or more, so
     # every CTA sums all of its KV head's query heads alone; ragged 64-key last tile, bf16
     "wide_bf16": Workload("wide_bf16", 16, 16, 8, 128, 256, 192, 2, 8, "bf16", 1.0),
