@@ -164,3 +164,13 @@ def test_entry_points_reject_bad_pointers_before_launch(lib):
     with pytest.raises(C.HGAError) as e:
         C.route(bad, ok, ok, ok, ok, ok, ok)
     assert e.value.code == C.HGA_ERR_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU or library fallback: without libhga.so every call raises."""
+    monkeypatch.setattr(C, "LIB_PATH", os.path.join(tmp_path, "libhga.so"))
+    monkeypatch.setattr(C, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        C.load()
+    with pytest.raises(RuntimeError, match="missing"):
+        C.workspace_size(cfg())
