@@ -49,7 +49,13 @@ def _peaks():
 
 
 def work_model(w) -> dict:
-    """Algorithmic work of each kernel of one step (bytes or flops per launch)."""
+    """Algorithmic work of each kernel of one step (bytes or flops per launch).
+
+    The backward is booked at the method's own work (FlashAttention-form backward over the routed
+    and local pairs, no history gradient): S and dP of a local pair count once, charged to the dQ
+    kernel (S, dP, dQ over routed + local pairs); the dK/dV kernel is charged its dK and dV products
+    only.  Its recomputation of S^T and dP^T is real work but not the method's: ``executed_flops``
+    lists it."""
     B, Hq, Hkv, D, H, S = w.B, w.Hq, w.Hkv, w.D, w.hist_len, w.seg_len
     esz = 2 if w.dtype == "bf16" else 4
     routed_pairs = B * Hq * S * 8 * w.top_groups            # (query, routed key) pairs
@@ -60,9 +66,24 @@ def work_model(w) -> dict:
         "route": ("hbm", B * Hq * S * D * esz + B * Hkv * (nch + ngr) * D * 4
                   + B * Hkv * nblk * (w.top_chunks + w.top_groups) * 4),
         "attn_fwd": ("tensor", 4 * D * (routed_pairs + local_pairs)),
-        "bwd_dkdv": ("tensor", 8 * D * local_pairs),
         "bwd_dq": ("tensor", 6 * D * (routed_pairs + local_pairs)),
+        "bwd_dkdv": ("tensor", 4 * D * local_pairs),
     }
+
+
+def executed_flops(w) -> dict:
+    """Flops the tensor-core kernels issue, recomputation included: the dK/dV kernel recomputes
+    S^T = K Q^T and dP^T = V dO^T over the local pairs (the dQ kernel already formed S and dP)."""
+    local_pairs = w.B * w.Hq * w.seg_len * (w.seg_len + 1) // 2
+    wm = work_model(w)
+    return {"attn_fwd": wm["attn_fwd"][1], "bwd_dq": wm["bwd_dq"][1], "bwd_dkdv": 8 * w.D * local_pairs}
+
+
+def method_flops(w) -> int:
+    """The method's flops per step: forward 4 D (routed + local pairs), backward 6 D (routed +
+    local) for S, dP, dQ plus 4 D local for dK, dV (no history gradient)."""
+    wm = work_model(w)
+    return wm["attn_fwd"][1] + wm["bwd_dq"][1] + wm["bwd_dkdv"][1]
 
 
 class ClockSampler:
@@ -170,51 +191,119 @@ def all_max(v: float, world: int, device) -> float:
     return float(t.item())
 
 
-def oracle_slice_pass(w, x) -> float:
-    """The CPU oracle over KV head 0 of batch 0 (its G query heads, every block): summaries,
-    routing, forward and backward.  Returns seconds."""
+def host_cores() -> int:
+    """Cores this process may run on (affinity / cgroup aware where the OS tells)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_layer_pass(w, x, workers: int, n_slices: int | None = None) -> float:
+    """The CPU oracle, as it stands, over the first n_slices (batch, KV head) slices of the layer
+    (all of them by default), on `workers` host threads: summaries and float32-decision routing per
+    slice, then the float64 forward and dQ of every (slice, 64-query block) unit and the dK/dV of
+    every slice, all as concurrent tasks (the oracle's C calls release the GIL).  A slice -- its G
+    query heads with their history, segment K/V and routing -- is independent of every other slice.
+    Returns seconds (wall clock)."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
     from oracle import oracle as O
-    G = w.Hq // w.Hkv
-    s = {k: (v[:1, :G] if k in ("q", "d_o") else v[:1, :1]) for k, v in x.items() if k != "needles"}
     t0 = time.perf_counter()
-    r = O.route_from_inputs(s["q"], s["k_hist"], 1, w.top_chunks, w.top_groups, prec=32)
-    O.attn_fwd(s["q"], s["k_hist"], s["v_hist"], s["k_seg"], s["v_seg"], r["group_idx"])
-    O.attn_bwd(s["q"], s["k_hist"], s["v_hist"], s["k_seg"], s["v_seg"], r["group_idx"], s["d_o"])
+    f64 = {k: v.double().numpy() for k, v in x.items() if k != "needles"}
+    G, S, nblk = w.Hq // w.Hkv, w.seg_len, w.seg_len // 64
+    slices = [(b, kh) for b in range(w.B) for kh in range(w.Hkv)][:n_slices]
+
+    def sl(b, kh):
+        hs = slice(kh * G, (kh + 1) * G)
+        return (f64["q"][b:b + 1, hs], f64["k_hist"][b:b + 1, kh:kh + 1], f64["v_hist"][b:b + 1, kh:kh + 1],
+                f64["k_seg"][b:b + 1, kh:kh + 1], f64["v_seg"][b:b + 1, kh:kh + 1]), f64["d_o"][b:b + 1, hs]
+
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        def route(b, kh):
+            (q, kh_, *_), _ = sl(b, kh)
+            return O.route_from_inputs(q, kh_, 1, w.top_chunks, w.top_groups, prec=32)["group_idx"]
+        gi = dict(zip(slices, ex.map(lambda j: route(*j), slices)))
+        tasks = []
+        for b, kh in slices:                     # dK/dV of a slice: the longest tasks, queued first
+            args, do = sl(b, kh)
+            tasks.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=np.array([0]),
+                                   keys=np.arange(S)))
+        for b, kh in slices:
+            args, do = sl(b, kh)
+            for n in range(nblk):                # forward and dQ of the block's G x 64 rows
+                rows = np.array([hh * S + n * 64 + t for hh in range(G) for t in range(64)], dtype=np.int64)
+                tasks.append(ex.submit(O.attn_fwd, *args, gi[(b, kh)], rows=rows))
+                tasks.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=rows, keys=np.array([S - 1])))
+        for t in tasks:
+            t.result()
     return time.perf_counter() - t0
 
 
-ORACLE_SAMPLE = ("one (batch, KV head) slice of the layer -- its 4 query heads over all 32 query blocks: "
-                 "summaries, routing, forward and backward in the float64 C oracle on one host thread; "
-                 "the layer is B*Hkv such independent slices of equal work, so tokens/s = B*S / (B*Hkv * t_slice)")
+ORACLE_SAMPLE = ("the CPU oracle as it stands (plain C, float32-decision routing, float64 attention) over {what}: "
+                 "summaries and routing per (batch, KV head), forward and dQ per (batch, KV head, 64-query block) "
+                 "unit, dK/dV per (batch, KV head), as concurrent tasks on {workers} host threads; wall clock")
+
+
+def _oracle_baseline(w, x, warm: bool = True) -> dict:
+    """The oracle over the whole layer on all host cores; when that takes longer than ~8 s, over the
+    first (batch, KV head) slices only, as many as fit ~8 s, scaled to the whole layer's tokens."""
+    workers = host_cores()
+    total = w.B * w.Hkv
+    n = total
+    if warm:
+        t1 = oracle_layer_pass(w, x, workers, n)
+        if t1 > 8.0:
+            n = max(1, min(total, int(total * 8.0 / t1)))
+    t = oracle_layer_pass(w, x, workers, n)
+    what = "the whole layer" if n == total else f"{n} of the layer's {total} (batch, KV head) slices"
+    tokens = w.B * w.seg_len * n / total
+    return {"value": tokens / t, "unit": "tokens/s", "cores": workers,
+            "kind": "oracle", "sample": ORACLE_SAMPLE.format(what=what, workers=workers), "seconds": t,
+            "slices": n, "host_cores": workers}
 
 
 def run_reference(args, w, world, rank):
+    """The reference arm: the CPU oracle as it stands, one layer pass (or the bounded slice sample
+    of _oracle_baseline) per step, on the host cores; rank 0 only."""
     if rank != 0:
         return
     x = HI.make_inputs(w, args.seed)
-    for _ in range(args.warmup):
-        oracle_slice_pass(w, x)
-    ts = [oracle_slice_pass(w, x) for _ in range(args.steps)]
-    t_step = statistics.mean(ts) * w.B * w.Hkv           # the whole layer
-    value = w.B * w.seg_len / t_step
+    workers = host_cores()
+    total = w.B * w.Hkv
+    n = total
+    for i in range(args.warmup):
+        t1 = oracle_layer_pass(w, x, workers, n)
+        if i == 0 and t1 > 8.0:                  # keep the whole run within a few minutes
+            n = max(1, min(total, int(total * 8.0 / t1)))
+    ts = [oracle_layer_pass(w, x, workers, n) for _ in range(args.steps)]
+    t_step = statistics.mean(ts)
+    tokens = w.B * w.seg_len * n / total
+    value = tokens / t_step
+    what = "the whole layer" if n == total else f"{n} of the layer's {total} (batch, KV head) slices"
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": _config(w, args), "gpu_launches": 0,
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": ORACLE_SAMPLE},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                             "sample": ORACLE_SAMPLE.format(what=what, workers=workers)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3, causal=False) -> float:
+def _time_layer(H, w, seed, dev, stream, flush_l2, steps=5, warmup=3, causal=False, summaries_from=None) -> float:
     """Mean device time (ms) of one whole layer step of workload w, L2 flushed before each step
-    (causal: with the strictly causal routing, the previous segment's last block as q_prev)."""
+    (causal: with the strictly causal routing, the previous segment's last block as q_prev;
+    summaries_from: the step computes the summaries of history tokens [summaries_from, H) only)."""
     x = {k: v.to(dev) for k, v in HI.make_inputs(w, seed).items() if k != "needles"}
     if causal:
         x["q_prev"] = HI.prev_block_q(w, seed).to(dev)
     cfg = H.make_config(x["q"], x["k_hist"], w.top_chunks, w.top_groups)
-    step = H.LayerStep(cfg, dev, causal_routing=causal)
+    step = H.LayerStep(cfg, dev, causal_routing=causal, summaries_from=summaries_from)
+    if summaries_from is not None:
+        step.build_all_summaries(x)
     graph = step.capture(x, warmup=warmup)            # replayed like the headline's step
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for e0, e1 in ev:
@@ -446,6 +535,16 @@ def main():
             budgets[f"top_chunks_{pw.top_chunks}_top_groups_{pw.top_groups}"] = {
                 "ms_per_step": ms, "tokens_per_s": pw.B * pw.seg_len * world / (ms * 1e-3)}
 
+    # the same step with the summaries built incrementally: only the 2048 tokens of the segment that
+    # closed last are summarised (the rest of the history's summaries are kept from earlier steps)
+    incremental = None
+    if w.hist_len >= w.seg_len and not args.no_positions:
+        ms = all_max(_time_layer(H, w, args.seed + rank, dev, stream, flush_l2,
+                                 summaries_from=w.hist_len - w.seg_len), world, dev)
+        incremental = {"ms_per_step": ms, "tokens_per_s": w.B * w.seg_len * world / (ms * 1e-3),
+                       "summaries": f"history tokens [{w.hist_len - w.seg_len}, {w.hist_len}) only "
+                                    "(hga_append_summaries of the segment that closed last)"}
+
     # strictly causal routing (block n routed with block n-1's query): same kernels, other routing
     causal = None
     if w.name == "ctx16k" and not args.no_positions:
@@ -482,14 +581,26 @@ def main():
             traffic = tr["dram_bytes_per_launch"]
     except (OSError, ValueError):
         pass
+    mflops = method_flops(w)
+    ex = executed_flops(w)
+    per_us = {n: 1e3 * sum(v) / K for n, v in kern_ms.items()}
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": dom, "peak_source": f"{pk['src']} (burst)",
-                "per_kernel_us": {n: 1e3 * sum(v) / K for n, v in kern_ms.items()},
+                "per_kernel_us": per_us,
                 "per_kernel_pass": f"a second pass of {K} steps, L2 flushed alike, with an event after every kernel "
                                    f"({t_step_kernel_events:.4f} ms per step with those events)",
                 "per_kernel_frac": {n: (wm[n][1] / (sum(kern_ms[n]) / K * 1e-3)
                                         / ((pk["bf16"] * 1e12) if wm[n][0] == "tensor" else (pk["hbm"] * 1e9)))
-                                    for n in names}}
+                                    for n in names},
+                "per_kernel_executed_frac": {n: ex[n] / (per_us[n] * 1e-6) / (pk["bf16"] * 1e12) for n in ex},
+                "work_booking": "backward at the method's work: S, dP, dQ over routed + local pairs charged to "
+                                "bwd_dq, dK and dV over local pairs to bwd_dkdv (its S^T, dP^T recomputation "
+                                "is in per_kernel_executed_frac only)"}
+    # the whole step against the method's flops (forward + backward, S and dP counted once)
+    method = {"gflop_per_step": mflops / 1e9, "achieved_tflops": mflops / t_step / 1e12,
+              "frac_burst": mflops / t_step / (pk["bf16"] * 1e12),
+              "frac_sustained": mflops / t_step / (pk["bf16_sustained"] * 1e12),
+              "peaks": f"{pk['src']}: {pk['bf16']} TFLOP/s burst, {pk['bf16_sustained']} sustained"}
 
     # end to end through the public API with pinned host buffers: every step copies its inputs in
     # and its outputs out.  Steps are pipelined the way a stream of steps would run: two sets of
@@ -563,20 +674,21 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_slice = oracle_slice_pass(w, x_cpu)
-        cpu = {"value": w.B * w.seg_len / (t_slice * w.B * w.Hkv), "unit": "tokens/s", "cores": 1,
-               "kind": "oracle", "sample": ORACLE_SAMPLE, "slice_seconds": t_slice}
+        cpu = _oracle_baseline(w, x_cpu, warm=False)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-                "config": _config(w, args), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "config": _config(w, args), "roofline": roofline, "method_frac": method["frac_burst"],
+                "method_roofline": method, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": K * len(calls), "clocks": clk.summary(),
                 "step_launch": "one CUDA graph replay per step: the step's kernels and their dependent "
                                "launches, captured once through the C ABI (the per-kernel pass launches "
                                "them one by one)",
                 "kernels_per_step": names}
+        if incremental:
+            line["incremental_summaries"] = incremental
         if positions:
             line["segment_positions"] = positions
         if budgets:

@@ -38,15 +38,17 @@ def _need(t: torch.Tensor, name: str, shape, dtype) -> None:
 
 
 def make_config(q: torch.Tensor, k_hist: torch.Tensor, top_chunks: int, top_groups: int,
-                softmax_scale: float | None = None, n_sink_tokens: int = 0) -> C.HGAConfig:
+                softmax_scale: float | None = None, n_sink_tokens: int = 0, wait_limit_ns: int = 0) -> C.HGAConfig:
     """Configuration from q [B,Hq,S,D] and k_hist [B,Hkv,H,D]; ``n_sink_tokens`` (a multiple of 64)
-    history tokens at the start form the sink window every query attends."""
+    history tokens at the start form the sink window every query attends; ``wait_limit_ns`` bounds
+    the tensor-core kernels' on-chip waits (0: 2 s)."""
     if q.dtype not in _DT:
         raise ValueError(f"unsupported dtype {q.dtype}")
     B, Hq, S, D = q.shape
     Hkv, H = k_hist.shape[1], k_hist.shape[2]
     return C.make_config(B, Hq, Hkv, H, S, top_chunks, top_groups, dtype=_DT[q.dtype], D=D,
-                         softmax_scale=float(softmax_scale or 0.0), n_sink_tokens=n_sink_tokens)
+                         softmax_scale=float(softmax_scale or 0.0), n_sink_tokens=n_sink_tokens,
+                         wait_limit_ns=wait_limit_ns)
 
 
 def _tdtype(cfg) -> torch.dtype:
@@ -190,9 +192,18 @@ class LayerStep:
     """One full pass of the hot path (summaries, routing, forward, backward) over preallocated
     buffers, for a fixed configuration.  Used by the benchmark and the smoke check."""
 
-    def __init__(self, cfg, device="cuda", causal_routing: bool = False):
+    def __init__(self, cfg, device="cuda", causal_routing: bool = False, summaries_from: int | None = None):
+        """summaries_from: None rebuilds the summaries of the whole history every step; a token
+        index (a multiple of the chunk) makes the step compute only those of history tokens
+        [summaries_from, H) -- the segment appended last -- with ``hga_append_summaries``, the
+        summaries of the earlier tokens being already in ``group_sum`` / ``chunk_sum`` (run
+        ``build_all_summaries`` once first)."""
         self.cfg = cfg
         self.causal_routing = causal_routing
+        if summaries_from is not None and not (0 <= summaries_from <= cfg.hist_len
+                                               and summaries_from % cfg.chunk == 0):
+            raise ValueError(f"summaries_from={summaries_from}: a multiple of {cfg.chunk} in [0, {cfg.hist_len}]")
+        self.summaries_from = summaries_from
         dev = torch.device(device)
         B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
         dt = _tdtype(cfg)
@@ -208,16 +219,19 @@ class LayerStep:
         self.dk = torch.empty(B, Hkv, S, D, dtype=dt, device=dev)
         self.dv = torch.empty(B, Hkv, S, D, dtype=dt, device=dev)
 
-    def calls(self, x: dict, stream: int | None = None):
+    def calls(self, x: dict, stream: int | None = None, cfg: "C.HGAConfig | None" = None):
         """The step as a list of (kernel name, zero-argument C-ABI call), one kernel each, in order.
-        Pointers are bound once so the timed loop does no tensor bookkeeping."""
-        cfg, ws = self.cfg, self.ws.data_ptr()
+        Pointers are bound once so the timed loop does no tensor bookkeeping.  ``cfg`` overrides the
+        step's configuration (same shapes; e.g. another wait limit)."""
+        cfg, ws = (self.cfg if cfg is None else cfg), self.ws.data_ptr()
         st = torch.cuda.current_stream(self.o.device).cuda_stream if stream is None else stream
         p = {k: v.data_ptr() for k, v in x.items() if isinstance(v, torch.Tensor) and v.is_cuda}
         gs, cs, ci, gi = (t.data_ptr() for t in (self.group_sum, self.chunk_sum, self.chunk_idx, self.group_idx))
         o, lse, dq, dk, dv = (t.data_ptr() for t in (self.o, self.lse, self.dq, self.dk, self.dv))
+        first = self.summaries_from
         return [
-            ("summaries", lambda: C.build_summaries(cfg, p["k_hist"], gs, cs, ws, st)),
+            ("summaries", (lambda: C.build_summaries(cfg, p["k_hist"], gs, cs, ws, st)) if first is None
+             else (lambda: C.append_summaries(cfg, p["k_hist"], gs, cs, first, ws, st))),
             ("route", (lambda: C.route_causal(cfg, p["q"], p.get("q_prev"), gs, cs, ci, gi, ws, st))
              if self.causal_routing else (lambda: C.route(cfg, p["q"], gs, cs, ci, gi, ws, st))),
             ("attn_fwd", lambda: C.attn_fwd(cfg, p["q"], p["k_hist"], p["v_hist"], p["k_seg"], p["v_seg"], gi, o,
@@ -228,6 +242,12 @@ class LayerStep:
             ("bwd_dkdv", lambda: C.attn_bwd_dkdv(cfg, p["q"], p["k_seg"], p["v_seg"], lse, p["d_o"], dk, dv, ws,
                                                  st)),
         ]
+
+    def build_all_summaries(self, x: dict) -> None:
+        """Summaries of the whole history of x into this step's buffers (the state an appending
+        step starts from)."""
+        C.build_summaries(self.cfg, x["k_hist"].data_ptr(), self.group_sum.data_ptr(), self.chunk_sum.data_ptr(),
+                          self.ws.data_ptr(), torch.cuda.current_stream(self.o.device).cuda_stream)
 
     def forward(self, x: dict) -> None:
         for _, call in self.calls(x)[:3]:
@@ -288,7 +308,8 @@ class TieredLayerStep:
         self.cfg, self.dev = cfg, dev
         self.ccfg = C.tier_cache_config(cfg)
         self.cfg1 = C.make_config(1, Hq, Hkv, H, S, cfg.top_chunks, cfg.top_groups, dtype=cfg.dtype, D=D,
-                                  softmax_scale=cfg.softmax_scale, n_sink_tokens=cfg.n_sink_tokens)
+                                  softmax_scale=cfg.softmax_scale, n_sink_tokens=cfg.n_sink_tokens,
+                                  wait_limit_ns=cfg.wait_limit_ns)
         self.ccfg1 = C.tier_cache_config(self.cfg1)
         self.cap = self.ccfg.hist_len // cfg.group
         nblk = S // cfg.qblock

@@ -14,12 +14,21 @@ def test_work_model_16k():
     # forward: S = Q K^T and O = P V, 2 flops per multiply-add each
     assert wm["attn_fwd"] == ("tensor", 4 * D * (routed + local))
     assert abs(wm["attn_fwd"][1] / 1e9 - 51.56) < 0.01
-    # dK/dV kernel: S^T, dP^T, dV, dK over the local pairs only (no history gradient)
-    assert wm["bwd_dkdv"] == ("tensor", 8 * D * local)
-    assert abs(wm["bwd_dkdv"][1] / 1e9 - 68.75) < 0.01
-    # dQ kernel: S, dP, dQ over routed and local pairs
+    # backward at the method's work (the FlashAttention-form backward over the same key sets, no
+    # history gradient): S, dP and dQ over routed and local pairs, charged to the dQ kernel ...
     assert wm["bwd_dq"] == ("tensor", 6 * D * (routed + local))
     assert abs(wm["bwd_dq"][1] / 1e9 - 77.34) < 0.01
+    # ... and dV = P^T dO, dK = dS^T Q over the local pairs, charged to the dK/dV kernel; S and dP of
+    # a local pair are not booked twice
+    assert wm["bwd_dkdv"] == ("tensor", 4 * D * local)
+    assert abs(wm["bwd_dkdv"][1] / 1e9 - 34.37) < 0.01
+    # the backward as a whole: 25.8 GFLOP routed (1.5 x the forward's 17.2) + 85.9 local (2.5 x 34.4)
+    bwd = wm["bwd_dq"][1] + wm["bwd_dkdv"][1]
+    assert bwd == 6 * D * routed + 10 * D * local
+    assert abs(bwd / 1e9 - 111.7) < 0.05
+    assert abs(bench.method_flops(HI.WORKLOADS["ctx16k"]) / 1e9 - 163.3) < 0.05
+    # what the dK/dV kernel executes: it recomputes S^T and dP^T
+    assert bench.executed_flops(HI.WORKLOADS["ctx16k"])["bwd_dkdv"] == 8 * D * local
     # summaries: read the bf16 history keys once, write float32 group and chunk means
     assert wm["summaries"] == ("hbm", Hkv * H * D * 2 + Hkv * (H // 8 + H // 64) * D * 4)
     # routing: read the bf16 queries and both float32 summary tables, write both index lists
