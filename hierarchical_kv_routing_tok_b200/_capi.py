@@ -29,7 +29,7 @@ HGA_BF16 = 1
 EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_append_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
            "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
-           "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
+           "hga_noalloc_read_status", "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
            "hga_read_status", "hga_strerror", "hga_version")
 
 
@@ -40,7 +40,7 @@ class HGAConfig(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("group", ctypes.c_int32), ("qblock", ctypes.c_int32),
                 ("top_chunks", ctypes.c_int32), ("top_groups", ctypes.c_int32),
                 ("n_sink_tokens", ctypes.c_int32), ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
-                ("hist_capacity", ctypes.c_int64)]
+                ("hist_capacity", ctypes.c_int64), ("wait_limit_ns", ctypes.c_int64)]
 
     def __repr__(self):
         return "HGAConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -77,6 +77,7 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd_dkdv": [C, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_dq": [C, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_attn_bwd_noalloc": [C, P, P, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_noalloc_read_status": [P, ctypes.POINTER(ctypes.c_int32)],
         "hga_tier_cache_config": [C, C],
         "hga_tier_plan": [C, P, P, P, P, P, P],
         "hga_tier_gather": [C, P, P, P, P, P, P, P],
@@ -108,9 +109,10 @@ def _call(name: str, *args) -> None:
 
 def make_config(B: int, Hq: int, Hkv: int, hist_len: int, seg_len: int, top_chunks: int, top_groups: int,
                 dtype: int = HGA_BF16, D: int = 128, softmax_scale: float = 0.0, chunk: int = 64,
-                group: int = 8, qblock: int = 64, n_sink_tokens: int = 0, hist_capacity: int = 0) -> HGAConfig:
+                group: int = 8, qblock: int = 64, n_sink_tokens: int = 0, hist_capacity: int = 0,
+                wait_limit_ns: int = 0) -> HGAConfig:
     return HGAConfig(B, Hq, Hkv, D, hist_len, seg_len, chunk, group, qblock, top_chunks, top_groups,
-                     n_sink_tokens, dtype, softmax_scale, hist_capacity)
+                     n_sink_tokens, dtype, softmax_scale, hist_capacity, wait_limit_ns)
 
 
 def workspace_size(cfg: HGAConfig) -> int:
@@ -169,6 +171,13 @@ def attn_bwd_noalloc(cfg, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_
     library's fixed per-device scratch is used instead; overlapping calls race)."""
     _call("hga_attn_bwd_noalloc", ctypes.byref(cfg), q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, d_o,
           dq, dk_seg, dv_seg, stream)
+
+
+def noalloc_read_status(stream=0) -> int:
+    """Device-side status of the last attn_bwd_noalloc call on the current device (read and cleared)."""
+    out = ctypes.c_int32(0)
+    _call("hga_noalloc_read_status", stream, ctypes.byref(out))
+    return int(out.value)
 
 
 def tier_cache_config(cfg) -> HGAConfig:

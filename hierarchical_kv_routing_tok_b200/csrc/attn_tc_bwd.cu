@@ -64,6 +64,7 @@ struct Params {
   float* delta;             // delta of this kernel's rows, written for the dK/dV kernel
   __nv_bfloat16* dq;
   int* status;
+  uint64_t wait_ns;     // limit of every bounded mbarrier wait (drains excepted)
 };
 
 struct Smem {
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       read_idx(k + 1, nxt);
       if (k > 0) {
         int okq = 1;
-        if (lane == 0) okq = mbar_wait(qdo_issued, k & 1, abort_flag, p.status);
+        if (lane == 0) okq = mbar_wait(qdo_issued, k & 1, abort_flag, p.status, p.wait_ns);
         ok = __shfl_sync(0xffffffffu, okq, 0) != 0;
         if (!ok) break;
       }
@@ -224,8 +225,8 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         const int ks = J % KS, vs = J % VS;
         int okk = 1;
         if (lane == 0) {
-          okk = is_v ? mbar_wait(v_empty(vs), ((J / VS) & 1) ^ 1, abort_flag, p.status)
-                     : mbar_wait(k_empty(ks), ((J / KS) & 1) ^ 1, abort_flag, p.status);
+          okk = is_v ? mbar_wait(v_empty(vs), ((J / VS) & 1) ^ 1, abort_flag, p.status, p.wait_ns)
+                     : mbar_wait(k_empty(ks), ((J / KS) & 1) ^ 1, abort_flag, p.status, p.wait_ns);
           if (okk) mbar_arrive_expect_tx(kv_full(ks), kKVTile);
         }
         ok = __shfl_sync(0xffffffffu, okk, 0) != 0;
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       for (int k = 0;; ++k) {
         const int u = unit_of_cta(k, cta, G);
         if (u >= n_units) break;
-        if (k > 0 && !mbar_wait(qdo_empty, (k - 1) & 1, abort_flag, p.status)) break;
+        if (k > 0 && !mbar_wait(qdo_empty, (k - 1) & 1, abort_flag, p.status, p.wait_ns)) break;
         const Unit x = decode_unit(u, p, n_rt);
         mbar_arrive_expect_tx(qdo_full, 2 * kQTile);
         for (int jh = 0; jh < 2; ++jh) {
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     int u = unit_of_cta(0, cta, G);
     if (u < n_units) {
       x = decode_unit(u, p, n_rt);
-      ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status);
+      ok = mbar_wait_w(qdo_full, 0, abort_flag, p.status, p.wait_ns) && mbar_wait_w(kv_full(0), 0, abort_flag, p.status, p.wait_ns);
       if (ok) {
         issue_s(0, 0 < n_rt);
         issue_dp(0, 0 < n_rt);
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         const int jn = last ? 0 : j + 1;          // the next tile's index in its unit
         const int Tn = last ? xn.T : x.T;
         auto finish_tile = [&]() {                // dQ (+)= dS(J) K(J), then K(J) is free
-          ok = mbar_wait_w(ds_full(J & 1), (J >> 1) & 1, abort_flag, p.status);
+          ok = mbar_wait_w(ds_full(J & 1), (J >> 1) & 1, abort_flag, p.status, p.wait_ns);
           if (!ok) return;
           tc_fence_after();
           issue_dq(J, j < n_rt, j == 0);
@@ -373,12 +374,12 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
           mma_commit_w(dq_ready);
         }
         if (next) {
-          if (last) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status);
-          if (ok) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status);
+          if (last) ok = mbar_wait_w(qdo_full, (k + 1) & 1, abort_flag, p.status, p.wait_ns);
+          if (ok) ok = mbar_wait_w(kv_full((J + 1) % KS), ((J + 1) / KS) & 1, abort_flag, p.status, p.wait_ns);
           if (!ok) break;
           issue_s(J + 1, jn < n_rt);
         }
-        ok = mbar_wait_w(dp_free, J & 1, abort_flag, p.status);
+        ok = mbar_wait_w(dp_free, J & 1, abort_flag, p.status, p.wait_ns);
         if (!ok) break;
         if (next) {
           issue_dp(J + 1, jn < n_rt);
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) ov[c] = orow[c];
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(qdo_full, k & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(qdo_full, k & 1, abort_flag, p.status, p.wait_ns));
       if (!ok) break;
       float part;
       {
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(delta_bar);
-      ok = __all_sync(0xffffffffu, mbar_wait(delta_bar, k & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(delta_bar, k & 1, abort_flag, p.status, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
       float dl;
@@ -473,7 +474,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
       for (int j = 0; j < x.T; ++j, ++J) {
         // P of this warpgroup's 32 keys from S (masked keys -> 0) while dP is still in the tensor
         // pipe; then dP, which frees the dP columns for the next tile's dP
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(J & 1), (J >> 1) & 1, abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(J & 1), (J >> 1) & 1, abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + (J & 1) * 128 + c0;
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
             for (int e = 0; e < 32; ++e) pr[e] = (c0 + e < nvalid) ? pexp(e) : 0.f;
           }
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, J & 1, abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, J & 1, abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         uint32_t dv[32], pk[16];
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(ds_full(J & 1));
       }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_ready, k & 1, abort_flag, p.status));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_ready, k & 1, abort_flag, p.status, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
       uint32_t v[32], pk[16];
@@ -551,6 +552,7 @@ __global__ void __launch_bounds__(128 + 32 * kEWWarps, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  pdl_wait();   // completes only after the kernel before, even when it gave up early
 }
 
 }  // namespace dq
@@ -580,6 +582,7 @@ struct Params {
   __nv_bfloat16* dv;
   float* xchg;          // cs == 2: per cluster, two [32 chunks of 4 columns x 2][64 rows] float32 areas
   int* status;
+  uint64_t wait_ns;     // limit of every bounded mbarrier wait (drains excepted)
 };
 
 struct Smem {
@@ -676,7 +679,7 @@ __global__ void __launch_bounds__(640, 1)
       for (int j = 0; j < NJ; ++j) {
         const int s = j % NS;
         const int t = j / Tq, i = j - t * Tq;
-        if (!mbar_wait(q_empty(s), ((j / NS) & 1) ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(q_empty(s), ((j / NS) & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
         mbar_arrive_expect_tx(q_full(s), 2 * kQTileB + kStatBytes);
         const int64_t row = ((int64_t)b * p.Hq + head0 + t) * p.S + (int64_t)(n0 + i) * BQ;
         tma_load_2d(sbase + L::kQ + s * kQTileB, &tm_q, 0, (int32_t)row, q_full(s));
@@ -732,9 +735,9 @@ __global__ void __launch_bounds__(640, 1)
           mma_ts_w(tmem + 384, tmem + x * 128 + 64 + acol, b2[ks], idesc_g, (j > 0 || ks > 0));
         }
       };
-      bool ok = mbar_wait_w(kv_full, 0, abort_flag, p.status);
+      bool ok = mbar_wait_w(kv_full, 0, abort_flag, p.status, p.wait_ns);
       for (int j = 0; ok && j < 2 && j < NJ; ++j) {
-        ok = mbar_wait_w(q_full(j % NS), (j / NS) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(q_full(j % NS), (j / NS) & 1, abort_flag, p.status, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         issue_sd(j, j & 1);
@@ -742,13 +745,13 @@ __global__ void __launch_bounds__(640, 1)
       }
       for (int j = 0; ok && j < NJ; ++j) {
         const int x = j & 1;
-        ok = mbar_wait_w(pd_full(x), (j >> 1) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(pd_full(x), (j >> 1) & 1, abort_flag, p.status, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         issue_grad(j, x);
         mma_commit_w(q_empty(j % NS));
         if (j + 2 < NJ) {
-          ok = mbar_wait_w(q_full((j + 2) % NS), ((j + 2) / NS) & 1, abort_flag, p.status);
+          ok = mbar_wait_w(q_full((j + 2) % NS), ((j + 2) / NS) & 1, abort_flag, p.status, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_sd(j + 2, x);
@@ -775,8 +778,8 @@ __global__ void __launch_bounds__(640, 1)
     for (int j = x; j < NJ; j += 2) {
       const int s = j % NS;
       const int i = j % Tq;
-      ok = mbar_wait(sd_full(x), (j >> 1) & 1, abort_flag, p.status);
-      if (ok) ok = mbar_wait(q_full(s), (j / NS) & 1, abort_flag, p.status);   // stats landed
+      ok = mbar_wait(sd_full(x), (j >> 1) & 1, abort_flag, p.status, p.wait_ns);
+      if (ok) ok = mbar_wait(q_full(s), (j / NS) & 1, abort_flag, p.status, p.wait_ns);   // stats landed
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -818,7 +821,7 @@ __global__ void __launch_bounds__(640, 1)
     // ---- epilogue: warpgroups 0,1 own dV columns 0-63 / 64-127, warpgroups 2,3 the same of dK;
     // after `done` every MMA has completed and each thread takes its 64 columns of the float32 sums
     // over this CTA's heads into registers.
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status, p.wait_ns));
     if (ok) {
       tc_fence_after();
       const uint32_t tacc = tmem + lane_off + (w4 >= 2 ? 384 : 256) + 64 * (w4 & 1);
@@ -904,6 +907,7 @@ __global__ void __launch_bounds__(640, 1)
     }
     __syncwarp();
   }
+  pdl_wait();   // completes only after the kernel before, even when it gave up early
 }
 
 }  // namespace dkdv
@@ -913,7 +917,7 @@ __global__ void __launch_bounds__(640, 1)
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* o, const void* d_o, float* delta,
                              void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg,
-                             float scale, int* status, cudaStream_t st) {
+                             float scale, int* status, uint64_t wait_ns, cudaStream_t st) {
   namespace K = tcbwd::dq;
   CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
   // with no history the history maps are never used: map the segment instead (maps need rows > 0)
@@ -927,7 +931,7 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, cons
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
   K::Params p{B, Hq, Hkv, G, kg, (int)(S / kQBlock), nsg, H, S, Hs, scale * tcbwd::kLog2e, scale, gi, lse,
-              static_cast<const __nv_bfloat16*>(o), delta, static_cast<__nv_bfloat16*>(dq), status};
+              static_cast<const __nv_bfloat16*>(o), delta, static_cast<__nv_bfloat16*>(dq), status, wait_ns};
   // persistent: one CTA per SM (or per unit, when there are fewer units than SMs)
   const int64_t units = (int64_t)B * Hkv * p.nblk * (G / 2);
   int dev = 0, sms = 0;
@@ -965,7 +969,7 @@ size_t dkdv_xchg_bytes(int B, int Hq, int Hkv, int64_t S) {
 // xchg: the exchange area (dkdv_xchg_bytes), or nullptr, in which case no CTAs are paired.
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
                                const float* delta, void* dk, void* dv, float* xchg, int B, int Hq, int Hkv, int64_t S,
-                               float scale, int* status, cudaStream_t st) {
+                               float scale, int* status, uint64_t wait_ns, cudaStream_t st) {
   namespace K = tcbwd::dkdv;
   CUtensorMap mq, mdo, mks, mvs, mdk, mdv;
   if (!make_map_bf16_rows(&mq, q, (uint64_t)B * Hq * S, K::BQ) ||
@@ -978,7 +982,7 @@ cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, co
   const int nkt = (int)((S + K::BM - 1) / K::BM);
   const int cs = xchg ? dkdv_cluster_size(B, Hkv, G, nkt) : 1;
   K::Params p{B, Hq, Hkv, G, cs, G / cs, (int)(S / kQBlock), nkt, S, scale * tcbwd::kLog2e, scale, lse, delta,
-              static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), xchg, status};
+              static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), xchg, status, wait_ns};
   const int64_t grid = (int64_t)B * Hkv * nkt * cs;
   const size_t smem = K::Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(K::dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -47,6 +47,7 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int* status;
+  uint64_t wait_ns;     // limit of every bounded mbarrier wait (drains excepted)
 };
 
 constexpr int kIdxRegs = 8;                // history slots per producer lane read up front (256)
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       const uint32_t dst = sbase + (kv ? L::kV : L::kK) + s * kTileBytes;
       int ok = 1;
       if (lane == 0) {
-        ok = mbar_wait(empty, ((j / NS) & 1) ^ 1, abort_flag, p.status);
+        ok = mbar_wait(empty, ((j / NS) & 1) ^ 1, abort_flag, p.status, p.wait_ns);
         if (ok) mbar_arrive_expect_tx(full, kTileBytes);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -213,10 +214,13 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       __syncwarp();
       ++issued[s];
     }
-    // every load this warp issued has landed before the CTA may exit
-    if (lane == 0)
+    // every load this warp issued has landed before the CTA may exit (the Q tile included: a CTA
+    // that gave up early may not have waited for it)
+    if (lane == 0) {
       for (int s = 0; s < NS; ++s)
         if (issued[s]) drain_wait(kv ? v_full(s) : k_full(s), (issued[s] - 1) & 1, p.status);
+      if (!kv) drain_wait(q_full, 0, p.status);
+    }
   } else if (warp == 1) {
     // ======================= MMA issuer: the whole warp runs the loop (warp-uniform descriptors
     // and waits) and one elected lane issues each tcgen05 instruction.  All shared-memory
@@ -236,7 +240,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         mnmajor_descs<8>(vd, sbase + L::kV + (j % VS) * kTileBytes, routed ? 1024u : kHalfBytes,
                          routed ? 2048u : 1024u);
       };
-      bool ok = mbar_wait_w(q_full, 0, abort_flag, p.status) && mbar_wait_w(k_full(0), 0, abort_flag, p.status);
+      bool ok = mbar_wait_w(q_full, 0, abort_flag, p.status, p.wait_ns) && mbar_wait_w(k_full(0), 0, abort_flag, p.status, p.wait_ns);
       if (ok) {
         tc_fence_after();
         build_k(0);
@@ -249,13 +253,13 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
         mma_commit_w(k_empty(0));
       }
       for (int j = 0; ok && j < T; ++j) {
-        ok = mbar_wait_w(v_full(j % VS), (j / VS) & 1, abort_flag, p.status);
+        ok = mbar_wait_w(v_full(j % VS), (j / VS) & 1, abort_flag, p.status, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         build_v(j);
 #pragma unroll
         for (int i = 0; i < NT; ++i) {
-          ok = mbar_wait_w(p_full(i), j & 1, abort_flag, p.status);
+          ok = mbar_wait_w(p_full(i), j & 1, abort_flag, p.status, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
           if (j + 1 < T) {
             // the next K tile is only needed now, after this tile's first PV is queued
             if (i == 0) {
-              ok = mbar_wait_w(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status);
+              ok = mbar_wait_w(k_full((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag, p.status, p.wait_ns);
               if (!ok) break;
               tc_fence_after();
               build_k(j + 1);
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      ok = mbar_wait(s_full(i), j & 1, abort_flag, p.status);
+      ok = mbar_wait(s_full(i), j & 1, abort_flag, p.status, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
       mbar_arrive(p_full(i));
     }
     if (ok) {
-      ok = mbar_wait(o_final, 0, abort_flag, p.status);
+      ok = mbar_wait(o_final, 0, abort_flag, p.status, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -418,6 +422,9 @@ __global__ void __launch_bounds__(128 + 128 * NT, 1)
     tc_fence_after();
     tmem_dealloc(tmem, NT * 256);
   }
+  // a CTA that gave up before reading the router's output still completes only after the kernel
+  // before it, so the launch chain keeps its order
+  pdl_wait();
 }
 
 }  // namespace tcfwd
@@ -475,7 +482,8 @@ bool attn_fwd_tc_supported(int Hq, int Hkv) {
 
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st) {
+                               int64_t Hs, int kg, int nsg, float scale, int* status, uint64_t wait_ns,
+                               cudaStream_t st) {
   CUtensorMap mq, mkh, mvh, mks, mvs;
   // with no history the history maps are never used: map the segment instead (maps need rows > 0)
   const void* kh_m = Hs ? kh : ks;
@@ -490,7 +498,7 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, co
     return cudaErrorInvalidValue;
   const int G = Hq / Hkv;
   tcfwd::Params p{B, Hq, Hkv, G, (G % 4 == 0) ? 4 : 2, kg, (int)(S / kQBlock), nsg, H, S, Hs,
-                  scale * 1.4426950408889634f, gi, static_cast<__nv_bfloat16*>(o), lse, status};
+                  scale * 1.4426950408889634f, gi, static_cast<__nv_bfloat16*>(o), lse, status, wait_ns};
   const int64_t grid = (int64_t)B * Hkv * p.nblk * (G / p.hpc);
   cudaError_t e;
   if (p.hpc == 4) {

@@ -23,15 +23,16 @@ cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const
 bool attn_fwd_tc_supported(int Hq, int Hkv);
 cudaError_t launch_attn_fwd_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                                const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv, int64_t H, int64_t S,
-                               int64_t Hs, int kg, int nsg, float scale, int* status, cudaStream_t st);
+                               int64_t Hs, int kg, int nsg, float scale, int* status, uint64_t wait_ns,
+                               cudaStream_t st);
 cudaError_t launch_bwd_dq_tc(const void* q, const void* kh, const void* vh, const void* ks, const void* vs,
                              const int32_t* gi, const float* lse, const void* o, const void* d_o, float* delta,
                              void* dq, int B, int Hq, int Hkv, int64_t H, int64_t S, int64_t Hs, int kg, int nsg,
-                             float scale, int* status, cudaStream_t st);
+                             float scale, int* status, uint64_t wait_ns, cudaStream_t st);
 size_t dkdv_xchg_bytes(int B, int Hq, int Hkv, int64_t S);
 cudaError_t launch_bwd_dkdv_tc(const void* q, const void* ks, const void* vs, const float* lse, const void* d_o,
                                const float* delta, void* dk, void* dv, float* xchg, int B, int Hq, int Hkv, int64_t S,
-                               float scale, int* status, cudaStream_t st);
+                               float scale, int* status, uint64_t wait_ns, cudaStream_t st);
 cudaError_t launch_bwd_delta_simt(bool bf16, const void* o, const void* d_o, float* delta, int B, int Hq,
                                   int64_t S, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_simt(bool bf16, const void* q, const void* ks, const void* vs, const float* lse,
@@ -82,6 +83,7 @@ int check_config(const hga_config_t* c) {
       return HGA_ERR_ARG;
   }
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return HGA_ERR_ARG;
+  if (c->wait_limit_ns < 0) return HGA_ERR_ARG;
   // grid dimensions are 32-bit
   if ((int64_t)c->B * c->Hq * (c->seg_len / c->qblock) > INT32_MAX) return HGA_ERR_UNSUPPORTED;
   if ((int64_t)c->B * c->Hkv * nch > (int64_t)INT32_MAX) return HGA_ERR_UNSUPPORTED;   // one CTA per chunk
@@ -122,6 +124,11 @@ int check_history(const hga_config_t* c, const void* k_hist, const void* v_hist,
   if (c->hist_len == 0) return HGA_OK;
   int rc = check_ptrs({k_hist, v_hist});
   return rc ? rc : check_idx({group_idx});
+}
+
+// Limit of the tensor-core kernels' bounded on-chip waits: wait_limit_ns, or 2 s when it is 0.
+uint64_t wait_limit(const hga_config_t* c) {
+  return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull;
 }
 
 float eff_scale(const hga_config_t* c) {
@@ -177,7 +184,8 @@ int bwd_dkdv_ws(const hga_config_t* cfg, const void* q, const void* k_seg, const
   if (use_tc(cfg))
     return from_cuda(hga::launch_bwd_dkdv_tc(q, k_seg, v_seg, lse, d_o, delta_of(workspace), dk_seg, dv_seg,
                                              xchg_of(workspace, cfg, ws_bytes), cfg->B, cfg->Hq, cfg->Hkv,
-                                             cfg->seg_len, eff_scale(cfg), status_of(workspace), st));
+                                             cfg->seg_len, eff_scale(cfg), status_of(workspace), wait_limit(cfg),
+                                             st));
   return from_cuda(hga::launch_bwd_dkdv_simt(cfg->dtype == HGA_BF16, q, k_seg, v_seg, lse, d_o, delta_of(workspace),
                                              dk_seg, dv_seg, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len,
                                              cfg->top_groups, eff_scale(cfg), st));
@@ -329,7 +337,8 @@ int hga_attn_fwd(const hga_config_t* cfg, const void* q, const void* k_hist, con
   if (use_tc(cfg))
     return from_cuda(hga::launch_attn_fwd_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B, cfg->Hq,
                                              cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg), cfg->top_groups,
-                                             sink_groups(cfg), eff_scale(cfg), status_of(workspace), st));
+                                             sink_groups(cfg), eff_scale(cfg), status_of(workspace), wait_limit(cfg),
+                                             st));
   return from_cuda(hga::launch_attn_fwd_simt(bf16, q, k_hist, v_hist, k_seg, v_seg, group_idx, o, lse, cfg->B,
                                              cfg->Hq, cfg->Hkv, cfg->hist_len, cfg->seg_len, hist_rows(cfg),
                                              cfg->top_groups, sink_groups(cfg), eff_scale(cfg), status_of(workspace),
@@ -368,7 +377,7 @@ int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* k_hist, 
     return from_cuda(hga::launch_bwd_dq_tc(q, k_hist, v_hist, k_seg, v_seg, group_idx, lse, o, d_o,
                                            delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,
                                            cfg->seg_len, hist_rows(cfg), cfg->top_groups, sink_groups(cfg),
-                                           eff_scale(cfg), status_of(workspace), st));
+                                           eff_scale(cfg), status_of(workspace), wait_limit(cfg), st));
   if ((rc = hga_attn_bwd_preprocess(cfg, o, d_o, workspace, stream))) return rc;
   return from_cuda(hga::launch_bwd_dq_simt(cfg->dtype == HGA_BF16, q, k_hist, v_hist, k_seg, v_seg, group_idx, lse,
                                            d_o, delta_of(workspace), dq, cfg->B, cfg->Hq, cfg->Hkv, cfg->hist_len,

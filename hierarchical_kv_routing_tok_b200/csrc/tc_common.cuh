@@ -64,10 +64,26 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Gives up after ~limit_ns, or at once when
 // *abort is set by another thread of the CTA; on giving up it sets *abort, records
-// HGA_ERR_TIMEOUT (-5) in the status word and returns false.
+// HGA_ERR_TIMEOUT (-5) in the status word and returns false.  The default limit is 2 s; a limit
+// below kPollLimitNs (a caller that wants the expiry path exercised) polls without suspending and
+// reads the clock on every try, so that a wait longer than the limit does expire.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
+constexpr uint64_t kPollLimitNs = 1000000ull;      // 1 ms
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_test_wait(bar, parity)) return true;   // already complete: no suspend
+  if (limit_ns < kPollLimitNs) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        set_status(status, -5);
+        return false;
+      }
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
@@ -77,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
+      } else if (now - t0 > limit_ns) {
         *abort = 1;
         set_status(status, -5);
         return false;
@@ -87,14 +103,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // Bounded wait by a whole warp with a warp-uniform result.
-__device__ __forceinline__ bool mbar_wait_w(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+__device__ __forceinline__ bool mbar_wait_w(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                            uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status, limit_ns));
 }
 
-// Bounded wait that ignores the abort flag: used only to drain own copies / MMAs before exit.
+// Bounded wait that ignores the abort flag and always takes the default 2 s limit: used only to
+// drain own copies / MMAs before exit (they do complete).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status) {
   volatile int never = 0;
-  mbar_wait(bar, parity, &never, status);
+  mbar_wait(bar, parity, &never, status, kWaitLimitNs);
 }
 
 // 2^x on the MUFU unit (hardware approximation, flush-to-zero).

@@ -68,7 +68,7 @@
 extern "C" {
 #endif
 
-#define HGA_VERSION 2
+#define HGA_VERSION 3
 
 /* Symbols of the shared library (built with hidden default visibility). */
 #if defined(__GNUC__)
@@ -108,7 +108,14 @@ enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 };
  * chunks are not routable, so 1 <= top_chunks <= (hist_len - n_sink_tokens) /
  * chunk; 1 <= top_groups <= top_chunks * (chunk / group).  group_idx passed to
  * the attention calls holds routed groups only (all >= n_sink_tokens / group).
- * softmax_scale = 0 selects 1 / sqrt(D). */
+ * softmax_scale = 0 selects 1 / sqrt(D).
+ * wait_limit_ns: how long a tensor-core kernel's on-chip pipeline wait may
+ * last before the kernel gives up, records HGA_ERR_TIMEOUT in the status word,
+ * lets its own copies and MMAs land, releases its tensor memory and returns
+ * (its outputs are then undefined); 0 selects 2 s, negative is HGA_ERR_ARG.  A
+ * limit below 1 ms makes those waits poll the clock on every try (used to
+ * exercise the expiry path: a limit shorter than a tile load's latency makes
+ * the call time out). */
 typedef struct hga_config {
   int32_t B, Hq, Hkv, D;
   int64_t hist_len, seg_len;
@@ -118,6 +125,7 @@ typedef struct hga_config {
   int32_t dtype;
   float softmax_scale;
   int64_t hist_capacity;
+  int64_t wait_limit_ns;
 } hga_config_t;
 
 /* Bytes of workspace the calls below need for this configuration. */
@@ -221,16 +229,20 @@ HGA_API int hga_attn_bwd_dq(const hga_config_t* cfg, const void* q, const void* 
  *
  * Scratch: instead of a caller workspace it uses one fixed device array of
  * 256 + 4 * HGA_NOALLOC_MAX_ROWS bytes (4 MiB + 256 B) that every GPU loading
- * the library holds until the process exits.  It has no dK/dV exchange area,
- * so the dK/dV kernel runs with unpaired CTAs here (same result up to float32
- * summation order, slower when B*Hkv*ceil(S/128) is below the SM count).  B * Hq * S must not exceed
- * HGA_NOALLOC_MAX_ROWS, else HGA_ERR_TOO_LARGE is returned and nothing runs.
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  Every call clears the array's status word and overwrites the
- * rest, and all calls share it: calls that overlap on the GPU (other streams,
- * other threads) race and corrupt each other's results -- serialise them.
- * Device-side status (see hga_read_status) is not reported by this entry.
+ * the library holds until the process exits.  Of it this entry uses the status
+ * word and the B*Hq*S delta rows only; there is no dK/dV exchange area, so the
+ * dK/dV kernel always runs with unpaired CTAs here (same result up to float32
+ * summation order, slower when B*Hkv*ceil(S/128) is below the SM count).
+ * B * Hq * S must not exceed HGA_NOALLOC_MAX_ROWS, else HGA_ERR_TOO_LARGE is
+ * returned and nothing runs.
+ * The array's device address is looked up with the device current on the
+ * first call in each CUDA context of a device (the first call on a device, and
+ * the first after cudaDeviceReset); make that call before any stream capture.
+ * Every call clears the array's status word and overwrites the rest, and all
+ * calls share it: calls that overlap on the GPU (other streams, other threads)
+ * race and corrupt each other's results -- serialise them.  The device-side
+ * status of the last call (HGA_ERR_TIMEOUT, HGA_ERR_ARG, see Workspace above)
+ * stays in the array's status word: read it with hga_noalloc_read_status.
  * Arguments as for hga_attn_bwd, without workspace. */
 #define HGA_NOALLOC_MAX_ROWS (1 << 20)
 HGA_API int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, const void* k_hist,
@@ -238,6 +250,13 @@ HGA_API int hga_attn_bwd_noalloc(const hga_config_t* cfg, const void* q, const v
                                  const int32_t* group_idx, const void* o, const float* lse,
                                  const void* d_o, void* dq, void* dk_seg, void* dv_seg,
                                  void* stream);
+
+/* As hga_read_status for the fixed scratch array of hga_attn_bwd_noalloc on the
+ * current device: synchronises `stream`, copies the array's status word (the
+ * device-side status of the last hga_attn_bwd_noalloc call on this device) to
+ * *status_out and clears it.  Allocates nothing.  The paper has no counterpart
+ * of this entry point either. */
+HGA_API int hga_noalloc_read_status(void* stream, int32_t* status_out);
 
 /* ---------------------------------------------------------------- tiered history
  * Tiered storage ("Technical Summary" 2.2, "Tiered Memory Hierarchy"; pith.science

@@ -106,6 +106,7 @@ def test_workspace_size(lib):
     (dict(dtype=7), C.HGA_ERR_ARG),
     (dict(softmax_scale=-1.0), C.HGA_ERR_ARG),
     (dict(softmax_scale=float("nan")), C.HGA_ERR_ARG),
+    (dict(wait_limit_ns=-1), C.HGA_ERR_ARG),          # the bounded-wait limit: 0 (2 s) or positive
     (dict(hist_len=64 * 40000, top_chunks=16), C.HGA_ERR_UNSUPPORTED),
 ])
 def test_config_validation(lib, kw, code):

@@ -20,7 +20,10 @@ def hga():
     return H
 
 
-@pytest.mark.parametrize("name,tol", [("small_bf16", 2e-2), ("tiny_f32", 1e-4)])
+# small_bf16: its caller workspace pairs dK/dV CTAs; ctx4k (the 4K layer, B*Hq*S = 65536 rows):
+# its 16 MiB exchange area would not fit the fixed array either -- this entry never pairs CTAs, so
+# both compare the unpaired tensor-core dK/dV path with the paired one of the workspace backward
+@pytest.mark.parametrize("name,tol", [("small_bf16", 2e-2), ("tiny_f32", 1e-4), ("ctx4k", 2e-2)])
 def test_noalloc_backward_matches_workspace_backward(hga, name, tol):
     C = hga._capi
     w = HI.WORKLOADS[name]
@@ -37,7 +40,7 @@ def test_noalloc_backward_matches_workspace_backward(hga, name, tol):
                            x["k_seg"].data_ptr(), x["v_seg"].data_ptr(), step.group_idx.data_ptr(),
                            step.o.data_ptr(), step.lse.data_ptr(), x["d_o"].data_ptr(), dq.data_ptr(),
                            dk.data_ptr(), dv.data_ptr(), st)
-        torch.cuda.synchronize()
+        assert C.noalloc_read_status(st) == 0          # no device-side error (read and cleared)
         for got, want in zip((dq, dk, dv), ref):
             assert torch.isfinite(got).all()
             assert (got.float() - want.float()).abs().max().item() <= tol
