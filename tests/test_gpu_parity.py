@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import hga_inputs as HI
+from oracle_slices import attn_sampled
 
 pytestmark = pytest.mark.gpu
 
@@ -181,6 +182,15 @@ def _sampled_rows(w, n, seed):
     return np.array(sorted(set(ids)), dtype=np.int64)
 
 
+def _sampled_keys(w):
+    """Segment keys of every (batch, KV head): both ends of every 128-key tile of the dK/dV kernel
+    (so every CTA, and both CTAs of every cluster pair, is looked at) plus two keys inside tiles."""
+    us = sorted({u for t in range(0, w.seg_len, 128) for u in (t, min(t + 127, w.seg_len - 1))}
+                | {min(64, w.seg_len - 1), w.seg_len // 2 + 37})
+    return np.array([(b * w.Hkv + kh) * w.seg_len + u for b in range(w.B) for kh in range(w.Hkv) for u in us],
+                    dtype=np.int64)
+
+
 @pytest.mark.parametrize("name,seed", [("ctx4k", 0), ("ctx4k", 1), ("ctx16k", 0), ("ctx16k", 2),
                                        ("ctx16k_kc8", 0), ("ctx16k_kc32", 0)])
 def test_full_size_layer_sampled(hga, oracle, name, seed):
@@ -191,12 +201,10 @@ def test_full_size_layer_sampled(hga, oracle, name, seed):
     assert np.array_equal(g["ci"].numpy(), r["chunk_idx"])
     assert np.array_equal(g["gi"].numpy(), r["group_idx"])
     rows = _sampled_rows(w, 96, seed)
-    # keys: two KV heads, spread over the segment including both ends
-    keys = np.array([kh * w.seg_len + u for kh in (0, w.Hkv - 1) for u in (0, 1, 63, 64, 1000, 2046, 2047)],
-                    dtype=np.int64)
-    args = (x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
-    o, lse = oracle.attn_fwd(*args, rows=rows)
-    dq, dk, dv = oracle.attn_bwd(*args, x["d_o"], rows=rows, keys=keys)
+    keys = _sampled_keys(w)
+    ref = attn_sampled(oracle, x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"], x["d_o"],
+                       rows=rows, keys=keys)
+    o, lse, dq, dk, dv = (ref[k] for k in ("o", "lse", "dq", "dk", "dv"))
     D = w.D
     e = dict(o=maxerr(g["o"].reshape(-1, D)[rows], o), lse=maxerr(g["lse"].reshape(-1)[rows], lse),
              dq=maxerr(g["dq"].reshape(-1, D)[rows], dq), dk=maxerr(g["dk"].reshape(-1, D)[keys], dk),

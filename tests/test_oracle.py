@@ -486,13 +486,13 @@ def test_invalid_arguments_raise(oracle):
 
 # --------------------------------------------------------------------------- inputs used by GPU parity
 PARITY_SEEDS = {"tiny_f32": [0, 1, 2, 3, 4], "small_bf16": [0, 1], "ctx4k": [0, 1], "ctx16k": [0, 2],
-                "ctx16k_kc8": [0], "ctx16k_kc32": [0], "ctx131k": [0]}
+                "ctx16k_kc8": [0], "ctx16k_kc32": [0], "ctx131k": [0], "ctx16k_b4": [11]}
 PARITY_SEEDS.update({name: [0] for name in HI.EDGE_WORKLOADS})
 MIN_GAP = 4e-6
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "small_bf16", "ctx4k", "ctx16k", "ctx16k_kc8", "ctx16k_kc32",
-                                  *HI.EDGE_WORKLOADS])
+                                  "ctx16k_b4", *HI.EDGE_WORKLOADS])
 def test_parity_seeds_have_routing_margins(oracle, name):
     """For the seeds the GPU parity tests use, the fp32 routing equals the fp64 routing and every
     selection boundary has a score gap >= MIN_GAP (far above fp32 rounding of these scores,

@@ -157,7 +157,9 @@ def test_two_layer_model_trained_segment_by_segment(hga, oracle):
     """A two-layer residual model with HGA attention, trained by TBPTT over four segments (loss
     back-propagated per segment, each layer's K/V appended to its history at the boundary): the
     per-segment losses and every parameter gradient equal those of the same model whose attention
-    is the float64 oracle (run with the routing the GPU chose)."""
+    is the float64 oracle, run with the routing the GPU chose.  That routing is itself checked: each
+    layer's GPU routing of each segment equals the oracle's float32 routing of the same projected q
+    and history keys (copied to the host), whose selection margins are checked to be >= MIN_GAP."""
     B, Hq, Hkv, D, S, nseg, dm, kc, kg = 1, 4, 1, 128, 128, 4, 32, 2, 8
     g = torch.Generator().manual_seed(21)
     params = {n: torch.randn(*shape, generator=g, dtype=torch.float64) * 0.3
@@ -174,6 +176,7 @@ def test_two_layer_model_trained_segment_by_segment(hga, oracle):
     pg = {n: p.float().cuda().requires_grad_(True) for n, p in params.items()}
     hists = [hga.HGAHistory(B, Hq, Hkv, nseg * S, dtype=torch.float32) for _ in range(2)]
     losses_gpu, routing = [], []
+    past_k = [[], []]                                     # host copies of each layer's earlier keys
     for s in range(nseg):
         h = xs[s].float().cuda()
         kv, gis = [], []
@@ -182,7 +185,19 @@ def test_two_layer_model_trained_segment_by_segment(hga, oracle):
             o, gi = hga.segment_attention(q, k, v, hists[l], kc, kg)
             h = h + o.transpose(1, 2).reshape(B, S, Hq * D) @ pg[f"wo{l}"]
             kv.append((k.detach(), v.detach()))
-            gis.append(gi.cpu().numpy() if hists[l].length else np.zeros((B, Hkv, S // 64, 0), np.int32))
+            if hists[l].length:
+                # the routing the GPU chose, against the oracle on the same float32 q and history keys
+                kc2, kg2, _ = _clamped(hists[l].length, kc, kg, 0)
+                qh, kh = q.detach().cpu(), torch.cat(past_k[l], dim=2)
+                r32 = oracle.route_from_inputs(qh, kh, Hkv, kc2, kg2, prec=32)
+                r64 = oracle.route_from_inputs(qh, kh, Hkv, kc2, kg2, prec=64)
+                assert np.array_equal(r32["group_idx"], r64["group_idx"])
+                assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
+                assert np.array_equal(gi.cpu().numpy(), r32["group_idx"]), (s, l)
+                gis.append(r32["group_idx"])
+            else:
+                gis.append(np.zeros((B, Hkv, S // 64, 0), np.int32))
+            past_k[l].append(k.detach().cpu())
         loss = ((h - tgt[s].float().cuda()) ** 2).mean()
         loss.backward()                                   # truncated: history is detached
         losses_gpu.append(loss.item())

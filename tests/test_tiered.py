@@ -1,12 +1,17 @@
 """Tiered history (history K/V in pinned host memory, compact device cache per step) on a B200:
-the plan is the exact union of the routed groups with order-preserving positions, the gather
-copies exactly those rows, and the whole tiered step equals the step over device-resident
-history bit for bit (hence the oracle parity of the resident step carries over)."""
+the tiered step matches the oracle over the whole history (routing bit-exact, outputs within the
+bars of the resident path), the plan is the exact union of the routed groups with
+order-preserving positions, the gather copies exactly those rows, and the whole tiered step
+equals the step over device-resident history bit for bit."""
 import numpy as np
 import pytest
 import torch
 
 import hga_inputs as HI
+from oracle_slices import attn_sampled
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+LSE_TOL = {"f32": 1e-4, "bf16": 1e-3}
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +45,67 @@ def _tiered(hga, cfg, step, x, xd):
     t(xd)
     t.wait(timeout_s=60)
     return t
+
+
+def _tiered_only(hga, w, x):
+    """The tiered step alone: summaries built on the device while the history keys are there (as
+    when the history is written), then K/V kept only in pinned host memory."""
+    xd = {k: x[k].cuda() for k in ("q", "k_seg", "v_seg", "d_o")}
+    cfg = hga.make_config(xd["q"], x["k_hist"], w.top_chunks, w.top_groups, n_sink_tokens=w.n_sink)
+    gs, cs = hga.build_summaries(cfg, x["k_hist"].cuda())
+    t = hga.TieredLayerStep(cfg, x["k_hist"].pin_memory(), x["v_hist"].pin_memory(), gs, cs)
+    t(xd)
+    t.wait(timeout_s=120)
+    return t
+
+
+@pytest.mark.parametrize("name", ["small_bf16", "sink_bf16", "gqa2_ragged_bf16", "tiny_f32"])
+def test_tiered_step_matches_oracle(hga, oracle, name):
+    """The tiered step against the oracle over the whole history, element by element."""
+    w = _wl(name)
+    x = HI.make_inputs(w, 0)
+    t = _tiered_only(hga, w, x)
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32, n_sink=w.n_sink)
+    assert np.array_equal(t.chunk_idx.cpu().numpy(), r["chunk_idx"])
+    assert np.array_equal(t.group_idx.cpu().numpy(), r["group_idx"])
+    args = (x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
+    o, lse = oracle.attn_fwd(*args, n_sink=w.n_sink)
+    dq, dk, dv = oracle.attn_bwd(*args, x["d_o"], n_sink=w.n_sink)
+    err = lambda a, b: float(np.abs(a.float().cpu().numpy() - b).max())
+    errs = dict(o=err(t.o, o), dq=err(t.dq, dq), dk=err(t.dk, dk), dv=err(t.dv, dv))
+    assert max(errs.values()) <= TOL[w.dtype], errs
+    assert err(t.lse, lse) <= LSE_TOL[w.dtype]
+
+
+def test_tiered_16k_batch4_matches_oracle_sampled(hga, oracle):
+    """The tiered-history workload itself (the 16K layer at batch 4, 224 MiB of history K/V in
+    pinned host memory): every routing index bit-exact, sampled rows of every batch element (block
+    ends included) and the keys at both ends of every 128-key tile of four (batch, KV head) slices."""
+    w = HI.WORKLOADS["ctx16k_b4"]
+    x = HI.make_inputs(w, 11)             # seed with routing margins >= MIN_GAP (checked on the CPU)
+    t = _tiered_only(hga, w, x)
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32)
+    assert np.array_equal(t.chunk_idx.cpu().numpy(), r["chunk_idx"])
+    assert np.array_equal(t.group_idx.cpu().numpy(), r["group_idx"])
+    ids = set(HI.sample_ids(w.B * w.Hq * w.seg_len, 96, 7).tolist())
+    for b in range(w.B):
+        for h in (0, w.Hq - 1):
+            for blk in (0, w.nblk - 1):
+                base = (b * w.Hq + h) * w.seg_len + blk * 64
+                ids |= {base, base + 63}
+    rows = np.array(sorted(ids), dtype=np.int64)
+    us = sorted({u for t0 in range(0, w.seg_len, 128) for u in (t0, t0 + 127)})
+    keys = np.array([(b * w.Hkv + kh) * w.seg_len + u for b in (0, w.B - 1) for kh in (0, w.Hkv - 1) for u in us],
+                    dtype=np.int64)
+    ref = attn_sampled(oracle, x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"], x["d_o"],
+                       rows=rows, keys=keys)
+    D = w.D
+    got = lambda t_, ids_: t_.reshape(-1, D)[torch.as_tensor(ids_, device=t_.device)].float().cpu().numpy()
+    e = dict(o=np.abs(got(t.o, rows) - ref["o"]).max(), dq=np.abs(got(t.dq, rows) - ref["dq"]).max(),
+             dk=np.abs(got(t.dk, keys) - ref["dk"]).max(), dv=np.abs(got(t.dv, keys) - ref["dv"]).max(),
+             lse=np.abs(t.lse.reshape(-1)[torch.as_tensor(rows, device=t.lse.device)].cpu().numpy()
+                        - ref["lse"]).max())
+    assert e["lse"] <= 1e-3 and max(e["o"], e["dq"], e["dk"], e["dv"]) <= 2e-2, e
 
 
 @pytest.mark.parametrize("name", ["small_bf16", "sink_bf16", "tiny_f32", "gqa2_ragged_bf16", "sink_f32"])
