@@ -347,7 +347,10 @@ def _leakage_probe(H, w, seed, dev) -> dict:
 
 def _time_tiered(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=2) -> dict:
     """The layer of workload w with its history K/V in pinned host memory (TieredLayerStep), and the
-    same layer with the history resident in device memory, both timed per step on the device."""
+    same layer with the history resident in device memory, both timed per step on the device; then
+    the pages' three tiers: also the group summaries in pinned host memory behind a device cache
+    smaller than the history (GroupSummaryCache), the chunk summaries alone resident, with two query
+    sets alternating from step to step so that steps fetch the chunks the cache lacks."""
     x = HI.make_inputs(w, seed)
     xd = {k: x[k].to(dev) for k in ("q", "k_seg", "v_seg", "d_o")}
     kh, vh = x["k_hist"].pin_memory(), x["v_hist"].pin_memory()
@@ -355,25 +358,48 @@ def _time_tiered(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=2) ->
     # summaries are built when the history is written, while its keys are still on the device
     gs, cs = H.build_summaries(cfg, x["k_hist"].to(dev))
     step = H.TieredLayerStep(cfg, kh, vh, gs, cs, dev)
-    for _ in range(warmup):
-        step(xd)
-    step.wait(timeout_s=60)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for e0, e1 in ev:
-        flush_l2()
-        e0.record(stream)
-        step(xd)
-        e1.record(stream)
-    step.wait(timeout_s=60)
-    ms = all_max(sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps, world, dev)
+
+    def timed(st, inputs):
+        for i in range(warmup):
+            st(inputs[i % len(inputs)])
+        st.wait(timeout_s=60)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i, (e0, e1) in enumerate(ev):
+            flush_l2()
+            e0.record(stream)
+            st(inputs[i % len(inputs)])
+            e1.record(stream)
+        st.wait(timeout_s=60)
+        return all_max(sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps, world, dev)
+
+    ms = timed(step, [xd])
     nbytes = step.gather_bytes()
     resident_ms = all_max(_time_layer(H, w, seed, dev, stream, flush_l2), world, dev)
     tokens = w.B * w.seg_len * world
+    # the three tiers: group summaries in host memory behind the device cache, 4 chunk slots short of
+    # the whole history (a step of these inputs chooses at most 215 of the 224 chunks of a KV head)
+    cap = max(1, w.nch - 4)
+    gcache = H.GroupSummaryCache(cfg, gs.cpu().pin_memory(), cap, dev)
+    step3 = H.TieredLayerStep(cfg, kh, vh, None, cs, dev, group_cache=gcache)
+    xd2 = dict(xd, q=HI.make_inputs(w, seed + 1)["q"].to(dev))
+    step3([xd, xd2][0])
+    step3.wait(timeout_s=60)
+    cold = gcache.stats()
+    ms3 = timed(step3, [xd2, xd])
+    warm = gcache.stats()
     return {"workload": f"{w.name}: the 16K layer at batch {w.B}, history K/V ({2 * kh.numel() * kh.element_size() >> 20}"
                         " MiB) in pinned host memory, summaries in device memory",
             "ms_per_step": ms, "tokens_per_s": tokens / (ms * 1e-3),
             "gather_bytes_per_step": nbytes, "host_link_GBps": nbytes / (ms * 1e-3) / 1e9,
-            "resident_ms_per_step": resident_ms, "resident_tokens_per_s": tokens / (resident_ms * 1e-3)}
+            "resident_ms_per_step": resident_ms, "resident_tokens_per_s": tokens / (resident_ms * 1e-3),
+            "group_summary_cache": {
+                "layout": f"chunk summaries in device memory; group summaries ({gs.numel() * 4 >> 20} MiB) in pinned "
+                          f"host memory behind a device cache of {cap} of the {w.nch} chunks per (batch, KV head) "
+                          "(8 group summaries = 4 KB per chunk slot, least recently used replaced); K/V as above; "
+                          "two query sets alternate from step to step",
+                "cap_chunks": cap, "ms_per_step": ms3, "tokens_per_s": tokens / (ms3 * 1e-3),
+                "first_step": cold, "last_step": warm,
+                "host_bytes_per_step": warm["host_bytes"] + step3.gather_bytes()}}
 
 
 def _time_forward_131k(H, w, seed, dev, stream, flush_l2, world, steps=5, warmup=3) -> dict:

@@ -29,7 +29,8 @@ HGA_BF16 = 1
 EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_append_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
            "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
-           "hga_noalloc_read_status", "hga_tier_cache_config", "hga_tier_plan", "hga_tier_gather",
+           "hga_noalloc_read_status", "hga_tier_cache_config", "hga_route_chunks", "hga_gcache_plan",
+           "hga_gcache_fetch", "hga_route_groups_cached", "hga_tier_plan", "hga_tier_gather",
            "hga_read_status", "hga_strerror", "hga_version")
 
 
@@ -79,6 +80,10 @@ def load() -> ctypes.CDLL:
         "hga_attn_bwd_noalloc": [C, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_noalloc_read_status": [P, ctypes.POINTER(ctypes.c_int32)],
         "hga_tier_cache_config": [C, C],
+        "hga_route_chunks": [C, P, P, P, P, P, P],
+        "hga_gcache_plan": [C, ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P, P],
+        "hga_gcache_fetch": [C, ctypes.c_int32, P, P, P, P, P, P],
+        "hga_route_groups_cached": [C, P, P, P, ctypes.c_int32, P, P, P, P],
         "hga_tier_plan": [C, P, P, P, P, P, P],
         "hga_tier_gather": [C, P, P, P, P, P, P, P],
         "hga_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
@@ -178,6 +183,27 @@ def noalloc_read_status(stream=0) -> int:
     out = ctypes.c_int32(0)
     _call("hga_noalloc_read_status", stream, ctypes.byref(out))
     return int(out.value)
+
+
+def route_chunks(cfg, q, chunk_sum, chunk_idx, qb, workspace, stream=0) -> None:
+    """Level 1 of the routing only: chunk_idx and the block queries qb."""
+    _call("hga_route_chunks", ctypes.byref(cfg), q, chunk_sum, chunk_idx, qb, workspace, stream)
+
+
+def gcache_plan(cfg, cap_chunks, chunk_idx, slot_of, chunk_of, stamp, step, miss_chunk, miss_slot, counts,
+                workspace, stream=0) -> None:
+    _call("hga_gcache_plan", ctypes.byref(cfg), int(cap_chunks), chunk_idx, slot_of, chunk_of, stamp, int(step),
+          miss_chunk, miss_slot, counts, workspace, stream)
+
+
+def gcache_fetch(cfg, cap_chunks, group_sum_src, miss_chunk, miss_slot, counts, gcache, stream=0) -> None:
+    _call("hga_gcache_fetch", ctypes.byref(cfg), int(cap_chunks), group_sum_src, miss_chunk, miss_slot, counts,
+          gcache, stream)
+
+
+def route_groups_cached(cfg, qb, chunk_idx, slot_of, cap_chunks, gcache, group_idx, workspace, stream=0) -> None:
+    _call("hga_route_groups_cached", ctypes.byref(cfg), qb, chunk_idx, slot_of, int(cap_chunks), gcache, group_idx,
+          workspace, stream)
 
 
 def tier_cache_config(cfg) -> HGAConfig:

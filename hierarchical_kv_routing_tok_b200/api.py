@@ -285,6 +285,64 @@ class LayerStep:
         return g
 
 
+class GroupSummaryCache:
+    """Device cache of the group summaries of a history whose group-summary table lives in host
+    memory ("Technical Summary" 2.1 Group Selection: group summaries are cached in device memory and
+    the missing ones fetched from host memory; the chunk summaries stay in device memory).  Each of
+    the ``cap_chunks`` slots per (batch, KV head) holds the 8 group summaries of one chunk; a step
+    routes level 1 on the device chunk summaries, fetches the chosen chunks the cache lacks (least
+    recently used slots make room) and routes level 2 from the cache, giving the same indices as
+    the routing over the full table.
+
+    group_sum_host: pinned CPU float32 [B, Hkv, Hs/8, D] (Hs = the history's capacity in tokens)."""
+
+    CHUNK_BYTES = 8 * 128 * 4          # one slot: 8 group summaries of 128 float32
+
+    def __init__(self, cfg, group_sum_host, cap_chunks: int, device="cuda"):
+        dev = torch.device(device)
+        B, Hkv, D = cfg.B, cfg.Hkv, cfg.D
+        hs = cfg.hist_capacity or cfg.hist_len
+        if group_sum_host.is_cuda or not group_sum_host.is_pinned():
+            raise ValueError("group_sum_host must be pinned host memory")
+        if (tuple(group_sum_host.shape) != (B, Hkv, hs // cfg.group, D) or group_sum_host.dtype != torch.float32
+                or not group_sum_host.is_contiguous()):
+            raise ValueError(f"group_sum_host: expected contiguous float32 {(B, Hkv, hs // cfg.group, D)}")
+        self.cfg, self.dev, self.cap = cfg, dev, int(cap_chunks)
+        self.host = group_sum_host
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.slot_of = torch.full((B, Hkv, hs // cfg.chunk), -1, **i32)
+        self.chunk_of = torch.full((B, Hkv, self.cap), -1, **i32)
+        self.stamp = torch.full((B, Hkv, self.cap), -1, **i32)
+        self.miss_chunk = torch.empty(B, Hkv, self.cap, **i32)
+        self.miss_slot = torch.empty(B, Hkv, self.cap, **i32)
+        self.counts = torch.zeros(B * Hkv, 2, **i32)
+        self.gcache = torch.empty(B, Hkv, self.cap, 8, D, dtype=torch.float32, device=dev)
+        self.qb = torch.empty(B, Hkv, cfg.seg_len // cfg.qblock, D, dtype=torch.float32, device=dev)
+        self.step = 0
+
+    def route(self, q, chunk_sum, chunk_idx, group_idx, workspace, stream: int | None = None) -> None:
+        """Both routing levels of one step through the cache (asynchronous on ``stream``)."""
+        cfg, cap = self.cfg, self.cap
+        st = torch.cuda.current_stream(self.dev).cuda_stream if stream is None else stream
+        ws = workspace.data_ptr()
+        C.route_chunks(cfg, q.data_ptr(), chunk_sum.data_ptr(), chunk_idx.data_ptr(), self.qb.data_ptr(), ws, st)
+        C.gcache_plan(cfg, cap, chunk_idx.data_ptr(), self.slot_of.data_ptr(), self.chunk_of.data_ptr(),
+                      self.stamp.data_ptr(), self.step, self.miss_chunk.data_ptr(), self.miss_slot.data_ptr(),
+                      self.counts.data_ptr(), ws, st)
+        C.gcache_fetch(cfg, cap, self.host.data_ptr(), self.miss_chunk.data_ptr(), self.miss_slot.data_ptr(),
+                       self.counts.data_ptr(), self.gcache.data_ptr(), st)
+        C.route_groups_cached(cfg, self.qb.data_ptr(), chunk_idx.data_ptr(), self.slot_of.data_ptr(), cap,
+                              self.gcache.data_ptr(), group_idx.data_ptr(), ws, st)
+        self.step += 1
+
+    def stats(self) -> dict:
+        """Hits and misses of the last step (chunks, summed over batch and KV heads) and the bytes of
+        group summaries it fetched from host memory (synchronises)."""
+        c = self.counts.sum(dim=0).tolist()
+        return {"hits": int(c[0]), "misses": int(c[1]), "host_bytes": int(c[1]) * self.CHUNK_BYTES,
+                "cap_chunks": self.cap}
+
+
 class TieredLayerStep:
     """One layer step with the detached history K/V in pinned host memory (tiered storage,
     "Technical Summary" 2.2): the summaries and the routing stay in device memory; per step only
@@ -293,9 +351,13 @@ class TieredLayerStep:
     overlaps the forward and backward of element b on the caller's stream.
 
     k_hist_host / v_hist_host: pinned CPU tensors [B, Hkv, H, D] (``pin_memory=True``);
-    group_sum / chunk_sum: the device summaries of that history (built when it was written)."""
+    group_sum / chunk_sum: the device summaries of that history (built when it was written);
+    group_cache: a GroupSummaryCache over the history's group summaries in host memory -- the
+    routing then reads the group summaries through it (group_sum may be None), so that only the
+    chunk summaries stay in device memory, as in the pages' three tiers."""
 
-    def __init__(self, cfg, k_hist_host, v_hist_host, group_sum, chunk_sum, device="cuda"):
+    def __init__(self, cfg, k_hist_host, v_hist_host, group_sum, chunk_sum, device="cuda",
+                 group_cache: "GroupSummaryCache | None" = None):
         dev = torch.device(device)
         B, Hq, Hkv, S, H, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.seg_len, cfg.hist_len, cfg.D
         dt = _tdtype(cfg)
@@ -315,6 +377,9 @@ class TieredLayerStep:
         nblk = S // cfg.qblock
         self.k_host, self.v_host = k_hist_host, v_hist_host
         self.group_sum, self.chunk_sum = group_sum, chunk_sum
+        self.group_cache = group_cache
+        if group_sum is None and group_cache is None:
+            raise ValueError("group_sum is needed unless a group_cache is given")
         i32 = dict(dtype=torch.int32, device=dev)
         self.chunk_idx = torch.empty(B, Hkv, nblk, cfg.top_chunks, **i32)
         self.group_idx = torch.empty(B, Hkv, nblk, cfg.top_groups, **i32)
@@ -342,8 +407,11 @@ class TieredLayerStep:
         main = torch.cuda.current_stream(self.dev)
         st, side = main.cuda_stream, self.side.cuda_stream
         ws = self.ws.data_ptr()
-        C.route(cfg, x["q"].data_ptr(), self.group_sum.data_ptr(), self.chunk_sum.data_ptr(),
-                self.chunk_idx.data_ptr(), self.group_idx.data_ptr(), ws, st)
+        if self.group_cache is not None:
+            self.group_cache.route(x["q"], self.chunk_sum, self.chunk_idx, self.group_idx, self.ws, st)
+        else:
+            C.route(cfg, x["q"].data_ptr(), self.group_sum.data_ptr(), self.chunk_sum.data_ptr(),
+                    self.chunk_idx.data_ptr(), self.group_idx.data_ptr(), ws, st)
         C.tier_plan(cfg, self.group_idx.data_ptr(), self.used_groups.data_ptr(), self.n_used.data_ptr(),
                     self.compact_idx.data_ptr(), ws, st)
         self.planned.record(main)

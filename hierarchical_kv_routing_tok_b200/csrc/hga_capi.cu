@@ -16,6 +16,18 @@ cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool caus
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
                          int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream);
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg);
+cudaError_t launch_route_chunks(bool bf16, const void* q, const void* q_prev, bool causal, const float* chunk_sum,
+                                int32_t* chunk_idx, float* qb, int B, int Hq, int Hkv, int64_t S, int nch,
+                                int nch_stride, int nsc, int kc, cudaStream_t stream);
+cudaError_t launch_route_groups_cached(const float* qb, const int32_t* chunk_idx, const int32_t* slot_of,
+                                       const float* gcache, int cap, int32_t* group_idx, int B, int Hkv, int64_t S,
+                                       int nch_stride, int kc, int kg, int* status, cudaStream_t stream);
+size_t gcache_plan_smem_bytes(int nchs, int cap);
+cudaError_t launch_gcache_plan(const int32_t* chunk_idx, int BHkv, int nidx, int nchs, int cap, int step,
+                               int32_t* slot_of, int32_t* chunk_of, int32_t* stamp, int32_t* miss_chunk,
+                               int32_t* miss_slot, int32_t* counts, int* status, cudaStream_t st);
+cudaError_t launch_gcache_fetch(const float* gsum, int64_t ngrs, const int32_t* miss_chunk, const int32_t* miss_slot,
+                                const int32_t* counts, int BHkv, int cap, float* gcache, cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(bool bf16, const void* q, const void* kh, const void* vh, const void* ks,
                                  const void* vs, const int32_t* gi, void* o, float* lse, int B, int Hq, int Hkv,
                                  int64_t H, int64_t S, int64_t Hs, int kg, int nsg, float scale, int* status,
@@ -434,6 +446,84 @@ int hga_tier_gather(const hga_config_t* cfg, const void* k_hist, const void* v_h
   return from_cuda(hga::launch_tier_gather(cfg->dtype == HGA_BF16, kh, vh, used_groups, n_used, cfg->B * cfg->Hkv,
                                            hist_rows(cfg), (int)tier_cap_groups(cfg), k_cache, v_cache,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- group-summary cache
+namespace {
+constexpr int kMaxCacheSlots = 4096;
+
+// cap_chunks: slots per (batch, KV head), 1 .. min(4096, the history's capacity in chunks).
+int check_cache(const hga_config_t* c, int32_t cap) {
+  const int64_t nchs = hist_rows(c) / c->chunk;
+  if (cap < 1 || cap > kMaxCacheSlots || cap > nchs) return HGA_ERR_ARG;
+  if (hga::gcache_plan_smem_bytes((int)nchs, cap) > 200 * 1024) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+}  // namespace
+
+int hga_route_chunks(const hga_config_t* cfg, const void* q, const float* chunk_sum, int32_t* chunk_idx, float* qb,
+                     void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_ptrs({q, chunk_sum}))) return rc;
+  (void)workspace;
+  if (cfg->hist_len == 0) return HGA_OK;        // nothing to route
+  if ((rc = check_idx({chunk_idx}))) return rc;
+  if ((rc = check_ptrs({qb}))) return rc;
+  return from_cuda(hga::launch_route_chunks(cfg->dtype == HGA_BF16, q, nullptr, false, chunk_sum, chunk_idx, qb,
+                                            cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len, (int)(cfg->hist_len / cfg->chunk),
+                                            (int)(hist_rows(cfg) / cfg->chunk), (int)(cfg->n_sink_tokens / cfg->chunk),
+                                            cfg->top_chunks, static_cast<cudaStream_t>(stream)));
+}
+
+int hga_gcache_plan(const hga_config_t* cfg, int32_t cap_chunks, const int32_t* chunk_idx, int32_t* slot_of,
+                    int32_t* chunk_of, int32_t* stamp, int32_t step, int32_t* miss_chunk, int32_t* miss_slot,
+                    int32_t* counts, void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (cfg->hist_len == 0) return HGA_OK;
+  if ((rc = check_cache(cfg, cap_chunks))) return rc;
+  if ((rc = check_idx({chunk_idx, slot_of, chunk_of, stamp, miss_chunk, miss_slot, counts}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  return from_cuda(hga::launch_gcache_plan(chunk_idx, cfg->B * cfg->Hkv,
+                                           (int)(cfg->seg_len / cfg->qblock) * cfg->top_chunks,
+                                           (int)(hist_rows(cfg) / cfg->chunk), cap_chunks, step, slot_of, chunk_of,
+                                           stamp, miss_chunk, miss_slot, counts, status_of(workspace),
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int hga_gcache_fetch(const hga_config_t* cfg, int32_t cap_chunks, const float* group_sum_src, const int32_t* miss_chunk,
+                     const int32_t* miss_slot, const int32_t* counts, float* gcache, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (cfg->hist_len == 0) return HGA_OK;
+  if ((rc = check_cache(cfg, cap_chunks))) return rc;
+  if ((rc = check_ptrs({group_sum_src, gcache}))) return rc;
+  if ((rc = check_idx({miss_chunk, miss_slot, counts}))) return rc;
+  const size_t bytes = (size_t)cfg->B * cfg->Hkv * (hist_rows(cfg) / cfg->group) * cfg->D * sizeof(float);
+  const void* src = device_view(group_sum_src, bytes);
+  if (!src) return HGA_ERR_ARG;                 // pageable host memory cannot be read by the device
+  return from_cuda(hga::launch_gcache_fetch(static_cast<const float*>(src), hist_rows(cfg) / cfg->group, miss_chunk,
+                                            miss_slot, counts, cfg->B * cfg->Hkv, cap_chunks, gcache,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int hga_route_groups_cached(const hga_config_t* cfg, const float* qb, const int32_t* chunk_idx,
+                            const int32_t* slot_of, int32_t cap_chunks, const float* gcache, int32_t* group_idx,
+                            void* workspace, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (cfg->hist_len == 0) return HGA_OK;
+  if ((rc = check_cache(cfg, cap_chunks))) return rc;
+  if ((rc = check_ptrs({qb, gcache}))) return rc;
+  if ((rc = check_idx({chunk_idx, slot_of, group_idx}))) return rc;
+  if (!workspace) return HGA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+  return from_cuda(hga::launch_route_groups_cached(qb, chunk_idx, slot_of, gcache, cap_chunks, group_idx, cfg->B,
+                                                   cfg->Hkv, cfg->seg_len, (int)(hist_rows(cfg) / cfg->chunk),
+                                                   cfg->top_chunks, cfg->top_groups, status_of(workspace),
+                                                   static_cast<cudaStream_t>(stream)));
 }
 
 int hga_read_status(void* workspace, void* stream, int32_t* status_out) {

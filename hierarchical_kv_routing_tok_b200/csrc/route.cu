@@ -12,6 +12,11 @@
 // finish with an index-ordered compaction, so ties go to the lower index and the
 // output comes out sorted ascending.  This is not a dense contraction
 // (M = 1 per CTA), so it runs on the CUDA cores.
+//
+// The same kernel also runs the two levels separately, for routing with a device cache of group
+// summaries (the group summaries of a long history in host memory, "Technical Summary" 2.1 Group
+// Selection): mode 1 stops after level 1 and writes the chunk indices and the block query; mode 2
+// starts from those and scores the group summaries of the chosen chunks from their cache slots.
 #include "common.cuh"
 
 namespace hga {
@@ -190,11 +195,21 @@ __device__ __forceinline__ void score_rows(const float* qb, const float* __restr
   }
 }
 
-template <typename T>
+// Routing modes and the inputs / outputs of the cached group level.
+enum RouteMode { kRouteFull = 0, kRouteChunks = 1, kRouteGroupsCached = 2 };
+struct RouteCache {
+  float* qb;                // [units][128] block queries: written in mode 1, read in mode 2
+  const int32_t* slot_of;   // mode 2: [B*Hkv][nch_stride] cache slot of each chunk (-1: not cached)
+  const float* gcache;      // mode 2: [B*Hkv][cap][8][128] group summaries of the cached chunks
+  int cap;                  // mode 2: cache slots per (batch, KV head)
+  int* status;              // mode 2: a chosen chunk missing from the cache records HGA_ERR_ARG here
+};
+
+template <typename T, int MODE>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     const T* __restrict__ q, const T* __restrict__ q_prev, int causal, const float* __restrict__ group_sum,
     const float* __restrict__ chunk_sum, int32_t* __restrict__ chunk_idx, int32_t* __restrict__ group_idx, int Hq,
-    int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg) {
+    int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, const RouteCache rc) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   if (threadIdx.x == 0) pdl_trigger();
   constexpr int N = Vec16<T>::N;
@@ -232,7 +247,13 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
       zero_query = true;
     }
   }
-  {
+  if (MODE == kRouteGroupsCached) {
+    // the block query and the chosen chunks come from the level-1 call (a kernel before)
+    pdl_wait();
+    if (threadIdx.x < kD) qb[threadIdx.x] = rc.qb[(int64_t)unit * kD + threadIdx.x];
+    for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] = chunk_idx[(int64_t)unit * kc + i];
+    __syncthreads();
+  } else {
     const int tid = threadIdx.x;
     const int col = (tid % LPR) * N, r0 = tid / LPR;
     float acc[N];
@@ -272,29 +293,54 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     __syncthreads();
   }
 
-  // the block query needs only q: the summaries are read once the kernel before has completed
-  pdl_wait();
+  if (MODE != kRouteGroupsCached) {
+    // the block query needs only q: the summaries are read once the kernel before has completed
+    pdl_wait();
 
-  // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
-  // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
-  const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
-  const int nc1 = nch - nsc;
-  score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
-  if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
-  __syncthreads();
-  if (nc1 <= kRouteThreads)
-    block_select_topk_small(keys, nc1, kc, csel, scratch);
-  else
-    block_select_topk(keys, nc1, kc, csel, hist, scratch);
-  if (nsc) {
-    for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] += nsc;
+    // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
+    // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
+    const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
+    const int nc1 = nch - nsc;
+    score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
+    if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
     __syncthreads();
+    if (nc1 <= kRouteThreads)
+      block_select_topk_small(keys, nc1, kc, csel, scratch);
+    else
+      block_select_topk(keys, nc1, kc, csel, hist, scratch);
+    if (nsc) {
+      for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] += nsc;
+      __syncthreads();
+    }
+    if (MODE == kRouteChunks) {
+      for (int i = threadIdx.x; i < kc; i += kRouteThreads) chunk_idx[(int64_t)unit * kc + i] = csel[i];
+      if (threadIdx.x < kD) rc.qb[(int64_t)unit * kD + threadIdx.x] = qb[threadIdx.x];
+      return;
+    }
   }
 
-  // ---- level 2: the 8 groups of every selected chunk
-  const float* gs = group_sum + (int64_t)bkh * nch_stride * (kChunk / kGroup) * kD;
+  // ---- level 2: the 8 groups of every selected chunk, from the summary table or from the chunk's
+  // cache slot (a chunk that has none records HGA_ERR_ARG and reads slot 0)
   const int ncand = kc * (kChunk / kGroup);
-  score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
+  if (MODE == kRouteGroupsCached) {
+    const float* gc = rc.gcache + (int64_t)bkh * rc.cap * (kChunk / kGroup) * kD;
+    const int32_t* so = rc.slot_of + (int64_t)bkh * nch_stride;
+    const int cap = rc.cap;
+    int* st = rc.status;
+    score_rows(qb, gc, ncand,
+               [csel, so, cap, st](int c) {
+                 int slot = __ldg(so + csel[c >> 3]);
+                 if (slot < 0 || slot >= cap) {
+                   set_status(st, -1);
+                   slot = 0;
+                 }
+                 return slot * 8 + (c & 7);
+               },
+               keys);
+  } else {
+    const float* gs = group_sum + (int64_t)bkh * nch_stride * (kChunk / kGroup) * kD;
+    score_rows(qb, gs, ncand, [csel](int c) { return csel[c >> 3] * 8 + (c & 7); }, keys);
+  }
   if (threadIdx.x < 4 && ncand + (int)threadIdx.x < ((ncand + 3) & ~3)) keys[ncand + threadIdx.x] = 0u;
   __syncthreads();
   if (ncand <= kRouteThreads)
@@ -314,30 +360,56 @@ size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
   return words * 4;
 }
 
+template <typename T, int MODE>
+static cudaError_t launch_route_t(const void* q, const void* q_prev, bool causal, const float* group_sum,
+                                  const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq,
+                                  int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, size_t smem,
+                                  const RouteCache& rc, cudaStream_t stream) {
+  const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
+  if (units == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(route_kernel<T, MODE>, dim3((unsigned)units), dim3(kRouteThreads), smem, stream, 1,
+                       static_cast<const T*>(q), static_cast<const T*>(q_prev), causal ? 1 : 0, group_sum, chunk_sum,
+                       chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg, rc);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
                          int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream) {
-  const int64_t units = (int64_t)B * Hkv * (S / kQBlock);
-  if (units == 0) return cudaSuccess;
   const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
-  cudaError_t e;
-  if (bf16) {
-    e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(route_kernel<__nv_bfloat16>, dim3((unsigned)units), dim3(kRouteThreads), smem, stream, 1,
-                         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(q_prev),
-                         causal ? 1 : 0, group_sum, chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc,
-                         kc, kg);
-    if (e != cudaSuccess) return e;
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(route_kernel<float>, dim3((unsigned)units), dim3(kRouteThreads), smem, stream, 1,
-                         static_cast<const float*>(q), static_cast<const float*>(q_prev), causal ? 1 : 0, group_sum,
-                         chunk_sum, chunk_idx, group_idx, Hq, Hkv, S, nch, nch_stride, nsc, kc, kg);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaGetLastError();
+  const RouteCache rc{nullptr, nullptr, nullptr, 0, nullptr};
+  return bf16 ? launch_route_t<__nv_bfloat16, kRouteFull>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq, Hkv,
+                                              S, nch, nch_stride, nsc, kc, kg, smem, rc, stream)
+              : launch_route_t<float, kRouteFull>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq,
+                                                  Hkv, S, nch, nch_stride, nsc, kc, kg, smem, rc, stream);
+}
+
+// Level 1 only: chunk_idx and the block queries qb [B, Hkv, S/64, 128] float32.
+cudaError_t launch_route_chunks(bool bf16, const void* q, const void* q_prev, bool causal, const float* chunk_sum,
+                                int32_t* chunk_idx, float* qb, int B, int Hq, int Hkv, int64_t S, int nch,
+                                int nch_stride, int nsc, int kc, cudaStream_t stream) {
+  const size_t smem = route_smem_bytes(bf16, nch, kc, 1);
+  const RouteCache rc{qb, nullptr, nullptr, 0, nullptr};
+  return bf16 ? launch_route_t<__nv_bfloat16, kRouteChunks>(q, q_prev, causal, nullptr, chunk_sum, chunk_idx, nullptr, B, Hq, Hkv, S,
+                                              nch, nch_stride, nsc, kc, 1, smem, rc, stream)
+              : launch_route_t<float, kRouteChunks>(q, q_prev, causal, nullptr, chunk_sum, chunk_idx, nullptr, B, Hq,
+                                                    Hkv, S, nch, nch_stride, nsc, kc, 1, smem, rc, stream);
+}
+
+// Level 2 from the group-summary cache: group_idx from the block queries and chunk_idx of level 1.
+cudaError_t launch_route_groups_cached(const float* qb, const int32_t* chunk_idx, const int32_t* slot_of,
+                                       const float* gcache, int cap, int32_t* group_idx, int B, int Hkv, int64_t S,
+                                       int nch_stride, int kc, int kg, int* status, cudaStream_t stream) {
+  // the kernel's shared memory holds keys for 8 kc candidates; no chunk level runs
+  const size_t smem = route_smem_bytes(false, 1, kc, kg);
+  const RouteCache rc{const_cast<float*>(qb), slot_of, gcache, cap, status};
+  // q is not read in this mode: any valid element type; Hq = Hkv (G = 1) keeps the unused block-query
+  // arithmetic trivially in range
+  return launch_route_t<float, kRouteGroupsCached>(qb, nullptr, false, nullptr, nullptr, const_cast<int32_t*>(chunk_idx), group_idx, B, Hkv,
+                               Hkv, S, 1, nch_stride, 0, kc, kg, smem, rc, stream);
 }
 
 }  // namespace hga

@@ -303,6 +303,57 @@ HGA_API int hga_tier_gather(const hga_config_t* cfg, const void* k_hist, const v
                             const int32_t* used_groups, const int32_t* n_used, void* k_cache,
                             void* v_cache, void* stream);
 
+/* ---------------------------------------------------------------- group-summary cache
+ * The middle tier of the tiered storage ("Technical Summary" 2.1 "Group Selection":
+ * group summaries are cached in device memory and the missing ones are fetched from
+ * host memory; 2.2: the chunk summaries stay resident; pith.science review, Figure 1
+ * caption): routing in two levels with the group summaries of a long history in host
+ * memory and a device cache of cap_chunks slots per (batch, KV head), each slot
+ * holding the 8 group summaries (8 x D float32, 4 KB) of one chunk.  Per step:
+ *   1. hga_route_chunks: level 1 -> chunk_idx, and the block queries qb;
+ *   2. hga_gcache_plan: hits refresh their slots; the chosen chunks without a slot take
+ *      the least recently used slots holding no chosen chunk; writes the miss list;
+ *   3. hga_gcache_fetch: copies the missed chunks' group summaries into their slots;
+ *   4. hga_route_groups_cached: level 2 from the slots -> group_idx.
+ * The summaries are the same float32 values, so chunk_idx and group_idx equal those of
+ * hga_route bit for bit.  A cache of at least min(chunks outside the sink, (S/64) *
+ * top_chunks) slots always holds a step's chosen chunks; a smaller one records
+ * HGA_ERR_ARG in the workspace status word when a step needs more.
+ * Cache state (device int32, owned by the caller, initialised once to -1 everywhere):
+ *   slot_of  [B, Hkv, hist_capacity/64]  slot of each chunk (-1: not cached)
+ *   chunk_of [B, Hkv, cap_chunks]        chunk held by each slot (-1: empty)
+ *   stamp    [B, Hkv, cap_chunks]        step that last used each slot (-1: never)
+ * Per-step buffers (device int32): miss_chunk, miss_slot [B, Hkv, cap_chunks];
+ * counts [B*Hkv, 2] = (hits, misses) of the step.  qb [B, Hkv, S/64, D] float32;
+ * gcache [B, Hkv, cap_chunks, 8, D] float32.  1 <= cap_chunks <= 4096. */
+
+/* Level 1 of hga_route (chunk selection) only: chunk_idx as hga_route writes it, and
+ * the block query of every (batch, KV head, block) into qb. */
+HGA_API int hga_route_chunks(const hga_config_t* cfg, const void* q, const float* chunk_sum,
+                             int32_t* chunk_idx, float* qb, void* workspace, void* stream);
+
+/* The cache plan of one step (`step` increases by one per step and is stored in the
+ * stamps).  Needs the workspace for its status word. */
+HGA_API int hga_gcache_plan(const hga_config_t* cfg, int32_t cap_chunks, const int32_t* chunk_idx,
+                            int32_t* slot_of, int32_t* chunk_of, int32_t* stamp, int32_t step,
+                            int32_t* miss_chunk, int32_t* miss_slot, int32_t* counts,
+                            void* workspace, void* stream);
+
+/* Copies the 8 group summaries of every missed chunk from group_sum_src [B, Hkv,
+ * hist_capacity/8, D] float32 -- pinned host memory mapped into the device address space
+ * (the SMs read it over the host link) or device memory; pageable host memory is
+ * rejected with HGA_ERR_ARG -- into their slots of gcache. */
+HGA_API int hga_gcache_fetch(const hga_config_t* cfg, int32_t cap_chunks, const float* group_sum_src,
+                             const int32_t* miss_chunk, const int32_t* miss_slot, const int32_t* counts,
+                             float* gcache, void* stream);
+
+/* Level 2 of hga_route (group selection) from the cache: group_idx as hga_route writes
+ * it, from qb and chunk_idx of hga_route_chunks and the group summaries in gcache.  A
+ * chosen chunk without a slot records HGA_ERR_ARG in the workspace status word. */
+HGA_API int hga_route_groups_cached(const hga_config_t* cfg, const float* qb, const int32_t* chunk_idx,
+                                    const int32_t* slot_of, int32_t cap_chunks, const float* gcache,
+                                    int32_t* group_idx, void* workspace, void* stream);
+
 /* Synchronises `stream`, copies the workspace status word to *status_out
  * (HGA_OK, HGA_ERR_TIMEOUT or HGA_ERR_ARG, see Workspace above) and clears it.  Returns HGA_ERR_CUDA if the
  * copy itself fails. */

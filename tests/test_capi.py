@@ -175,3 +175,29 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
         C.load()
     with pytest.raises(RuntimeError, match="missing"):
         C.workspace_size(cfg())
+
+
+def test_group_cache_entry_points_validate_before_launch(lib):
+    """The group-summary cache calls reject a slot count outside [1, min(4096, history chunks)] and
+    missing pointers or workspace before anything is launched."""
+    c = cfg()                                       # 224 history chunks
+    ok = 1 << 20
+    for cap in (0, -1, 225, 5000):
+        with pytest.raises(C.HGAError) as e:
+            C.gcache_plan(c, cap, ok, ok, ok, ok, 0, ok, ok, ok, ok)
+        assert e.value.code == C.HGA_ERR_ARG, cap
+        with pytest.raises(C.HGAError) as e:
+            C.route_groups_cached(c, ok, ok, ok, cap, ok, ok, ok)
+        assert e.value.code == C.HGA_ERR_ARG, cap
+    with pytest.raises(C.HGAError) as e:
+        C.gcache_plan(c, 16, ok, ok, ok, ok, 0, ok, ok, ok, None)
+    assert e.value.code == C.HGA_ERR_WORKSPACE
+    with pytest.raises(C.HGAError) as e:
+        C.route_groups_cached(c, ok, ok, ok, 16, ok, ok, None)
+    assert e.value.code == C.HGA_ERR_WORKSPACE
+    with pytest.raises(C.HGAError) as e:
+        C.route_chunks(c, ok, ok, ok, None, None)      # no block-query buffer
+    assert e.value.code == C.HGA_ERR_ARG
+    with pytest.raises(C.HGAError) as e:
+        C.gcache_fetch(c, 16, ok, None, ok, ok, ok)
+    assert e.value.code == C.HGA_ERR_ARG

@@ -509,6 +509,22 @@ def test_parity_seeds_have_routing_margins(oracle, name):
         assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
 
 
+@pytest.mark.parametrize("name,q_seeds", [("gcache_small", [0, 1, 2, 3, 4, 5]), ("ctx16k", [0, 2, 1])])
+def test_cache_test_steps_have_routing_margins(oracle, name, q_seeds):
+    """The group-summary cache tests route the queries of several seeds against the history of seed
+    0; every such step has the same margins as the other parity inputs."""
+    w = (HI.Workload("gcache_small", 2, 8, 2, 128, 4096, 256, 4, 16, "bf16", 1.0) if name == "gcache_small"
+         else HI.WORKLOADS[name])
+    kh = HI.make_inputs(w, 0)["k_hist"]
+    for s in q_seeds:
+        q = HI.make_inputs(w, s)["q"]
+        r32 = oracle.route_from_inputs(q, kh, w.Hkv, w.top_chunks, w.top_groups, prec=32)
+        r64 = oracle.route_from_inputs(q, kh, w.Hkv, w.top_chunks, w.top_groups, prec=64)
+        assert np.array_equal(r32["chunk_idx"], r64["chunk_idx"])
+        assert np.array_equal(r32["group_idx"], r64["group_idx"])
+        assert r64["chunk_gap"].min() >= MIN_GAP and r64["group_gap"].min() >= MIN_GAP
+
+
 @pytest.mark.parametrize("name", ["small_bf16", "sink_bf16", "ctx16k"])
 def test_causal_parity_inputs_have_routing_margins(oracle, name):
     """Block 0 of the causal routing in the GPU tests is routed with a separately drawn previous
