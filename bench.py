@@ -603,7 +603,7 @@ def main():
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             tr = json.load(f).get(f"{w.name}:{dom}")
-        if tr and tr.get("kernel_source_sha") == _kernel_sha():
+        if tr and tr.get("kernel_source_sha") == _kernel_sha(dom):
             traffic = tr["dram_bytes_per_launch"]
     except (OSError, ValueError):
         pass
@@ -731,11 +731,23 @@ def main():
         dist.destroy_process_group()
 
 
-def _kernel_sha() -> str:
+# The sources each timed kernel is compiled from (its file, the shared device helpers it includes).
+KERNEL_SOURCES = {
+    "summaries": ("summaries.cu", "common.cuh"),
+    "route": ("route.cu", "common.cuh"),
+    "attn_fwd": ("attn_tc_fwd.cu", "tc_common.cuh", "common.cuh"),
+    "bwd_dq": ("attn_tc_bwd.cu", "tc_common.cuh", "common.cuh"),
+    "bwd_dkdv": ("attn_tc_bwd.cu", "tc_common.cuh", "common.cuh"),
+}
+
+
+def _kernel_sha(kernel: str) -> str:
+    """Hash of the sources of one kernel: a DRAM-traffic record in profiles/traffic.json is used
+    only while this matches the hash stored with it."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_kv_routing_tok_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
