@@ -489,6 +489,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
     calls = step.calls(x, stream.cuda_stream)
     names = [n for n, _ in calls]
+    # the routing call launches one kernel, or three for a long history (block queries, chunk scores
+    # of all blocks at once, selection + group level)
+    launches_per_step = len(calls) - 1 + H._capi.route_launches(cfg, with_workspace=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     drain = torch.ones(L2_DRAIN_BYTES // 4, dtype=torch.float32, device=dev)
     drain_out = torch.empty((), dtype=torch.float32, device=dev)
@@ -708,11 +711,12 @@ def main():
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
                 "config": _config(w, args), "roofline": roofline, "method_frac": method["frac_burst"],
                 "method_roofline": method, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": K * len(calls), "clocks": clk.summary(),
+                "gpu_launches": K * launches_per_step, "clocks": clk.summary(),
                 "step_launch": "one CUDA graph replay per step: the step's kernels and their dependent "
                                "launches, captured once through the C ABI (the per-kernel pass launches "
                                "them one by one)",
-                "kernels_per_step": names}
+                "kernels_per_step": names,
+                "route_launches": launches_per_step - (len(calls) - 1)}
         if incremental:
             line["incremental_summaries"] = incremental
         if positions:

@@ -26,7 +26,7 @@ HGA_F32 = 0
 HGA_BF16 = 1
 
 #: every entry point declared in include/hga.h
-EXPORTS = ("hga_workspace_size", "hga_build_summaries", "hga_append_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
+EXPORTS = ("hga_workspace_size", "hga_route_launches", "hga_build_summaries", "hga_append_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd",
            "hga_attn_bwd",
            "hga_attn_bwd_preprocess", "hga_attn_bwd_dkdv", "hga_attn_bwd_dq", "hga_attn_bwd_noalloc",
            "hga_noalloc_read_status", "hga_tier_cache_config", "hga_route_chunks", "hga_gcache_plan",
@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
     P, C = ctypes.c_void_p, ctypes.POINTER(HGAConfig)
     sig = {
         "hga_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
+        "hga_route_launches": [C, ctypes.c_int, ctypes.POINTER(ctypes.c_int32)],
         "hga_build_summaries": [C, P, P, P, P, P],
         "hga_append_summaries": [C, P, P, P, ctypes.c_int64, P, P],
         "hga_route": [C, P, P, P, P, P, P, P],
@@ -118,6 +119,12 @@ def make_config(B: int, Hq: int, Hkv: int, hist_len: int, seg_len: int, top_chun
                 wait_limit_ns: int = 0) -> HGAConfig:
     return HGAConfig(B, Hq, Hkv, D, hist_len, seg_len, chunk, group, qblock, top_chunks, top_groups,
                      n_sink_tokens, dtype, softmax_scale, hist_capacity, wait_limit_ns)
+
+
+def route_launches(cfg: HGAConfig, with_workspace: bool = True) -> int:
+    out = ctypes.c_int32()
+    _call("hga_route_launches", ctypes.byref(cfg), 1 if with_workspace else 0, ctypes.byref(out))
+    return out.value
 
 
 def workspace_size(cfg: HGAConfig) -> int:

@@ -12,6 +12,11 @@
 namespace hga {
 cudaError_t launch_summaries(bool bf16, const void* k_hist, float* group_sum, float* chunk_sum, int64_t BHkv,
                              int64_t Hs, int64_t c0, int64_t c1, cudaStream_t stream);
+size_t route_split_bytes(int64_t units, int64_t nblk, int nch, int nsc);
+cudaError_t launch_route_split(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
+                               const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq,
+                               int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, void* scratch,
+                               cudaStream_t stream);
 cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
                          int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream);
@@ -177,7 +182,18 @@ size_t base_workspace_bytes(const hga_config_t* c) { return hga::kStatusBytes + 
 size_t xchg_bytes(const hga_config_t* c) {
   return use_tc(c) ? hga::dkdv_xchg_bytes(c->B, c->Hq, c->Hkv, c->seg_len) : 0;
 }
-size_t full_workspace_bytes(const hga_config_t* c) { return base_workspace_bytes(c) + xchg_bytes(c); }
+// Scratch of the three-launch routing of long histories (block queries and chunk scores; 0 when the
+// history is short enough for the single launch).  Routing and the dK/dV kernel never run at once on
+// a workspace, so the two share the region after the status word and the delta rows.
+size_t route_bytes(const hga_config_t* c) {
+  const int64_t nblk = c->seg_len / c->qblock;
+  return hga::route_split_bytes((int64_t)c->B * c->Hkv * nblk, nblk, (int)(c->hist_len / c->chunk),
+                                (int)(c->n_sink_tokens / c->chunk));
+}
+size_t full_workspace_bytes(const hga_config_t* c) {
+  const size_t x = xchg_bytes(c), r = route_bytes(c);
+  return base_workspace_bytes(c) + (x > r ? x : r);
+}
 float* xchg_of(void* workspace, const hga_config_t* c, size_t ws_bytes) {
   const size_t x = xchg_bytes(c);
   if (x == 0 || ws_bytes < base_workspace_bytes(c) + x) return nullptr;
@@ -282,6 +298,14 @@ int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out) {
   return HGA_OK;
 }
 
+int hga_route_launches(const hga_config_t* cfg, int with_workspace, int32_t* launches_out) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!launches_out) return HGA_ERR_ARG;
+  *launches_out = cfg->hist_len == 0 ? 0 : (with_workspace && route_bytes(cfg) > 0) ? 3 : 1;
+  return HGA_OK;
+}
+
 int hga_build_summaries(const hga_config_t* cfg, const void* k_hist, float* group_sum, float* chunk_sum,
                         void* workspace, void* stream) {
   int rc = check_config(cfg);
@@ -310,13 +334,21 @@ int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum, co
   int rc = check_config(cfg);
   if (rc) return rc;
   if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
-  (void)workspace;
   if (cfg->hist_len == 0) return HGA_OK;        // nothing to route
   if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
+  const int nch = (int)(cfg->hist_len / cfg->chunk), nsc = (int)(cfg->n_sink_tokens / cfg->chunk);
+  if (workspace && route_bytes(cfg) > 0) {
+    if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+    return from_cuda(hga::launch_route_split(cfg->dtype == HGA_BF16, q, nullptr, false, group_sum, chunk_sum, chunk_idx,
+                                             group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len, nch,
+                                             (int)(hist_rows(cfg) / cfg->chunk), nsc, cfg->top_chunks,
+                                             cfg->top_groups,
+                                             static_cast<char*>(workspace) + base_workspace_bytes(cfg),
+                                             static_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, nullptr, false, group_sum, chunk_sum, chunk_idx,
-                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
-                                     (int)(cfg->hist_len / cfg->chunk), (int)(hist_rows(cfg) / cfg->chunk),
-                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
+                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len, nch,
+                                     (int)(hist_rows(cfg) / cfg->chunk), nsc, cfg->top_chunks, cfg->top_groups,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -326,13 +358,21 @@ int hga_route_causal(const hga_config_t* cfg, const void* q, const void* q_prev,
   if (rc) return rc;
   if ((rc = check_ptrs({q, group_sum, chunk_sum}))) return rc;
   if (q_prev && !aligned16(q_prev)) return HGA_ERR_ALIGN;
-  (void)workspace;
   if (cfg->hist_len == 0) return HGA_OK;        // nothing to route
   if ((rc = check_idx({chunk_idx, group_idx}))) return rc;
+  const int nch = (int)(cfg->hist_len / cfg->chunk), nsc = (int)(cfg->n_sink_tokens / cfg->chunk);
+  if (workspace && route_bytes(cfg) > 0) {
+    if (!aligned16(workspace)) return HGA_ERR_ALIGN;
+    return from_cuda(hga::launch_route_split(cfg->dtype == HGA_BF16, q, q_prev, true, group_sum, chunk_sum, chunk_idx,
+                                             group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len, nch,
+                                             (int)(hist_rows(cfg) / cfg->chunk), nsc, cfg->top_chunks,
+                                             cfg->top_groups,
+                                             static_cast<char*>(workspace) + base_workspace_bytes(cfg),
+                                             static_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(hga::launch_route(cfg->dtype == HGA_BF16, q, q_prev, true, group_sum, chunk_sum, chunk_idx,
-                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len,
-                                     (int)(cfg->hist_len / cfg->chunk), (int)(hist_rows(cfg) / cfg->chunk),
-                                     (int)(cfg->n_sink_tokens / cfg->chunk), cfg->top_chunks, cfg->top_groups,
+                                     group_idx, cfg->B, cfg->Hq, cfg->Hkv, cfg->seg_len, nch,
+                                     (int)(hist_rows(cfg) / cfg->chunk), nsc, cfg->top_chunks, cfg->top_groups,
                                      static_cast<cudaStream_t>(stream)));
 }
 

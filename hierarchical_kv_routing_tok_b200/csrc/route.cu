@@ -17,11 +17,21 @@
 // summaries (the group summaries of a long history in host memory, "Technical Summary" 2.1 Group
 // Selection): mode 1 stops after level 1 and writes the chunk indices and the block query; mode 2
 // starts from those and scores the group summaries of the chosen chunks from their cache slots.
+//
+// Long histories route in three launches instead of one, so that each chunk summary is read once
+// per (batch, KV head) rather than once per query block: mode 3 forms the block queries;
+// chunk_score_kernel scores every chunk of a (batch, KV head) against all of its block queries (a
+// warp per chunk row, the row in registers, the block queries in shared memory); mode 4 selects
+// each block's chunks from its row of scores and runs level 2 as mode 0 does.
 #include "common.cuh"
 
 namespace hga {
 
 constexpr int kRouteThreads = 512;
+// Candidates up to which a level selects by rank counting (n^2 / threads comparisons per thread);
+// above it the radix select (four 8-bit passes) is cheaper: routing 384 chunks took 24.6 us with
+// the radix select against 30.7 with rank counting (B200, one launch, summaries not in L2).
+constexpr int kRankSelectMax = 256;
 constexpr int kScratchInts = 32;   // warp totals (16) + broadcast slots
 
 // Larger score -> larger key; +0 and -0 map to the same key.
@@ -196,13 +206,15 @@ __device__ __forceinline__ void score_rows(const float* qb, const float* __restr
 }
 
 // Routing modes and the inputs / outputs of the cached group level.
-enum RouteMode { kRouteFull = 0, kRouteChunks = 1, kRouteGroupsCached = 2 };
+enum RouteMode { kRouteFull = 0, kRouteChunks = 1, kRouteGroupsCached = 2, kRouteQuery = 3, kRouteFromScores = 4 };
 struct RouteCache {
-  float* qb;                // [units][128] block queries: written in mode 1, read in mode 2
+  float* qb;                // [units][128] block queries: written in modes 1 and 3, read in modes 2 and 4
   const int32_t* slot_of;   // mode 2: [B*Hkv][nch_stride] cache slot of each chunk (-1: not cached)
   const float* gcache;      // mode 2: [B*Hkv][cap][8][128] group summaries of the cached chunks
   int cap;                  // mode 2: cache slots per (batch, KV head)
   int* status;              // mode 2: a chosen chunk missing from the cache records HGA_ERR_ARG here
+  const uint32_t* scores;   // mode 4: [units][nc_pad] order keys of the chunk scores (chunk_score_kernel)
+  int nc_pad;               // mode 4: row stride of `scores`
 };
 
 template <typename T, int MODE>
@@ -253,6 +265,13 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     if (threadIdx.x < kD) qb[threadIdx.x] = rc.qb[(int64_t)unit * kD + threadIdx.x];
     for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] = chunk_idx[(int64_t)unit * kc + i];
     __syncthreads();
+  } else if (MODE == kRouteFromScores) {
+    // the block query (mode 3) and this block's row of chunk scores (chunk_score_kernel)
+    pdl_wait();
+    if (threadIdx.x < kD) qb[threadIdx.x] = rc.qb[(int64_t)unit * kD + threadIdx.x];
+    const uint4* src = reinterpret_cast<const uint4*>(rc.scores + (int64_t)unit * rc.nc_pad);
+    for (int i = threadIdx.x; i < rc.nc_pad / 4; i += kRouteThreads) reinterpret_cast<uint4*>(keys)[i] = src[i];
+    __syncthreads();
   } else {
     const int tid = threadIdx.x;
     const int col = (tid % LPR) * N, r0 = tid / LPR;
@@ -291,20 +310,27 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
       qb[tid] = s / (float)R;
     }
     __syncthreads();
+    if (MODE == kRouteQuery) {
+      if (tid < kD) rc.qb[(int64_t)unit * kD + tid] = qb[tid];
+      pdl_wait();   // completes only after the kernel before: the launch chain keeps its order
+      return;
+    }
   }
 
   if (MODE != kRouteGroupsCached) {
-    // the block query needs only q: the summaries are read once the kernel before has completed
-    pdl_wait();
-
-    // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
-    // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
-    const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
     const int nc1 = nch - nsc;
-    score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
-    if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
-    __syncthreads();
-    if (nc1 <= kRouteThreads)
+    if (MODE != kRouteFromScores) {
+      // the block query needs only q: the summaries are read once the kernel before has completed
+      pdl_wait();
+
+      // ---- level 1: the chunks outside the sink window (the first nsc chunks are always attended
+      // and never routed); candidate i is chunk nsc + i, so lower position = lower chunk index
+      const float* cs = chunk_sum + (int64_t)bkh * nch_stride * kD;   // summary buffers hold nch_stride chunks
+      score_rows(qb, cs, nc1, [nsc](int i) { return nsc + i; }, keys);
+      if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
+      __syncthreads();
+    }
+    if (nc1 <= kRankSelectMax)
       block_select_topk_small(keys, nc1, kc, csel, scratch);
     else
       block_select_topk(keys, nc1, kc, csel, hist, scratch);
@@ -343,7 +369,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   }
   if (threadIdx.x < 4 && ncand + (int)threadIdx.x < ((ncand + 3) & ~3)) keys[ncand + threadIdx.x] = 0u;
   __syncthreads();
-  if (ncand <= kRouteThreads)
+  if (ncand <= kRankSelectMax)
     block_select_topk_small(keys, ncand, kg, gpos, scratch);
   else
     block_select_topk(keys, ncand, kg, gpos, hist, scratch);
@@ -380,7 +406,7 @@ cudaError_t launch_route(bool bf16, const void* q, const void* q_prev, bool caus
                          const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq, int Hkv,
                          int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, cudaStream_t stream) {
   const size_t smem = route_smem_bytes(bf16, nch, kc, kg);
-  const RouteCache rc{nullptr, nullptr, nullptr, 0, nullptr};
+  const RouteCache rc{nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0};
   return bf16 ? launch_route_t<__nv_bfloat16, kRouteFull>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq, Hkv,
                                               S, nch, nch_stride, nsc, kc, kg, smem, rc, stream)
               : launch_route_t<float, kRouteFull>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq,
@@ -392,7 +418,7 @@ cudaError_t launch_route_chunks(bool bf16, const void* q, const void* q_prev, bo
                                 int32_t* chunk_idx, float* qb, int B, int Hq, int Hkv, int64_t S, int nch,
                                 int nch_stride, int nsc, int kc, cudaStream_t stream) {
   const size_t smem = route_smem_bytes(bf16, nch, kc, 1);
-  const RouteCache rc{qb, nullptr, nullptr, 0, nullptr};
+  const RouteCache rc{qb, nullptr, nullptr, 0, nullptr, nullptr, 0};
   return bf16 ? launch_route_t<__nv_bfloat16, kRouteChunks>(q, q_prev, causal, nullptr, chunk_sum, chunk_idx, nullptr, B, Hq, Hkv, S,
                                               nch, nch_stride, nsc, kc, 1, smem, rc, stream)
               : launch_route_t<float, kRouteChunks>(q, q_prev, causal, nullptr, chunk_sum, chunk_idx, nullptr, B, Hq,
@@ -405,11 +431,139 @@ cudaError_t launch_route_groups_cached(const float* qb, const int32_t* chunk_idx
                                        int nch_stride, int kc, int kg, int* status, cudaStream_t stream) {
   // the kernel's shared memory holds keys for 8 kc candidates; no chunk level runs
   const size_t smem = route_smem_bytes(false, 1, kc, kg);
-  const RouteCache rc{const_cast<float*>(qb), slot_of, gcache, cap, status};
+  const RouteCache rc{const_cast<float*>(qb), slot_of, gcache, cap, status, nullptr, 0};
   // q is not read in this mode: any valid element type; Hq = Hkv (G = 1) keeps the unused block-query
   // arithmetic trivially in range
   return launch_route_t<float, kRouteGroupsCached>(qb, nullptr, false, nullptr, nullptr, const_cast<int32_t*>(chunk_idx), group_idx, B, Hkv,
                                Hkv, S, 1, nch_stride, 0, kc, kg, smem, rc, stream);
+}
+
+// ---- chunk scores of all block queries of a (batch, KV head), for the three-launch routing
+constexpr int kScoreWarps = 8;
+constexpr int kScoreRowsPerWarp = 4;
+
+// Grid (B*Hkv, row slices).  Warp w of CTA (bkh, y) scores chunk rows nsc + i, i = (y * 8 + w) * 4 ..
+// + 3, against the block queries qb[bkh*nblk .. + nblk) (shared memory): lane l holds dims 4l .. 4l+3
+// of the row, multiplies them with the same dims of 32 block queries at a time, and a recursive-
+// halving exchange over the lanes leaves lane b with the full dot product of block b.  Writes the
+// order keys to scores[(bkh*nblk + blk) * nc_pad + i]; the pad entries [nc1, nc_pad) get 0, which
+// every score precedes.
+__global__ void __launch_bounds__(kScoreWarps * 32) chunk_score_kernel(const float* __restrict__ qb_all,
+                                                                      const float* __restrict__ chunk_sum,
+                                                                      uint32_t* __restrict__ scores, int nblk,
+                                                                      int nch_stride, int nsc, int nc1, int nc_pad) {
+  extern __shared__ __align__(16) float qs[];   // [nblk rounded up to 32][128]
+  if (threadIdx.x == 0) pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t bkh = blockIdx.x;
+  const int nb32 = (nblk + 31) & ~31;
+  pdl_wait();   // the block queries come from the kernel before, the summaries from the one before it
+  {
+    const float4* src = reinterpret_cast<const float4*>(qb_all + bkh * nblk * kD);
+    float4* dst = reinterpret_cast<float4*>(qs);
+    for (int i = threadIdx.x; i < nb32 * (kD / 4); i += blockDim.x)
+      dst[i] = i < nblk * (kD / 4) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  const int i0 = ((int)blockIdx.y * kScoreWarps + warp) * kScoreRowsPerWarp;
+  float4 row[kScoreRowsPerWarp];
+  const float* cs = chunk_sum + (bkh * nch_stride + nsc) * kD;
+#pragma unroll
+  for (int r = 0; r < kScoreRowsPerWarp; ++r)
+    row[r] = i0 + r < nc1 ? __ldg(reinterpret_cast<const float4*>(cs + (int64_t)(i0 + r) * kD) + lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  uint32_t* out = scores + bkh * nblk * (int64_t)nc_pad;
+  for (int g = 0; g < nb32; g += 32) {
+    // each block query's 16 bytes are read once for the warp's four rows
+    float p[kScoreRowsPerWarp][32];
+#pragma unroll
+    for (int b = 0; b < 32; ++b) {
+      const float4 q4 = reinterpret_cast<const float4*>(qs + (g + b) * kD)[lane];
+#pragma unroll
+      for (int r = 0; r < kScoreRowsPerWarp; ++r)
+        p[r][b] = q4.x * row[r].x + q4.y * row[r].y + q4.z * row[r].z + q4.w * row[r].w;
+    }
+#pragma unroll
+    for (int r = 0; r < kScoreRowsPerWarp; ++r) {
+      // recursive halving: after the step with offset o, lane l keeps the o blocks whose index has
+      // bit log2(o) equal to that bit of l, summed over lane pairs l, l ^ o; at the end lane b holds
+      // block b's sum over all 32 lanes
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < o; ++k) {
+          const float send = upper ? p[r][k] : p[r][k + o];
+          const float keep = upper ? p[r][k + o] : p[r][k];
+          p[r][k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      const int i = i0 + r, blk = g + lane;
+      if (blk < nblk) {
+        if (i < nc1) out[(int64_t)blk * nc_pad + i] = order_key(p[r][0]);
+        else if (i < nc_pad) out[(int64_t)blk * nc_pad + i] = 0u;
+      }
+    }
+  }
+}
+
+// Chunks (outside the sink window) from which routing runs in three launches when the caller passes
+// a workspace.  Measured on B200 (B = 1, 8 KV heads, 32 blocks, 16 / 64 routed chunks / groups, 32 /
+// 128 at 2016 chunks; summaries not in L2), one launch against three: 224 chunks 22.6 against
+// 25.6 us, 512 26.7 against 25.6, 1024 34.8 against 29.8, 2016 55.3 against 44.0.
+constexpr int kSplitMinChunks = 512;
+
+// chunk_score_kernel keeps all block queries of a (batch, KV head) in shared memory
+constexpr size_t kScoreSmemMax = 200 * 1024;
+
+int route_split_nc_pad(int nch, int nsc) { return ((nch - nsc) + 3) & ~3; }
+bool route_uses_split(int64_t nblk, int nch, int nsc) {
+  return nch - nsc >= kSplitMinChunks && (size_t)((nblk + 31) & ~31) * kD * sizeof(float) <= kScoreSmemMax;
+}
+// units = B * Hkv * nblk
+size_t route_split_bytes(int64_t units, int64_t nblk, int nch, int nsc) {
+  if (!route_uses_split(nblk, nch, nsc)) return 0;
+  return (size_t)units * kD * sizeof(float) + (size_t)units * route_split_nc_pad(nch, nsc) * sizeof(uint32_t);
+}
+
+// Three-launch routing with scratch = route_split_bytes(...) bytes (16-byte aligned): block queries,
+// chunk scores, selection + level 2.  Same outputs as launch_route.
+cudaError_t launch_route_split(bool bf16, const void* q, const void* q_prev, bool causal, const float* group_sum,
+                               const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx, int B, int Hq,
+                               int Hkv, int64_t S, int nch, int nch_stride, int nsc, int kc, int kg, void* scratch,
+                               cudaStream_t stream) {
+  const int64_t nblk = S / kQBlock;
+  const int64_t units = (int64_t)B * Hkv * nblk;
+  if (units == 0) return cudaSuccess;
+  const int nc1 = nch - nsc, nc_pad = route_split_nc_pad(nch, nsc);
+  float* qb = static_cast<float*>(scratch);
+  uint32_t* scores = reinterpret_cast<uint32_t*>(qb + units * kD);
+  // 1. block queries
+  RouteCache rc{qb, nullptr, nullptr, 0, nullptr, nullptr, 0};
+  cudaError_t e = bf16 ? launch_route_t<__nv_bfloat16, kRouteQuery>(q, q_prev, causal, nullptr, nullptr, nullptr, nullptr, B, Hq,
+                                                            Hkv, S, nch, nch_stride, nsc, kc, kg,
+                                                            route_smem_bytes(true, 1, 1, 1), rc, stream)
+                       : launch_route_t<float, kRouteQuery>(q, q_prev, causal, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv,
+                                                            S, nch, nch_stride, nsc, kc, kg,
+                                                            route_smem_bytes(false, 1, 1, 1), rc, stream);
+  if (e != cudaSuccess) return e;
+  // 2. chunk scores
+  const int rows_per_cta = kScoreWarps * kScoreRowsPerWarp;
+  const dim3 grid((unsigned)(B * Hkv), (unsigned)((nc_pad + rows_per_cta - 1) / rows_per_cta));
+  const size_t smem2 = (size_t)((nblk + 31) & ~31) * kD * sizeof(float);
+  e = cudaFuncSetAttribute(chunk_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(chunk_score_kernel, grid, dim3(kScoreWarps * 32), smem2, stream, 1,
+                       static_cast<const float*>(qb), chunk_sum, scores, (int)nblk, nch_stride, nsc, nc1, nc_pad);
+  if (e != cudaSuccess) return e;
+  // 3. selection from the scores, then level 2
+  rc.scores = scores;
+  rc.nc_pad = nc_pad;
+  const size_t smem3 = route_smem_bytes(bf16, nc_pad, kc, kg);
+  return bf16 ? launch_route_t<__nv_bfloat16, kRouteFromScores>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B,
+                                                        Hq, Hkv, S, nch, nch_stride, nsc, kc, kg, smem3, rc, stream)
+              : launch_route_t<float, kRouteFromScores>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq,
+                                                        Hkv, S, nch, nch_stride, nsc, kc, kg, smem3, rc, stream);
 }
 
 }  // namespace hga

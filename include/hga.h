@@ -131,6 +131,14 @@ typedef struct hga_config {
 /* Bytes of workspace the calls below need for this configuration. */
 HGA_API int hga_workspace_size(const hga_config_t* cfg, size_t* bytes_out);
 
+/* Kernels that one hga_route or hga_route_causal call launches for this
+ * configuration, given a workspace (with_workspace != 0) or not: 0 when
+ * hist_len = 0; 3 with a workspace and at least 512 routable chunks (chunks
+ * outside the sink window), as long as the S/64 block queries of a (batch, KV
+ * head) fit in 200 KB of shared memory; else 1.  For counting launches (a CUDA
+ * graph, a profiler's kernel filter); no device work. */
+HGA_API int hga_route_launches(const hga_config_t* cfg, int with_workspace, int32_t* launches_out);
+
 /* Summaries (Technical Summary 2.1, chunk and group selection; review,
  * Figure 1): group_sum[b,kh,j,:] = mean of history keys 8j..8j+7;
  * chunk_sum[b,kh,i,:] = mean of history keys 64i..64i+63.
@@ -158,7 +166,17 @@ HGA_API int hga_append_summaries(const hga_config_t* cfg, const void* k_hist, fl
  *   q          [B, Hq, S, D]               cfg->dtype  (in)
  *   group_sum, chunk_sum                   float32     (in, from above)
  *   chunk_idx  [B, Hkv, S/64, top_chunks]  int32       (out)
- *   group_idx  [B, Hkv, S/64, top_groups]  int32       (out) */
+ *   group_idx  [B, Hkv, S/64, top_groups]  int32       (out)
+ *   workspace  hga_workspace_size(cfg) bytes, 16-byte aligned, or NULL.
+ * With a workspace and a long history (hga_route_launches) the routing runs in
+ * three launches: the block queries; every chunk summary of a (batch, KV head)
+ * scored against all of its block queries in one pass (each summary read once
+ * per (batch, KV head), not once per block); then each block's selection and
+ * the group level.  The scores come from the same float32 operations in the
+ * same order as in the single launch, so the indices are the same bit for bit.
+ * The scratch shares the workspace region of the backward's dK/dV exchange
+ * area: the routing and a backward call must not run at the same time on one
+ * workspace.  Without a workspace: one launch. */
 HGA_API int hga_route(const hga_config_t* cfg, const void* q, const float* group_sum,
               const float* chunk_sum, int32_t* chunk_idx, int32_t* group_idx,
               void* workspace, void* stream);

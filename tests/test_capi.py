@@ -65,14 +65,22 @@ def cfg(**kw):
     return C.make_config(**base)
 
 
-def _expected_ws(B, Hq, Hkv, S, bf16=True, sms=148):
-    """Status word, delta rows, and (bf16 tensor-core path, fewer (batch, KV head, 128-key tile)
-    units than SMs: the dK/dV kernel pairs CTAs) one 2 x 64 KB exchange area per unit."""
+def _expected_ws(B, Hq, Hkv, S, bf16=True, sms=148, hist=14336, sink=0):
+    """Status word, delta rows, then one region shared by (a) the dK/dV exchange area (bf16
+    tensor-core path, fewer (batch, KV head, 128-key tile) units than SMs: the kernel pairs CTAs;
+    2 x 64 KB per unit) and (b) the scratch of the three-launch routing (at least 128 routable
+    chunks: a float32 block query and a row of chunk-score keys, padded to 4, per (batch, KV head,
+    block)); the region is the larger of the two."""
     r256 = lambda x: (x + 255) // 256 * 256
     delta = B * Hq * S * 4
     units = B * Hkv * ((S + 127) // 128)
     paired = bf16 and (Hq // Hkv) % 2 == 0 and units < sms
-    return 256 + r256(delta) + (units * 2 * 64 * 256 * 4 if paired else 0)
+    xchg = units * 2 * 64 * 256 * 4 if paired else 0
+    nblk, nc1 = S // 64, hist // 64 - sink // 64
+    blocks = B * Hkv * nblk
+    split = nc1 >= 512 and (nblk + 31) // 32 * 32 * 512 <= 200 * 1024
+    route = blocks * 128 * 4 + blocks * ((nc1 + 3) // 4 * 4) * 4 if split else 0
+    return 256 + r256(delta) + max(xchg, route)
 
 
 def test_workspace_size(lib):
@@ -81,8 +89,30 @@ def test_workspace_size(lib):
     assert C.workspace_size(cfg(B=3, Hq=4, Hkv=1, seg_len=64)) % 256 == 0
     # float32, odd G and many units: no exchange area
     assert C.workspace_size(cfg(dtype=C.HGA_F32)) == 256 + 1 * 32 * 2048 * 4
+    # a long history routes in three launches and needs routing scratch (a shorter one does not)
+    assert C.workspace_size(cfg(dtype=C.HGA_F32, hist_len=64 * 511)) == 256 + 1 * 32 * 2048 * 4
+    assert C.workspace_size(cfg(dtype=C.HGA_F32, hist_len=64 * 512)) == (
+        256 + 1 * 32 * 2048 * 4 + 8 * 32 * (128 + 512) * 4)
+    assert C.workspace_size(cfg(dtype=C.HGA_F32, hist_len=64 * 515, n_sink_tokens=64)) == _expected_ws(
+        1, 32, 8, 2048, bf16=False, hist=64 * 515, sink=64)
+    assert C.workspace_size(cfg(hist_len=64 * 2016)) == _expected_ws(1, 32, 8, 2048, hist=64 * 2016)
     assert C.workspace_size(cfg(Hq=24)) == _expected_ws(1, 24, 8, 2048, sms=0)
     assert C.workspace_size(cfg(B=4)) == _expected_ws(4, 32, 8, 2048, sms=0)
+
+
+def test_route_launches(lib):
+    """Three launches with a workspace and at least 512 routable chunks, one without a workspace or
+    for a shorter history (the 16K layer has 224 chunks), none without a history."""
+    long = dict(hist_len=64 * 2016, top_chunks=32, top_groups=128)
+    assert C.route_launches(cfg()) == 1
+    assert C.route_launches(cfg(**long)) == 3
+    assert C.route_launches(cfg(**long), with_workspace=False) == 1
+    assert C.route_launches(cfg(hist_len=64 * 511)) == 1
+    assert C.route_launches(cfg(hist_len=64 * 512)) == 3
+    assert C.route_launches(cfg(hist_len=64 * 512, n_sink_tokens=64)) == 1   # 511 routable
+    # the 400 block queries of a 25,600-token segment would need 208 KB of shared memory
+    assert C.route_launches(cfg(seg_len=64 * 400, **long)) == 1
+    assert C.route_launches(cfg(seg_len=64 * 384, **long)) == 3
 
 
 @pytest.mark.parametrize("kw,code", [
