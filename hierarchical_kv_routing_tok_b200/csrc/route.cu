@@ -149,30 +149,76 @@ __device__ void block_select_topk(const uint32_t* keys, int n, int k, int* out, 
 // (number of keys that precede it in the order "larger first, lower position first") by comparing
 // against broadcast 16-byte shared-memory reads of four keys at a time (keys[n..n4) hold 0, which
 // precedes nothing and is preceded by every score), keeps it if rank < k, and an index-ordered
-// scan of the kept flags writes the positions ascending.  One pass, two barriers.
-__device__ void block_select_topk_small(const uint32_t* keys, int n, int k, int* out, int* scratch) {
+// scan of the kept flags writes the positions ascending.  One pass, two barriers.  A key at a lower
+// position precedes key i when it is >= key i, one at a higher position when it is > key i: every
+// score's key is at least 1, so the four-key groups before i's own compare against ki - 1 and the
+// others against ki, and i's own group adds its earlier equal keys.
+__device__ void block_select_topk_small(const uint32_t* keys, int n, int k, int* out, int* scratch,
+                                        const int* pos_of = nullptr) {
   const int i = threadIdx.x;
   bool take = false;
   if (i < n) {
     const uint32_t ki = keys[i];
     const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-    const int n4 = (n + 3) >> 2;
+    const int n4 = (n + 3) >> 2, i4 = i >> 2;
     int rank = 0;
 #pragma unroll 4
     for (int j4 = 0; j4 < n4; ++j4) {
       const uint4 v = k4[j4];
-      const int j = 4 * j4;
-      rank += (v.x > ki) | ((v.x == ki) & (j < i));
-      rank += (v.y > ki) | ((v.y == ki) & (j + 1 < i));
-      rank += (v.z > ki) | ((v.z == ki) & (j + 2 < i));
-      rank += (v.w > ki) | ((v.w == ki) & (j + 3 < i));
+      const uint32_t thr = ki - (j4 < i4 ? 1u : 0u);
+      rank += (int)(v.x > thr) + (int)(v.y > thr) + (int)(v.z > thr) + (int)(v.w > thr);
     }
+    const uint4 v = k4[i4];
+    const int e = i & 3;
+    rank += (int)(e > 0 && v.x == ki) + (int)(e > 1 && v.y == ki) + (int)(e > 2 && v.z == ki);
     take = rank < k;
   }
   int tot;
   const int pos = block_exclusive_scan(take ? 1 : 0, scratch, &tot);
-  if (take) out[pos] = i;
+  if (take) out[pos] = pos_of ? pos_of[i] : i;
   __syncthreads();
+}
+
+// Select the k largest of keys[0..n) for k <= n, n > kRankSelectMax.  Every key >= T, T the least
+// of the maxima of k disjoint position ranges, is a candidate: each range holds a key >= T, so at
+// least k keys are >= T and the k largest (ties included) all are.  The candidates, compacted in
+// position order into ckeys / cpos, are ranked as in block_select_topk_small when there are at most
+// kRouteThreads of them (the order among them is the order among all keys); otherwise the radix
+// select runs on all n keys.  Writes the selected positions ascending to out[0..k).
+__device__ void block_select_topk_filtered(const uint32_t* keys, int n, int k, int* out, int* hist, int* scratch,
+                                           uint32_t* ckeys, int* cpos) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned* thr = reinterpret_cast<unsigned*>(hist);
+  if (tid == 0) *thr = 0xffffffffu;
+  __syncthreads();
+  for (int g = warp; g < k; g += kRouteThreads / 32) {
+    const int lo = (int)((int64_t)g * n / k), hi = (int)((int64_t)(g + 1) * n / k);
+    unsigned m = 0u;
+    for (int i = lo + lane; i < hi; i += 32) m = max(m, keys[i]);
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0) atomicMin(thr, m);
+  }
+  __syncthreads();
+  const unsigned T = *thr;
+  const int per = (n + kRouteThreads - 1) / kRouteThreads;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) cnt += keys[i] >= T;
+  int tot;
+  int pos = block_exclusive_scan(cnt, scratch, &tot);
+  if (tot > kRouteThreads) {                  // block-uniform
+    block_select_topk(keys, n, k, out, hist, scratch);
+    return;
+  }
+  for (int i = lo; i < hi; ++i)
+    if (keys[i] >= T) {
+      ckeys[pos] = keys[i];
+      cpos[pos] = i;
+      ++pos;
+    }
+  if (tid < 4 && tot + tid < ((tot + 3) & ~3)) ckeys[tot + tid] = 0u;
+  __syncthreads();
+  block_select_topk_small(ckeys, tot, k, out, scratch, cpos);
 }
 
 // Dot products of qb (smem, 128 floats) with `count` rows of a float32 [*, 128] table,
@@ -241,6 +287,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   int* csel = scratch + kScratchInts;                             // [kc]
   int* gpos = csel + ((kc + 3) & ~3);                             // [kg]
   uint32_t* keys = reinterpret_cast<uint32_t*>(gpos + ((kg + 3) & ~3));   // [max(nch, 8kc) rounded to 4]
+  const int nkeys4 = (((nch > 8 * kc) ? nch : 8 * kc) + 3) & ~3;
+  uint32_t* ckeys = keys + nkeys4;                                        // [kRouteThreads] candidates
+  int* cpos = reinterpret_cast<int*>(ckeys + kRouteThreads);              // [kRouteThreads]
 
   // ---- block query: mean over G heads x 64 positions of the routing block -- block n itself, or
   // for strictly causal routing block n-1 (block 0: the previous segment's last block q_prev
@@ -333,7 +382,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
     if (nc1 <= kRankSelectMax)
       block_select_topk_small(keys, nc1, kc, csel, scratch);
     else
-      block_select_topk(keys, nc1, kc, csel, hist, scratch);
+      block_select_topk_filtered(keys, nc1, kc, csel, hist, scratch, ckeys, cpos);
     if (nsc) {
       for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] += nsc;
       __syncthreads();
@@ -372,7 +421,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   if (ncand <= kRankSelectMax)
     block_select_topk_small(keys, ncand, kg, gpos, scratch);
   else
-    block_select_topk(keys, ncand, kg, gpos, hist, scratch);
+    block_select_topk_filtered(keys, ncand, kg, gpos, hist, scratch, ckeys, cpos);
 
   for (int i = threadIdx.x; i < kc; i += kRouteThreads) chunk_idx[(int64_t)unit * kc + i] = csel[i];
   for (int i = threadIdx.x; i < kg; i += kRouteThreads)
@@ -382,7 +431,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
 size_t route_smem_bytes(bool bf16, int nch, int kc, int kg) {
   const int RP = kRouteThreads / (kD / (bf16 ? 8 : 4));
   size_t words = (size_t)RP * kD + kD + 256 + kScratchInts + ((kc + 3) & ~3) + ((kg + 3) & ~3) +
-                 (size_t)(((nch > 8 * kc ? nch : 8 * kc) + 3) & ~3);
+                 (size_t)(((nch > 8 * kc ? nch : 8 * kc) + 3) & ~3) + 2 * kRouteThreads;
   return words * 4;
 }
 
@@ -439,25 +488,40 @@ cudaError_t launch_route_groups_cached(const float* qb, const int32_t* chunk_idx
 }
 
 // ---- chunk scores of all block queries of a (batch, KV head), for the three-launch routing
-constexpr int kScoreWarps = 8;
-constexpr int kScoreRowsPerWarp = 4;
+constexpr int kScoreWarps = 16;
+constexpr int kScoreRowsPerWarp = 2;   // rows a warp scores per round
+constexpr int kScoreRowsPerRound = kScoreWarps * kScoreRowsPerWarp;
 
-// Grid (B*Hkv, row slices).  Warp w of CTA (bkh, y) scores chunk rows nsc + i, i = (y * 8 + w) * 4 ..
-// + 3, against the block queries qb[bkh*nblk .. + nblk) (shared memory): lane l holds dims 4l .. 4l+3
-// of the row, multiplies them with the same dims of 32 block queries at a time, and a recursive-
-// halving exchange over the lanes leaves lane b with the full dot product of block b.  Writes the
-// order keys to scores[(bkh*nblk + blk) * nc_pad + i]; the pad entries [nc1, nc_pad) get 0, which
-// every score precedes.
-__global__ void __launch_bounds__(kScoreWarps * 32) chunk_score_kernel(const float* __restrict__ qb_all,
-                                                                      const float* __restrict__ chunk_sum,
-                                                                      uint32_t* __restrict__ scores, int nblk,
-                                                                      int nch_stride, int nsc, int nc1, int nc_pad) {
+// Grid (B*Hkv, row slices of `rounds` x 32 rows: one wave on the GPU).  In round t, warp w of CTA
+// (bkh, y) scores chunk rows nsc + i, i = y * 32 * rounds + 32 t + 2 w (+ 1), against the block queries
+// qb[bkh*nblk .. + nblk) (shared memory), the next round's rows already loading: lane l holds dims
+// 4l .. 4l+3 of a row and multiplies them with the same dims of 32 block queries at a time, and a
+// recursive-halving exchange over the lanes leaves lane b with the full dot product of block b.
+// Writes the order keys to scores[(bkh*nblk + blk) * nc_pad + i]; the pad entries [nc1, nc_pad) get
+// 0, which every score precedes.
+__global__ void __launch_bounds__(kScoreWarps * 32, 1) chunk_score_kernel(const float* __restrict__ qb_all,
+                                                                         const float* __restrict__ chunk_sum,
+                                                                         uint32_t* __restrict__ scores, int nblk,
+                                                                         int nch_stride, int nsc, int nc1, int nc_pad,
+                                                                         int rounds) {
   extern __shared__ __align__(16) float qs[];   // [nblk rounded up to 32][128]
   if (threadIdx.x == 0) pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t bkh = blockIdx.x;
   const int nb32 = (nblk + 31) & ~31;
+  const int base = (int)blockIdx.y * kScoreRowsPerRound * rounds + kScoreRowsPerWarp * warp;
+  const float* cs = chunk_sum + (bkh * nch_stride + nsc) * kD;
+  auto load_rows = [&](int t, float4(&rw)[kScoreRowsPerWarp]) {
+#pragma unroll
+    for (int r = 0; r < kScoreRowsPerWarp; ++r) {
+      const int i = base + kScoreRowsPerRound * t + r;
+      rw[r] = i < nc1 ? __ldg(reinterpret_cast<const float4*>(cs + (int64_t)i * kD) + lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
   pdl_wait();   // the block queries come from the kernel before, the summaries from the one before it
+  float4 cur[kScoreRowsPerWarp], nxt[kScoreRowsPerWarp];
+  load_rows(0, cur);
   {
     const float4* src = reinterpret_cast<const float4*>(qb_all + bkh * nblk * kD);
     float4* dst = reinterpret_cast<float4*>(qs);
@@ -465,45 +529,43 @@ __global__ void __launch_bounds__(kScoreWarps * 32) chunk_score_kernel(const flo
       dst[i] = i < nblk * (kD / 4) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
-  const int i0 = ((int)blockIdx.y * kScoreWarps + warp) * kScoreRowsPerWarp;
-  float4 row[kScoreRowsPerWarp];
-  const float* cs = chunk_sum + (bkh * nch_stride + nsc) * kD;
-#pragma unroll
-  for (int r = 0; r < kScoreRowsPerWarp; ++r)
-    row[r] = i0 + r < nc1 ? __ldg(reinterpret_cast<const float4*>(cs + (int64_t)(i0 + r) * kD) + lane)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
   uint32_t* out = scores + bkh * nblk * (int64_t)nc_pad;
-  for (int g = 0; g < nb32; g += 32) {
-    // each block query's 16 bytes are read once for the warp's four rows
-    float p[kScoreRowsPerWarp][32];
+  for (int t = 0; t < rounds; ++t) {
+    if (t + 1 < rounds) load_rows(t + 1, nxt);
+    for (int g = 0; g < nb32; g += 32) {
+      // each block query's 16 bytes are read once for the warp's rows
+      float p[kScoreRowsPerWarp][32];
 #pragma unroll
-    for (int b = 0; b < 32; ++b) {
-      const float4 q4 = reinterpret_cast<const float4*>(qs + (g + b) * kD)[lane];
+      for (int b = 0; b < 32; ++b) {
+        const float4 q4 = reinterpret_cast<const float4*>(qs + (g + b) * kD)[lane];
 #pragma unroll
-      for (int r = 0; r < kScoreRowsPerWarp; ++r)
-        p[r][b] = q4.x * row[r].x + q4.y * row[r].y + q4.z * row[r].z + q4.w * row[r].w;
-    }
+        for (int r = 0; r < kScoreRowsPerWarp; ++r)
+          p[r][b] = q4.x * cur[r].x + q4.y * cur[r].y + q4.z * cur[r].z + q4.w * cur[r].w;
+      }
 #pragma unroll
-    for (int r = 0; r < kScoreRowsPerWarp; ++r) {
-      // recursive halving: after the step with offset o, lane l keeps the o blocks whose index has
-      // bit log2(o) equal to that bit of l, summed over lane pairs l, l ^ o; at the end lane b holds
-      // block b's sum over all 32 lanes
+      for (int r = 0; r < kScoreRowsPerWarp; ++r) {
+        // recursive halving: after the step with offset o, lane l keeps the o blocks whose index has
+        // bit log2(o) equal to that bit of l, summed over lane pairs l, l ^ o; at the end lane b holds
+        // block b's sum over all 32 lanes
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const bool upper = (lane & o) != 0;
+        for (int o = 16; o > 0; o >>= 1) {
+          const bool upper = (lane & o) != 0;
 #pragma unroll
-        for (int k = 0; k < o; ++k) {
-          const float send = upper ? p[r][k] : p[r][k + o];
-          const float keep = upper ? p[r][k + o] : p[r][k];
-          p[r][k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          for (int k = 0; k < o; ++k) {
+            const float send = upper ? p[r][k] : p[r][k + o];
+            const float keep = upper ? p[r][k + o] : p[r][k];
+            p[r][k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+        }
+        const int i = base + kScoreRowsPerRound * t + r, blk = g + lane;
+        if (blk < nblk) {
+          if (i < nc1) out[(int64_t)blk * nc_pad + i] = order_key(p[r][0]);
+          else if (i < nc_pad) out[(int64_t)blk * nc_pad + i] = 0u;
         }
       }
-      const int i = i0 + r, blk = g + lane;
-      if (blk < nblk) {
-        if (i < nc1) out[(int64_t)blk * nc_pad + i] = order_key(p[r][0]);
-        else if (i < nc_pad) out[(int64_t)blk * nc_pad + i] = 0u;
-      }
     }
+#pragma unroll
+    for (int r = 0; r < kScoreRowsPerWarp; ++r) cur[r] = nxt[r];
   }
 }
 
@@ -542,24 +604,31 @@ cudaError_t launch_route_split(bool bf16, const void* q, const void* q_prev, boo
   RouteCache rc{qb, nullptr, nullptr, 0, nullptr, nullptr, 0};
   cudaError_t e = bf16 ? launch_route_t<__nv_bfloat16, kRouteQuery>(q, q_prev, causal, nullptr, nullptr, nullptr, nullptr, B, Hq,
                                                             Hkv, S, nch, nch_stride, nsc, kc, kg,
-                                                            route_smem_bytes(true, 1, 1, 1), rc, stream)
+                                                            route_smem_bytes(true, nch, kc, kg), rc, stream)
                        : launch_route_t<float, kRouteQuery>(q, q_prev, causal, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv,
                                                             S, nch, nch_stride, nsc, kc, kg,
-                                                            route_smem_bytes(false, 1, 1, 1), rc, stream);
+                                                            route_smem_bytes(false, nch, kc, kg), rc, stream);
   if (e != cudaSuccess) return e;
-  // 2. chunk scores
-  const int rows_per_cta = kScoreWarps * kScoreRowsPerWarp;
+  // 2. chunk scores: enough rounds per CTA that the grid is one wave
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int64_t total_rounds = (int64_t)B * Hkv * ((nc_pad + kScoreRowsPerRound - 1) / kScoreRowsPerRound);
+  const int rounds = (int)((total_rounds + sms - 1) / sms);
+  const int rows_per_cta = kScoreRowsPerRound * rounds;
   const dim3 grid((unsigned)(B * Hkv), (unsigned)((nc_pad + rows_per_cta - 1) / rows_per_cta));
   const size_t smem2 = (size_t)((nblk + 31) & ~31) * kD * sizeof(float);
   e = cudaFuncSetAttribute(chunk_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
   if (e != cudaSuccess) return e;
   e = launch_dependent(chunk_score_kernel, grid, dim3(kScoreWarps * 32), smem2, stream, 1,
-                       static_cast<const float*>(qb), chunk_sum, scores, (int)nblk, nch_stride, nsc, nc1, nc_pad);
+                       static_cast<const float*>(qb), chunk_sum, scores, (int)nblk, nch_stride, nsc, nc1, nc_pad,
+                       rounds);
   if (e != cudaSuccess) return e;
   // 3. selection from the scores, then level 2
   rc.scores = scores;
   rc.nc_pad = nc_pad;
-  const size_t smem3 = route_smem_bytes(bf16, nc_pad, kc, kg);
+  // the kernel lays its shared memory out from nch (>= nc_pad: nch = nsc + nc1, nc_pad = nc1 rounded up to 4)
+  const size_t smem3 = route_smem_bytes(bf16, nch, kc, kg);
   return bf16 ? launch_route_t<__nv_bfloat16, kRouteFromScores>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B,
                                                         Hq, Hkv, S, nch, nch_stride, nsc, kc, kg, smem3, rc, stream)
               : launch_route_t<float, kRouteFromScores>(q, q_prev, causal, group_sum, chunk_sum, chunk_idx, group_idx, B, Hq,

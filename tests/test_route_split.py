@@ -73,3 +73,22 @@ def test_split_ragged_matches_oracle(hga, oracle):
     assert np.array_equal(r32["group_idx"], r64["group_idx"]) and np.array_equal(r32["chunk_idx"], r64["chunk_idx"])
     assert r64["chunk_gap"].min() >= 4e-6 and r64["group_gap"].min() >= 4e-6
     assert np.array_equal(ci_s, r32["chunk_idx"]) and np.array_equal(gi_s, r32["group_idx"])
+
+
+@pytest.mark.parametrize("fill", [0.25, 0.0])
+def test_large_selection_ties_go_to_lower_index(hga, fill):
+    """All history keys equal, so every score ties: 600 routable chunks (more candidates than a CTA
+    has threads, so the filtered selection falls back to the radix select) and 320 candidate groups
+    (filtered, then ranked): the lowest indices are selected, by the three launches and by one."""
+    w = HI.Workload("split_ties", 1, 4, 2, 128, 64 * 600, 128, 40, 300, "bf16", 0.5)
+    x = HI.make_inputs(w, 0)
+    q = x["q"].cuda()
+    kh = torch.full_like(x["k_hist"], fill).cuda()
+    cfg = hga.make_config(q, kh, w.top_chunks, w.top_groups)
+    ws = hga.new_workspace(cfg, q.device)
+    gs, cs = hga.build_summaries(cfg, kh, workspace=ws)
+    for workspace in (ws, None):
+        ci, gi = hga.route(cfg, q, gs, cs, workspace=workspace)
+        torch.cuda.synchronize()
+        assert (ci.cpu() == torch.arange(w.top_chunks, dtype=torch.int32)).all()
+        assert (gi.cpu() == torch.arange(w.top_groups, dtype=torch.int32)).all()
