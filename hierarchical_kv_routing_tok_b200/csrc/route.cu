@@ -7,8 +7,9 @@
 // One CTA per (batch, KV head, 64-query block).  The block query (mean over
 // the block's positions and the KV head's query heads) stays in shared memory,
 // scores are warp dot products against float32 summaries (L2-resident), and
-// the top-k is exact: a one-pass rank selection when a level has at most 256
-// candidates, else a CTA-wide radix select on order-preserving 32-bit keys; both
+// the top-k is exact: a one-pass rank selection, a CTA-wide radix select on
+// order-preserving 32-bit keys, or a threshold filter followed by the rank
+// selection of the keys that pass it, whichever is cheapest for the level's size; all
 // finish with an index-ordered compaction, so ties go to the lower index and the
 // output comes out sorted ascending.  This is not a dense contraction
 // (M = 1 per CTA), so it runs on the CUDA cores.
@@ -28,10 +29,14 @@
 namespace hga {
 
 constexpr int kRouteThreads = 512;
-// Candidates up to which a level selects by rank counting (n^2 / threads comparisons per thread);
-// above it the radix select (four 8-bit passes) is cheaper: routing 384 chunks took 24.6 us with
-// the radix select against 30.7 with rank counting (B200, one launch, summaries not in L2).
+// Choice of exact top-k for n candidates (cycles of one CTA of 512 threads, two CTAs per SM, B200):
+// rank counting grows as n^2 (n = 128: 2.9K, 224: 6.5K, 256: 7.3K, 512: 24.5K), the radix select is
+// flat (6.8K-7.3K up to n = 512, 9.7K at 2016), the threshold filter pays when few keys pass it
+// (k <= n / 8: n = 224, k = 16: 4.7K; n = 2016, k = 32: 8.4K) and not otherwise (n = 256, k = 128:
+// 18.8K).
 constexpr int kRankSelectMax = 256;
+__device__ __forceinline__ void block_select_topk_any(const uint32_t* keys, int n, int k, int* out, int* hist,
+                                                      int* scratch, uint32_t* ckeys, int* cpos);
 constexpr int kScratchInts = 32;   // warp totals (16) + broadcast slots
 
 // Larger score -> larger key; +0 and -0 map to the same key.
@@ -221,6 +226,18 @@ __device__ void block_select_topk_filtered(const uint32_t* keys, int n, int k, i
   block_select_topk_small(ckeys, tot, k, out, scratch, cpos);
 }
 
+__device__ __forceinline__ void block_select_topk_any(const uint32_t* keys, int n, int k, int* out, int* hist,
+                                                      int* scratch, uint32_t* ckeys, int* cpos) {
+  if (n <= 128)
+    block_select_topk_small(keys, n, k, out, scratch);
+  else if (8 * k <= n)
+    block_select_topk_filtered(keys, n, k, out, hist, scratch, ckeys, cpos);
+  else if (n <= kRankSelectMax)
+    block_select_topk_small(keys, n, k, out, scratch);
+  else
+    block_select_topk(keys, n, k, out, hist, scratch);
+}
+
 // Dot products of qb (smem, 128 floats) with `count` rows of a float32 [*, 128] table,
 // row ids given by row_of(i); one warp per row, 8 rows in flight per warp.
 template <typename RowOf>
@@ -379,10 +396,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
       if (threadIdx.x < 4 && nc1 + (int)threadIdx.x < ((nc1 + 3) & ~3)) keys[nc1 + threadIdx.x] = 0u;
       __syncthreads();
     }
-    if (nc1 <= kRankSelectMax)
-      block_select_topk_small(keys, nc1, kc, csel, scratch);
-    else
-      block_select_topk_filtered(keys, nc1, kc, csel, hist, scratch, ckeys, cpos);
+    block_select_topk_any(keys, nc1, kc, csel, hist, scratch, ckeys, cpos);
     if (nsc) {
       for (int i = threadIdx.x; i < kc; i += kRouteThreads) csel[i] += nsc;
       __syncthreads();
@@ -418,10 +432,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(
   }
   if (threadIdx.x < 4 && ncand + (int)threadIdx.x < ((ncand + 3) & ~3)) keys[ncand + threadIdx.x] = 0u;
   __syncthreads();
-  if (ncand <= kRankSelectMax)
-    block_select_topk_small(keys, ncand, kg, gpos, scratch);
-  else
-    block_select_topk_filtered(keys, ncand, kg, gpos, hist, scratch, ckeys, cpos);
+  block_select_topk_any(keys, ncand, kg, gpos, hist, scratch, ckeys, cpos);
 
   for (int i = threadIdx.x; i < kc; i += kRouteThreads) chunk_idx[(int64_t)unit * kc + i] = csel[i];
   for (int i = threadIdx.x; i < kg; i += kRouteThreads)

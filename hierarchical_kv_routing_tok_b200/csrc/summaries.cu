@@ -34,9 +34,16 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k_
   const int col = (lane % LPR) * N;
   const int rsub = lane / LPR;
   const T* base = k_hist + (bkh * Hs + c * kChunk + (int64_t)g * kGroup + rsub) * kD + col;
+  // streaming loads (evict first): the history is read once here, and its lines would otherwise push
+  // the summaries this kernel writes, which the router reads next, out of L2 (131K: 47 against 51 us)
   float v[LOADS][N];
+  {
+    uint4 raw[LOADS];
 #pragma unroll
-  for (int i = 0; i < LOADS; ++i) Vec16<T>::load(base + (int64_t)i * RPL * kD, v[i]);
+    for (int i = 0; i < LOADS; ++i) raw[i] = __ldcs(reinterpret_cast<const uint4*>(base + (int64_t)i * RPL * kD));
+#pragma unroll
+    for (int i = 0; i < LOADS; ++i) Vec16<T>::load(reinterpret_cast<const T*>(&raw[i]), v[i]);
+  }
   float acc[N];
 #pragma unroll
   for (int e = 0; e < N; ++e) {
