@@ -199,13 +199,14 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_layer_pass(w, x, workers: int, n_slices: int | None = None) -> float:
+def oracle_layer_pass(w, x, workers: int, n_slices: int | None = None, stages: dict | None = None) -> float:
     """The CPU oracle, as it stands, over the first n_slices (batch, KV head) slices of the layer
-    (all of them by default), on `workers` host threads: summaries and float32-decision routing per
-    slice, then the float64 forward and dQ of every (slice, 64-query block) unit and the dK/dV of
-    every slice, all as concurrent tasks (the oracle's C calls release the GIL).  A slice -- its G
-    query heads with their history, segment K/V and routing -- is independent of every other slice.
-    Returns seconds (wall clock)."""
+    (all of them by default), on `workers` host threads, in three phases of concurrent tasks (the
+    oracle's C calls release the GIL): summaries and float32-decision routing per slice; the
+    float64 forward of every (slice, 64-query block) unit; the dK/dV of every slice and the dQ of
+    every unit.  A slice -- its G query heads with their history, segment K/V and routing -- is
+    independent of every other slice.  Returns seconds (wall clock); `stages`, when given, receives
+    each phase's seconds."""
     import concurrent.futures as cf
 
     import numpy as np
@@ -226,25 +227,38 @@ def oracle_layer_pass(w, x, workers: int, n_slices: int | None = None) -> float:
             (q, kh_, *_), _ = sl(b, kh)
             return O.route_from_inputs(q, kh_, 1, w.top_chunks, w.top_groups, prec=32)["group_idx"]
         gi = dict(zip(slices, ex.map(lambda j: route(*j), slices)))
-        tasks = []
+        t1 = time.perf_counter()
+        block_rows = [np.array([hh * S + n * 64 + t for hh in range(G) for t in range(64)], dtype=np.int64)
+                      for n in range(nblk)]
+        fwd = []
+        for b, kh in slices:
+            args, _ = sl(b, kh)
+            for rows in block_rows:               # forward of the block's G x 64 rows
+                fwd.append(ex.submit(O.attn_fwd, *args, gi[(b, kh)], rows=rows))
+        for t in fwd:
+            t.result()
+        t2 = time.perf_counter()
+        bwd = []
         for b, kh in slices:                     # dK/dV of a slice: the longest tasks, queued first
             args, do = sl(b, kh)
-            tasks.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=np.array([0]),
-                                   keys=np.arange(S)))
+            bwd.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=np.array([0]),
+                                 keys=np.arange(S)))
         for b, kh in slices:
             args, do = sl(b, kh)
-            for n in range(nblk):                # forward and dQ of the block's G x 64 rows
-                rows = np.array([hh * S + n * 64 + t for hh in range(G) for t in range(64)], dtype=np.int64)
-                tasks.append(ex.submit(O.attn_fwd, *args, gi[(b, kh)], rows=rows))
-                tasks.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=rows, keys=np.array([S - 1])))
-        for t in tasks:
+            for rows in block_rows:               # dQ of the block's G x 64 rows
+                bwd.append(ex.submit(O.attn_bwd, *args, gi[(b, kh)], do, rows=rows, keys=np.array([S - 1])))
+        for t in bwd:
             t.result()
-    return time.perf_counter() - t0
+        t3 = time.perf_counter()
+    if stages is not None:
+        stages.update(summaries_and_route_s=t1 - t0, fwd_s=t2 - t1, bwd_s=t3 - t2)
+    return t3 - t0
 
 
-ORACLE_SAMPLE = ("the CPU oracle as it stands (plain C, float32-decision routing, float64 attention) over {what}: "
-                 "summaries and routing per (batch, KV head), forward and dQ per (batch, KV head, 64-query block) "
-                 "unit, dK/dV per (batch, KV head), as concurrent tasks on {workers} host threads; wall clock")
+ORACLE_SAMPLE = ("the CPU oracle as it stands (plain C, float32-decision routing, float64 attention) over {what}, "
+                 "in three phases of concurrent tasks on {workers} host threads: summaries and routing per (batch, "
+                 "KV head); forward per (batch, KV head, 64-query block) unit; dK/dV per (batch, KV head) and dQ per "
+                 "unit; wall clock")
 
 
 def _oracle_baseline(w, x, warm: bool = True) -> dict:
@@ -257,12 +271,13 @@ def _oracle_baseline(w, x, warm: bool = True) -> dict:
         t1 = oracle_layer_pass(w, x, workers, n)
         if t1 > 8.0:
             n = max(1, min(total, int(total * 8.0 / t1)))
-    t = oracle_layer_pass(w, x, workers, n)
+    stages = {}
+    t = oracle_layer_pass(w, x, workers, n, stages)
     what = "the whole layer" if n == total else f"{n} of the layer's {total} (batch, KV head) slices"
     tokens = w.B * w.seg_len * n / total
     return {"value": tokens / t, "unit": "tokens/s", "cores": workers,
             "kind": "oracle", "sample": ORACLE_SAMPLE.format(what=what, workers=workers), "seconds": t,
-            "slices": n, "host_cores": workers}
+            "stages_seconds": {k: round(v, 3) for k, v in stages.items()}, "slices": n, "host_cores": workers}
 
 
 def run_reference(args, w, world, rank):
