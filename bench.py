@@ -48,6 +48,9 @@ def _peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
+NOMINAL_HBM_GBS = 8000.0   # the B200 datasheet figure, for context next to the measured copy rate
+
+
 def work_model(w) -> dict:
     """Algorithmic work of each kernel of one step (bytes or flops per launch).
 
@@ -637,6 +640,9 @@ def main():
                                         / ((pk["bf16"] * 1e12) if wm[n][0] == "tensor" else (pk["hbm"] * 1e9)))
                                     for n in names},
                 "per_kernel_executed_frac": {n: ex[n] / (per_us[n] * 1e-6) / (pk["bf16"] * 1e12) for n in ex},
+                # the memory-bound kernels also against the nominal 8 TB/s of the part
+                "per_kernel_frac_nominal_hbm": {n: wm[n][1] / (per_us[n] * 1e-6) / (NOMINAL_HBM_GBS * 1e9)
+                                                for n in names if wm[n][0] == "hbm"},
                 "work_booking": "backward at the method's work: S, dP, dQ over routed + local pairs charged to "
                                 "bwd_dq, dK and dV over local pairs to bwd_dkdv (its S^T, dP^T recomputation "
                                 "is in per_kernel_executed_frac only)"}
