@@ -92,3 +92,28 @@ def test_large_selection_ties_go_to_lower_index(hga, fill):
         torch.cuda.synchronize()
         assert (ci.cpu() == torch.arange(w.top_chunks, dtype=torch.int32)).all()
         assert (gi.cpu() == torch.arange(w.top_groups, dtype=torch.int32)).all()
+
+
+def test_layer_step_with_split_routing_and_paired_dkdv_matches_oracle(hga, oracle):
+    """A whole layer step (summaries, three-launch routing, forward, backward) on one workspace whose
+    region after the delta rows serves first as the routing scratch and then as the dK/dV exchange
+    area (4 key tiles x 2 KV heads = 8 units, so the dK/dV kernel pairs CTAs): routing bit-exact,
+    outputs and gradients within the bf16 bars of the oracle."""
+    w = HI.Workload("split_step", 1, 8, 2, 128, 64 * 520, 512, 8, 32, "bf16", 0.5)
+    x = HI.make_inputs(w, 0)
+    xd = {k: v.cuda() for k, v in x.items() if k != "needles"}
+    cfg = hga.make_config(xd["q"], xd["k_hist"], w.top_chunks, w.top_groups)
+    assert hga._capi.route_launches(cfg) == 3
+    step = hga.LayerStep(cfg)
+    step(xd)
+    torch.cuda.synchronize()
+    assert hga.read_status(step.ws) == hga._capi.HGA_OK
+    r = oracle.route_from_inputs(x["q"], x["k_hist"], w.Hkv, w.top_chunks, w.top_groups, prec=32)
+    assert np.array_equal(step.chunk_idx.cpu().numpy(), r["chunk_idx"])
+    assert np.array_equal(step.group_idx.cpu().numpy(), r["group_idx"])
+    args = (x["q"], x["k_hist"], x["v_hist"], x["k_seg"], x["v_seg"], r["group_idx"])
+    o, lse = oracle.attn_fwd(*args)
+    dq, dk, dv = oracle.attn_bwd(*args, x["d_o"])
+    err = lambda a, b: float(np.abs(a.float().cpu().numpy() - b).max())
+    assert max(err(step.o, o), err(step.dq, dq), err(step.dk, dk), err(step.dv, dv)) <= 2e-2
+    assert err(step.lse, lse) <= 1e-3
