@@ -113,6 +113,7 @@ def test_route_launches(lib):
     # the 400 block queries of a 25,600-token segment would need 208 KB of shared memory
     assert C.route_launches(cfg(seg_len=64 * 400, **long)) == 1
     assert C.route_launches(cfg(seg_len=64 * 384, **long)) == 3
+    assert C.route_launches(cfg(hist_len=0, top_chunks=0, top_groups=0)) == 0   # first segment: no history
 
 
 @pytest.mark.parametrize("kw,code", [
